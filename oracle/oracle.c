@@ -1,0 +1,276 @@
+/*
+ * CPU oracle for exact scaled-dot-product attention.  TEST INFRASTRUCTURE ONLY:
+ * only the tests, the smoke check and the benchmark's CPU-baseline leg load
+ * this code.  It shares nothing with the CUDA library.
+ *
+ * What it computes (plain definition, fp64 throughout):
+ *
+ *   O = softmax(scale * Q K^T [+ causal mask]) V,   lse = log(sum_j e^{s_j})
+ *
+ * following the standard three-step statement of attention (Gemini 3 Flash
+ * kernel-fusion post, "traditional attention": S = QK^T, P = softmax(S),
+ * O = PV; GPU-optimisation tag page, "algorithm principle": S = Q K^T / sqrt(d))
+ * and the three-sweep softmax of the FlashAttention optimisation article
+ * (section 2.2: one sweep for the row max, one for exp(x - max) and its sum,
+ * one to normalise).
+ *
+ * Readings where the pages are silent (each listed in the design notes):
+ *  - causal masking is aligned bottom-right: key j is visible to query i iff
+ *    j <= i + (Nkv - Nq); with Nq == Nkv that is the usual j <= i;
+ *  - a row with no visible key returns O = 0 and lse = -inf;
+ *  - lse is the natural log of the scaled scores' normaliser: m + ln(l);
+ *  - query head hq reads KV head hq / (Hq / Hkv) (consecutive heads share one
+ *    KV head, GPU-optimisation tag page, GQA section);
+ *  - the paged cache is [num_pages_total, Hkv, page_size, d]; logical token t
+ *    of sequence s lives at page block_table[s][t / page_size], row
+ *    t % page_size (paged-gather article, section 2.1/2.3: a per-sequence list
+ *    of physical blocks); table entries beyond the sequence are never read.
+ *
+ * All bf16 inputs are passed as uint16 bit patterns and widened exactly.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_TABLE 4
+#define ORACLE_ERR_NOMEM 6
+
+static double bf16_to_f64(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/*
+ * One query row against n keys/values (rows of length d, row stride d).
+ * s is scratch of length n.  Writes o[0..d) and *lse.
+ * visible = number of leading keys the query may see (keys >= visible are
+ * masked to -inf explicitly before the softmax).
+ */
+static void attend_row(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       int n, int d, double scale, int visible,
+                       double *s, double *o, double *lse)
+{
+    /* scores, with the mask written out explicitly */
+    for (int j = 0; j < n; ++j) {
+        if (j >= visible) {
+            s[j] = -INFINITY;
+            continue;
+        }
+        double acc = 0.0;
+        const uint16_t *kj = k + (size_t)j * d;
+        for (int t = 0; t < d; ++t)
+            acc += bf16_to_f64(q[t]) * bf16_to_f64(kj[t]);
+        s[j] = scale * acc;
+    }
+    /* sweep 1: row maximum */
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j)
+        if (s[j] > m)
+            m = s[j];
+    for (int t = 0; t < d; ++t)
+        o[t] = 0.0;
+    if (m == -INFINITY) {       /* no visible key */
+        *lse = -INFINITY;
+        return;
+    }
+    /* sweep 2: normaliser */
+    double l = 0.0;
+    for (int j = 0; j < n; ++j)
+        if (s[j] != -INFINITY)
+            l += exp(s[j] - m);
+    /* sweep 3: normalised weights times V */
+    for (int j = 0; j < n; ++j) {
+        if (s[j] == -INFINITY)
+            continue;
+        double p = exp(s[j] - m) / l;
+        const uint16_t *vj = v + (size_t)j * d;
+        for (int t = 0; t < d; ++t)
+            o[t] += p * bf16_to_f64(vj[t]);
+    }
+    *lse = m + log(l);
+}
+
+static int visible_keys(int i, int Nq, int Nkv, int causal)
+{
+    if (!causal)
+        return Nkv;
+    long lim = (long)i + (long)(Nkv - Nq) + 1;
+    if (lim < 0)
+        lim = 0;
+    if (lim > Nkv)
+        lim = Nkv;
+    return (int)lim;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/*
+ * Contiguous attention.  q [B,Hq,Nq,d], k/v [B,Hkv,Nkv,d] (bf16 bits).
+ * rows: optional list of flat row ids r = (b*Hq + hq)*Nq + i to evaluate;
+ * if rows == NULL every row is evaluated in order.  o is [nrows, d] fp64,
+ * lse is [nrows] fp64 (may be NULL).
+ */
+int oracle_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                double scale, int causal, const int64_t *rows, int64_t nrows,
+                double *o, double *lse)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nkv < 0 || d <= 0 || Hq % Hkv)
+        return ORACLE_ERR_ARG;
+    const int64_t total = (int64_t)B * Hq * Nq;
+    if (!rows)
+        nrows = total;
+    const int G = Hq / Hkv;
+    int err = ORACLE_OK;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Nkv > 0 ? Nkv : 1));
+        if (!s) {
+#pragma omp atomic write
+            err = ORACLE_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < nrows; ++r) {
+            if (!s)
+                continue;
+            int64_t id = rows ? rows[r] : r;
+            if (id < 0 || id >= total) {
+#pragma omp atomic write
+                err = ORACLE_ERR_ARG;
+                continue;
+            }
+            int i = (int)(id % Nq);
+            int64_t bh = id / Nq;
+            int hq = (int)(bh % Hq);
+            int b = (int)(bh / Hq);
+            int hkv = hq / G;
+            const uint16_t *qi = q + (size_t)id * d;
+            const uint16_t *kb = k + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
+            const uint16_t *vb = v + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
+            double l;
+            attend_row(qi, kb, vb, Nkv, d, scale, visible_keys(i, Nq, Nkv, causal),
+                       s, o + (size_t)r * d, &l);
+            if (lse)
+                lse[r] = l;
+        }
+        free(s);
+    }
+    return err;
+}
+
+/*
+ * Explicit gather of one sequence's logical K and V rows for KV head hkv:
+ * k_out/v_out [seq_len, d] (bf16 bits) = cache[block_table[seq][t/ps], hkv, t%ps, :].
+ * Returns ORACLE_ERR_TABLE if a needed table entry is outside [0, num_pages_total)
+ * or the length does not fit in max_pages pages.
+ */
+int oracle_paged_gather(const uint16_t *k_cache, const uint16_t *v_cache,
+                        const int32_t *block_table, const int32_t *seq_lens,
+                        int seq, int hkv, int page_size, int Hkv, int d,
+                        int max_pages, int64_t num_pages_total,
+                        uint16_t *k_out, uint16_t *v_out)
+{
+    if (page_size <= 0 || Hkv <= 0 || d <= 0 || hkv < 0 || hkv >= Hkv || seq < 0)
+        return ORACLE_ERR_ARG;
+    int len = seq_lens[seq];
+    if (len < 0 || (int64_t)len > (int64_t)max_pages * page_size)
+        return ORACLE_ERR_TABLE;
+    for (int t = 0; t < len; ++t) {
+        int32_t page = block_table[(size_t)seq * max_pages + t / page_size];
+        if (page < 0 || page >= num_pages_total)
+            return ORACLE_ERR_TABLE;
+        size_t src = (((size_t)page * Hkv + hkv) * page_size + (size_t)(t % page_size)) * d;
+        memcpy(k_out + (size_t)t * d, k_cache + src, sizeof(uint16_t) * (size_t)d);
+        memcpy(v_out + (size_t)t * d, v_cache + src, sizeof(uint16_t) * (size_t)d);
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Paged decode: one query token per sequence attends all seq_lens[s] keys of
+ * its sequence (no mask).  q/o [num_seqs, Hq, d], lse [num_seqs, Hq].
+ * seqs: optional list of sequences to evaluate (o/lse rows follow that list).
+ */
+int oracle_paged_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                        const int32_t *block_table, const int32_t *seq_lens,
+                        int page_size, int num_seqs, int Hq, int Hkv, int d,
+                        int max_pages, int64_t num_pages_total, double scale,
+                        const int32_t *seqs, int nseqs, double *o, double *lse)
+{
+    if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv || page_size <= 0)
+        return ORACLE_ERR_ARG;
+    if (!seqs)
+        nseqs = num_seqs;
+    const int G = Hq / Hkv;
+    int err = ORACLE_OK;
+    const int64_t items = (int64_t)nseqs * Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t it = 0; it < items; ++it) {
+        int si = (int)(it / Hkv), hkv = (int)(it % Hkv);
+        int s = seqs ? seqs[si] : si;
+        if (s < 0 || s >= num_seqs) {
+#pragma omp atomic write
+            err = ORACLE_ERR_ARG;
+            continue;
+        }
+        int len = seq_lens[s];
+        if (len < 0)
+            len = 0;
+        size_t n = (size_t)(len > 0 ? len : 1);
+        uint16_t *kg = (uint16_t *)malloc(sizeof(uint16_t) * n * d);
+        uint16_t *vg = (uint16_t *)malloc(sizeof(uint16_t) * n * d);
+        double *sc = (double *)malloc(sizeof(double) * n);
+        if (!kg || !vg || !sc) {
+#pragma omp atomic write
+            err = ORACLE_ERR_NOMEM;
+        } else {
+            int e = oracle_paged_gather(k_cache, v_cache, block_table, seq_lens, s, hkv,
+                                        page_size, Hkv, d, max_pages, num_pages_total, kg, vg);
+            if (e) {
+#pragma omp atomic write
+                err = e;
+            } else {
+                for (int g = 0; g < G; ++g) {
+                    int hq = hkv * G + g;
+                    size_t row = (size_t)si * Hq + hq;
+                    double l;
+                    attend_row(q + ((size_t)s * Hq + hq) * d, kg, vg, len, d, scale, len,
+                               sc, o + row * d, &l);
+                    if (lse)
+                        lse[row] = l;
+                }
+            }
+        }
+        free(kg);
+        free(vg);
+        free(sc);
+    }
+    return err;
+}

@@ -1,0 +1,48 @@
+"""Plant plausible mistakes in a copy of oracle.c and check that the pins
+catch every one of them (CPU only; the planted copies never leave a temp dir)."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import oracle_pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTANTS = {
+    "dropped_scale": ("s[j] = scale * acc;", "s[j] = acc;"),
+    "causal_off_by_one": ("(long)(Nkv - Nq) + 1;", "(long)(Nkv - Nq);"),
+    "alignment_sign": ("(long)(Nkv - Nq) + 1;", "(long)(Nq - Nkv) + 1;"),
+    "no_normalisation": ("double p = exp(s[j] - m) / l;", "double p = exp(s[j] - m);"),
+    "wrong_exp_sign": ("double p = exp(s[j] - m) / l;", "double p = exp(m - s[j]) / l;"),
+    "lse_without_log": ("*lse = m + log(l);", "*lse = m;"),
+    "lse_log2": ("*lse = m + log(l);", "*lse = m + log2(l);"),
+    "gqa_mapping": ("int hkv = hq / G;", "int hkv = hq % Hkv;"),
+    "reversed_feature": ("bf16_to_f64(kj[t]);", "bf16_to_f64(kj[d - 1 - t]);"),
+    "v_row_index": ("const uint16_t *vj = v + (size_t)j * d;", "const uint16_t *vj = v + (size_t)(n - 1 - j) * d;"),
+    "page_row_index": ("(size_t)(t % page_size)) * d;", "(size_t)(t / page_size)) * d;"),
+    "sum_without_max": ("l += exp(s[j] - m);", "l += exp(s[j]);"),
+    "decode_head_mapping": ("int hq = hkv * G + g;", "int hq = g * Hkv + hkv;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    mutated = src.replace(old, new, 1)
+    c = tmp_path / "mutant.c"
+    c.write_text(mutated)
+    so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", str(so), str(c), "-lm"],
+                   check=True)
+    variant = oracle.Variant(str(so))
+    failed = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(variant)
+        except (AssertionError, RuntimeError, FloatingPointError, ValueError) as e:
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught mutant {name}"
