@@ -1,0 +1,168 @@
+/*
+ * tiledattn.h - C ABI of the B200 fused tiled-attention library (libtiledattn.so).
+ *
+ * The library computes exact scaled-dot-product attention
+ *
+ *     O = softmax(scale * Q K^T [+ causal mask]) V
+ *
+ * in one fused, tiled pass (online softmax: running row max m and sum l,
+ * rescaling of the partial output on every new K/V tile), so the N x N score
+ * and probability matrices never reach HBM.  Problem statement: Gemini 3 Flash
+ * kernel-fusion post, sections "traditional attention" (S = QK^T, P = softmax(S),
+ * O = PV) and 1-3 (fusion, tiling, online softmax); FlashAttention optimisation
+ * article, sections 2.1 and 3.1-3.2.
+ *
+ * Conventions shared by every call
+ *  - All Q/K/V/O arrays are bfloat16, dense, row-major, with 16-byte aligned
+ *    base pointers (128-byte alignment recommended; FlashAttention article 5.2,
+ *    kernel-fusion post "data layout").  lse arrays are float32.
+ *  - Pointers are DEVICE pointers unless stated otherwise.  The caller owns
+ *    every buffer and the stream.  No call allocates memory or synchronises;
+ *    work is enqueued on `stream` and the call returns.
+ *  - Argument errors are detected on the host before anything is enqueued and
+ *    return TA_ERR_INVALID_ARG or TA_ERR_UNSUPPORTED.  A failed launch returns
+ *    TA_ERR_CUDA.  Faults found on the device (a block-table entry outside the
+ *    pool, a bounded wait that gave up) never trap: the kernel clamps or skips,
+ *    records a bit in a device status word, and the caller may read that word
+ *    with attn_paged_decode_check() / ta_device_status().
+ *  - Grouped-query attention: query head hq reads KV head hq / (Hq / Hkv), i.e.
+ *    consecutive query heads share a KV head (GPU-optimisation tag page, GQA).
+ *  - Causal masking is aligned to the bottom-right corner: query i sees keys
+ *    j <= i + (Nkv - Nq).  A query with no visible key gets O = 0, lse = -inf.
+ *  - lse (optional, may be NULL) is the natural log of the softmax normaliser
+ *    of the scaled scores: lse = m + ln(sum_j exp(s_j - m)).  It is the per-row
+ *    max and normaliser the kernel-fusion post (section 4) keeps for a
+ *    recomputing backward pass.
+ */
+#ifndef TILEDATTN_H
+#define TILEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without requiring the CUDA headers; NULL = legacy default stream. */
+typedef struct CUstream_st *ta_stream_t;
+
+typedef enum {
+    TA_OK = 0,
+    TA_ERR_INVALID_ARG = 1,     /* bad pointer, shape, alignment or size */
+    TA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (head dim, page size, ...) */
+    TA_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed */
+    TA_ERR_BAD_BLOCK_TABLE = 4, /* a block-table entry or length was out of range */
+    TA_ERR_DEVICE_TIMEOUT = 5   /* a bounded device-side wait gave up */
+} ta_status;
+
+/* Bits of the device status word. */
+#define TA_DEV_TIMEOUT 1u
+#define TA_DEV_BAD_BLOCK_TABLE 2u
+#define TA_DEV_BAD_SEQ_LEN 4u
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *ta_status_string(ta_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int ta_version(void);
+
+/*
+ * attn_fwd - fused attention forward (prefill).
+ *
+ *   q   [B, Hq,  Nq,  d]  bf16     o   [B, Hq, Nq, d] bf16 (written)
+ *   k   [B, Hkv, Nkv, d]  bf16     lse [B, Hq, Nq]    fp32 (written; may be NULL)
+ *   v   [B, Hkv, Nkv, d]  bf16
+ *
+ * scale: multiplier of the scores (1/sqrt(d) in the pages' statement,
+ * GPU-optimisation tag page "algorithm principle"); must be finite and >= 0.
+ * causal: 0 or 1.  Supported: d in {64, 128}, Hq % Hkv == 0, all sizes >= 0
+ * (B*Hq*Nq == 0 does nothing; Nkv == 0 writes O = 0, lse = -inf).
+ * o must not overlap q, k or v.
+ */
+ta_status attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                   int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                   float scale, int causal, ta_stream_t stream);
+
+/*
+ * Bytes of device workspace attn_paged_decode needs for these sizes (256-byte
+ * aligned).  Pure host arithmetic; returns 0 for invalid sizes.
+ */
+size_t attn_paged_decode_workspace_size(int num_seqs, int Hq, int Hkv, int d,
+                                        int max_pages, int page_size);
+
+/*
+ * attn_paged_decode - one query token per sequence against a paged KV cache
+ * (PagedAttention-style pool: GPU-optimisation tag page, "PagedAttention";
+ * block gather fused with the dot products and the weighted sum of V: paged
+ * gather article, sections 2.1-2.4).
+ *
+ *   q, o         [num_seqs, Hq, d] bf16
+ *   lse          [num_seqs, Hq]    fp32 (may be NULL)
+ *   k_cache,
+ *   v_cache      [num_pages_total, Hkv, page_size, d] bf16
+ *   block_table  [num_seqs, max_pages] int32: logical page t of sequence s is
+ *                physical page block_table[s][t]; entries past the last page
+ *                of a sequence are ignored
+ *   seq_lens     [num_seqs] int32, 0 <= len <= max_pages * page_size; token t
+ *                of sequence s is row t % page_size of page
+ *                block_table[s][t / page_size].  A sequence of length 0 gets
+ *                O = 0, lse = -inf.
+ *   workspace    >= attn_paged_decode_workspace_size(...) bytes, 256-byte
+ *                aligned; holds split partials and the status word.  Must not
+ *                be shared by calls that may run concurrently.
+ *
+ * Supported: d in {64, 128}, page_size in {8, 16, 32, 64}, Hq % Hkv == 0,
+ * Hq / Hkv in {1, 2, 4, 8}.  Table entries outside [0, num_pages_total) and
+ * lengths outside [0, max_pages * page_size] are clamped on the device (never
+ * dereferenced) and flagged in the status word; see attn_paged_decode_check.
+ */
+ta_status attn_paged_decode(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *block_table, const int32_t *seq_lens, int page_size,
+                            int num_seqs, int Hq, int Hkv, int d, int max_pages,
+                            int num_pages_total, float scale, void *o, float *lse,
+                            void *workspace, size_t workspace_bytes, ta_stream_t stream);
+
+/*
+ * Checked mode for paged decode: waits for `stream`, reads the status word the
+ * last attn_paged_decode wrote into `workspace`, stores it in *flags (host
+ * pointer, may be NULL) and returns TA_ERR_BAD_BLOCK_TABLE or
+ * TA_ERR_DEVICE_TIMEOUT if a bit is set, else TA_OK.  Synchronises the stream.
+ */
+ta_status attn_paged_decode_check(const void *workspace, unsigned *flags, ta_stream_t stream);
+
+/*
+ * Test/diagnostic export: writes the logical K and V rows of (seq, hkv),
+ * gathered through the block table by the same device gather routine that
+ * attn_paged_decode uses, to k_out/v_out [max_pages * page_size, d] bf16
+ * (rows >= seq_lens[seq] are left untouched).  Same layouts and limits as
+ * attn_paged_decode; bad entries are clamped and flagged in the library status
+ * word (ta_device_status).
+ */
+ta_status attn_paged_gather_debug(const void *k_cache, const void *v_cache,
+                                  const int32_t *block_table, const int32_t *seq_lens,
+                                  int seq, int hkv, int page_size, int Hkv, int d, int max_pages,
+                                  int num_pages_total, void *k_out, void *v_out, ta_stream_t stream);
+
+/*
+ * Library-wide device status word of the current device (bounded-wait
+ * timeouts of attn_fwd, gather-debug flags).  Synchronises the device, stores
+ * the word in *flags (host pointer, may be NULL), clears it if `reset` is
+ * non-zero, and returns TA_ERR_DEVICE_TIMEOUT / TA_ERR_BAD_BLOCK_TABLE if the
+ * corresponding bit was set, else TA_OK.
+ */
+ta_status ta_device_status(unsigned *flags, int reset);
+
+/*
+ * Self-test of the bounded waits: launches one CTA that waits on an mbarrier
+ * nothing will ever complete, with a limit of `limit_us` microseconds
+ * (1..1000000).  The wait gives up, sets TA_DEV_TIMEOUT in the library status
+ * word and the kernel exits normally; the context stays usable.
+ */
+ta_status ta_selftest_bounded_wait(unsigned limit_us, ta_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TILEDATTN_H */

@@ -1,0 +1,109 @@
+"""The C-ABI library on the host (no GPU needed): it builds, loads, exports
+every entry point the header declares, and rejects bad arguments before any
+CUDA call."""
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tiledattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_attention_17_b200 import binding, build
+    build.build()
+    return binding
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)) - {"defined"})
+
+
+def test_header_functions_exported(lib):
+    import ctypes
+    L = lib.load()
+    names = declared_functions()
+    assert set(lib.EXPORTS) == set(names), (names, lib.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+        assert isinstance(getattr(L, n), ctypes._CFuncPtr)
+
+
+def test_status_strings(lib):
+    assert lib.ta_status_string(0) == "TA_OK"
+    assert lib.ta_status_string(4) == "TA_ERR_BAD_BLOCK_TABLE"
+    assert lib.ta_status_string(99) == "TA_ERR_UNKNOWN"
+    assert lib.ta_version() == 10000
+
+
+def code(lib, c):
+    return lib.STATUS_NAMES[c]
+
+
+def test_attn_fwd_validation(lib):
+    a = 256  # any 16-byte-aligned non-null value: rejected before use
+    f = lambda *x, **kw: code(lib, lib.attn_fwd(*x, check=False, stream=0, **kw))
+    assert f(a, a, a, a, None, 1, 3, 2, 128, 128, 128, 0.1, 0) == "TA_ERR_INVALID_ARG"   # Hq % Hkv
+    assert f(a, a, a, a, None, 1, 1, 1, 128, 128, 96, 0.1, 0) == "TA_ERR_UNSUPPORTED"   # head dim
+    assert f(a + 2, a, a, a, None, 1, 1, 1, 128, 128, 128, 0.1, 0) == "TA_ERR_INVALID_ARG"  # alignment
+    assert f(a, a, a, a, a + 2, 1, 1, 1, 128, 128, 128, 0.1, 0) == "TA_ERR_INVALID_ARG"  # lse alignment
+    assert f(a, a, a, a, None, 1, 1, 1, 128, 128, 128, -0.5, 0) == "TA_ERR_UNSUPPORTED"  # negative scale
+    assert f(a, a, a, a, None, 1, 1, 1, 128, 128, 128, float("nan"), 0) == "TA_ERR_UNSUPPORTED"
+    assert f(a, a, a, a, None, 1, 1, 1, 128, 128, 128, 0.1, 2) == "TA_ERR_INVALID_ARG"   # causal flag
+    assert f(a, a, a, a, None, -1, 1, 1, 128, 128, 128, 0.1, 0) == "TA_ERR_INVALID_ARG"  # negative size
+    assert f(None, a, a, a, None, 1, 1, 1, 128, 128, 128, 0.1, 0) == "TA_ERR_INVALID_ARG"  # null
+    assert f(a, a, a, a, None, 0, 1, 1, 128, 128, 128, 0.1, 0) == "TA_OK"                # empty: no-op
+    assert f(None, None, None, None, None, 1, 1, 1, 0, 128, 128, 0.1, 0) == "TA_OK"
+
+
+def test_decode_validation(lib):
+    a = 256
+    f = lambda *x: code(lib, lib.attn_paged_decode(*x, check=False, stream=0))
+    ws = lib.attn_paged_decode_workspace_size(4, 8, 2, 128, 64, 16)
+    good = dict(q=a, kc=a, vc=a, bt=a, sl=a, ps=16, S=4, Hq=8, Hkv=2, d=128, mp=64, P=100)
+
+    def call(**kw):
+        g = dict(good, **kw)
+        return f(g["q"], g["kc"], g["vc"], g["bt"], g["sl"], g["ps"], g["S"], g["Hq"], g["Hkv"], g["d"],
+                 g["mp"], g["P"], 0.1, a, None, a, kw.get("wsb", ws))
+
+    assert call(ps=12) == "TA_ERR_UNSUPPORTED"
+    assert call(ps=128) == "TA_ERR_UNSUPPORTED"
+    assert call(Hq=6, Hkv=4) == "TA_ERR_INVALID_ARG"
+    assert call(Hq=24, Hkv=2) == "TA_ERR_UNSUPPORTED"      # group of 12
+    assert call(d=80) == "TA_ERR_UNSUPPORTED"
+    assert call(wsb=ws - 1) == "TA_ERR_INVALID_ARG"
+    assert call(q=a + 8) == "TA_ERR_INVALID_ARG"
+    assert call(bt=a + 2) == "TA_ERR_INVALID_ARG"
+    assert call(P=0) == "TA_ERR_INVALID_ARG"
+    assert call(S=0) == "TA_OK"
+
+
+def test_workspace_plan(lib):
+    # 64 sequences x 8 KV heads x 2048 pages of 16: 1024-token splits -> 32 splits
+    ws = lib.attn_paged_decode_workspace_size(64, 32, 8, 128, 2048, 16)
+    rows = 64 * 32 * 32
+    assert ws >= rows * 128 * 4 + rows * 4 + 256
+    assert ws % 256 == 0
+    assert lib.attn_paged_decode_workspace_size(64, 32, 8, 128, 2048, 12) == 0
+    assert lib.attn_paged_decode_workspace_size(64, 30, 8, 128, 2048, 16) == 0
+    # a single short-batch sequence splits finer to fill the GPU
+    ws1 = lib.attn_paged_decode_workspace_size(1, 32, 8, 128, 2048, 16)
+    assert ws1 > 1 * 32 * 32 * 128 * 4
+
+
+def test_gather_debug_validation(lib):
+    a = 256
+    c = lib.attn_paged_gather_debug(a, a, a, a, 0, 2, 16, 2, 128, 8, 10, a, a, stream=0, check=False)
+    assert code(lib, c) == "TA_ERR_INVALID_ARG"     # hkv out of range
+    c = lib.attn_paged_gather_debug(a, a, a, a, 0, 0, 16, 2, 96, 8, 10, a, a, stream=0, check=False)
+    assert code(lib, c) == "TA_ERR_UNSUPPORTED"
+
+
+def test_selftest_validation(lib):
+    assert code(lib, lib.ta_selftest_bounded_wait(0, stream=0)) == "TA_ERR_INVALID_ARG"
+    assert code(lib, lib.ta_selftest_bounded_wait(2_000_000, stream=0)) == "TA_ERR_INVALID_ARG"

@@ -1,0 +1,195 @@
+"""ctypes binding of libtiledattn.so (argument marshalling only).
+
+Every function here passes device pointers, sizes and the CUDA stream through
+to the C ABI declared in include/tiledattn.h; all computation happens in the
+library's kernels.  There is no fallback: if the shared object cannot be
+loaded, every call raises.
+
+Functions with the C names take raw integers (device pointers) or torch
+tensors (their data_ptr() is passed).  `attention()` and `paged_decode()` are
+conveniences that allocate outputs with torch and call the C entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libtiledattn.so")
+
+TA_OK = 0
+STATUS_NAMES = {0: "TA_OK", 1: "TA_ERR_INVALID_ARG", 2: "TA_ERR_UNSUPPORTED", 3: "TA_ERR_CUDA",
+                4: "TA_ERR_BAD_BLOCK_TABLE", 5: "TA_ERR_DEVICE_TIMEOUT"}
+TA_DEV_TIMEOUT = 1
+TA_DEV_BAD_BLOCK_TABLE = 2
+TA_DEV_BAD_SEQ_LEN = 4
+
+EXPORTS = ["ta_status_string", "ta_version", "attn_fwd", "attn_paged_decode_workspace_size",
+           "attn_paged_decode", "attn_paged_decode_check", "attn_paged_gather_debug",
+           "ta_device_status", "ta_selftest_bounded_wait"]
+
+
+class TiledAttnError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(code, code)}")
+
+
+_lib = None
+
+
+def load(path: str | None = None):
+    """Load (once) and return the ctypes handle of libtiledattn.so."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"libtiledattn.so not found at {p}; build it with "
+                           f"`python -m tiled_attention_17_b200.build`")
+    L = ctypes.CDLL(p)
+    vp, i32, f32, sz, u32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint
+    L.ta_status_string.argtypes = [i32]
+    L.ta_status_string.restype = ctypes.c_char_p
+    L.ta_version.restype = i32
+    L.attn_fwd.argtypes = [vp, vp, vp, vp, vp] + [i32] * 6 + [f32, i32, vp]
+    L.attn_fwd.restype = i32
+    L.attn_paged_decode_workspace_size.argtypes = [i32] * 6
+    L.attn_paged_decode_workspace_size.restype = sz
+    L.attn_paged_decode.argtypes = [vp, vp, vp, vp, vp] + [i32] * 7 + [f32, vp, vp, vp, sz, vp]
+    L.attn_paged_decode.restype = i32
+    L.attn_paged_decode_check.argtypes = [vp, ctypes.POINTER(u32), vp]
+    L.attn_paged_decode_check.restype = i32
+    L.attn_paged_gather_debug.argtypes = [vp, vp, vp, vp] + [i32] * 7 + [vp, vp, vp]
+    L.attn_paged_gather_debug.restype = i32
+    L.ta_device_status.argtypes = [ctypes.POINTER(u32), i32]
+    L.ta_device_status.restype = i32
+    L.ta_selftest_bounded_wait.argtypes = [u32, vp]
+    L.ta_selftest_bounded_wait.restype = i32
+    if path is None:
+        _lib = L
+    return L
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn, code):
+    if code != TA_OK:
+        raise TiledAttnError(fn, code)
+
+
+# ---------------------------------------------------------------------------
+# C-named entry points
+# ---------------------------------------------------------------------------
+
+def ta_status_string(code: int) -> str:
+    return load().ta_status_string(code).decode()
+
+
+def ta_version() -> int:
+    return load().ta_version()
+
+
+def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream=None, check=True) -> int:
+    code = load().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nkv, d,
+                           float(scale), int(causal), _stream(stream))
+    if check:
+        _check("attn_fwd", code)
+    return code
+
+
+def attn_paged_decode_workspace_size(num_seqs, Hq, Hkv, d, max_pages, page_size) -> int:
+    return load().attn_paged_decode_workspace_size(num_seqs, Hq, Hkv, d, max_pages, page_size)
+
+
+def attn_paged_decode(q, k_cache, v_cache, block_table, seq_lens, page_size, num_seqs, Hq, Hkv, d,
+                      max_pages, num_pages_total, scale, o, lse, workspace, workspace_bytes,
+                      stream=None, check=True) -> int:
+    code = load().attn_paged_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                    page_size, num_seqs, Hq, Hkv, d, max_pages, num_pages_total, float(scale),
+                                    _ptr(o), _ptr(lse), _ptr(workspace), int(workspace_bytes), _stream(stream))
+    if check:
+        _check("attn_paged_decode", code)
+    return code
+
+
+def attn_paged_decode_check(workspace, stream=None):
+    flags = ctypes.c_uint(0)
+    code = load().attn_paged_decode_check(_ptr(workspace), ctypes.byref(flags), _stream(stream))
+    return code, flags.value
+
+
+def attn_paged_gather_debug(k_cache, v_cache, block_table, seq_lens, seq, hkv, page_size, Hkv, d, max_pages,
+                            num_pages_total, k_out, v_out, stream=None, check=True) -> int:
+    code = load().attn_paged_gather_debug(_ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seq_lens),
+                                          seq, hkv, page_size, Hkv, d, max_pages, num_pages_total,
+                                          _ptr(k_out), _ptr(v_out), _stream(stream))
+    if check:
+        _check("attn_paged_gather_debug", code)
+    return code
+
+
+def ta_device_status(reset: bool = True):
+    flags = ctypes.c_uint(0)
+    code = load().ta_device_status(ctypes.byref(flags), int(reset))
+    return code, flags.value
+
+
+def ta_selftest_bounded_wait(limit_us: int, stream=None) -> int:
+    return load().ta_selftest_bounded_wait(int(limit_us), _stream(stream))
+
+
+# ---------------------------------------------------------------------------
+# torch conveniences (allocate outputs, then call the C entry points)
+# ---------------------------------------------------------------------------
+
+def attention(q, k, v, causal: bool, scale: float | None = None, out=None, lse=None, stream=None):
+    """q [B,Hq,Nq,d], k/v [B,Hkv,Nkv,d] bf16 CUDA tensors -> (o, lse)."""
+    import torch
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nkv, _ = k.shape
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    if scale is None:
+        scale = d ** -0.5
+    o = out if out is not None else torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream)
+    return o, lse
+
+
+def paged_decode(q, k_cache, v_cache, block_table, seq_lens, scale: float | None = None, workspace=None,
+                 out=None, lse=None, stream=None):
+    """q [S,Hq,d]; caches [P,Hkv,page,d] bf16; block_table [S,max_pages] int32; seq_lens [S] int32."""
+    import torch
+    S, Hq, d = q.shape
+    P, Hkv, ps, _ = k_cache.shape
+    max_pages = block_table.shape[1]
+    if scale is None:
+        scale = d ** -0.5
+    ws_bytes = attn_paged_decode_workspace_size(S, Hq, Hkv, d, max_pages, ps)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
+    o = out if out is not None else torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    attn_paged_decode(q, k_cache, v_cache, block_table, seq_lens, ps, S, Hq, Hkv, d, max_pages, P, scale,
+                      o, lse, workspace, workspace.numel(), stream)
+    return o, lse, workspace

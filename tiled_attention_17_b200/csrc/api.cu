@@ -1,0 +1,178 @@
+// C ABI of libtiledattn.so: host-side argument validation, the library status
+// word, and dispatch to the kernels.  Declarations and the contract of every
+// entry point are in include/tiledattn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "ptx.cuh"
+#include "tiledattn_internal.h"
+
+namespace ta {
+
+static_assert(kDevTimeout == TA_DEV_TIMEOUT && kDevBadBlockTable == TA_DEV_BAD_BLOCK_TABLE &&
+                  kDevBadSeqLen == TA_DEV_BAD_SEQ_LEN,
+              "device status bits");
+
+// One status word per device (a __device__ variable exists once per device
+// the library is loaded on).  Bits: TA_DEV_*.
+__device__ unsigned g_status_word;
+
+unsigned* device_status_ptr() {
+  static unsigned* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> g(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<unsigned*>(p);
+  }
+  return ptrs[dev];
+}
+
+PFN_encodeTiled get_encode_tiled() {
+  static PFN_encodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  });
+  return fn;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace ta
+
+using namespace ta;
+
+extern "C" {
+
+const char* ta_status_string(ta_status s) {
+  switch (s) {
+    case TA_OK: return "TA_OK";
+    case TA_ERR_INVALID_ARG: return "TA_ERR_INVALID_ARG";
+    case TA_ERR_UNSUPPORTED: return "TA_ERR_UNSUPPORTED";
+    case TA_ERR_CUDA: return "TA_ERR_CUDA";
+    case TA_ERR_BAD_BLOCK_TABLE: return "TA_ERR_BAD_BLOCK_TABLE";
+    case TA_ERR_DEVICE_TIMEOUT: return "TA_ERR_DEVICE_TIMEOUT";
+  }
+  return "TA_ERR_UNKNOWN";
+}
+
+int ta_version(void) { return 10000; }
+
+ta_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                   int Nkv, int d, float scale, int causal, ta_stream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nkv < 0 || d <= 0) return TA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return TA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return TA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return TA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return TA_ERR_UNSUPPORTED;
+  // sizes the kernels index with 32-bit coordinates
+  if (static_cast<long long>(B) * Hq > INT32_MAX / 2 || Nq > (1 << 30) || Nkv > (1 << 30)) return TA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq * Nq == 0) return TA_OK;
+  if (!q || !o || (Nkv > 0 && (!k || !v))) return TA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return TA_ERR_INVALID_ARG;
+  const long long pairs = (static_cast<long long>(Nq) + 255) / 256;
+  if (pairs * B * Hq > INT32_MAX) return TA_ERR_UNSUPPORTED;
+  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t attn_paged_decode_workspace_size(int num_seqs, int Hq, int Hkv, int d, int max_pages, int page_size) {
+  if (Hkv <= 0 || Hq <= 0 || Hq % Hkv) return 0;
+  DecodePlan plan;
+  if (!make_decode_plan(num_seqs, Hq, Hkv, d, max_pages, page_size, &plan)) return 0;
+  return plan.bytes;
+}
+
+static ta_status validate_decode_shape(int page_size, int num_seqs, int Hq, int Hkv, int d, int max_pages,
+                                       int num_pages_total) {
+  if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || max_pages <= 0 || num_pages_total <= 0 || page_size <= 0)
+    return TA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return TA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return TA_ERR_UNSUPPORTED;
+  if (page_size != 8 && page_size != 16 && page_size != 32 && page_size != 64) return TA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return TA_ERR_UNSUPPORTED;
+  if (num_seqs > 65535 || Hkv > 65535) return TA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_pages) * page_size > INT32_MAX) return TA_ERR_UNSUPPORTED;
+  return TA_OK;
+}
+
+ta_status attn_paged_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                            const int32_t* seq_lens, int page_size, int num_seqs, int Hq, int Hkv, int d,
+                            int max_pages, int num_pages_total, float scale, void* o, float* lse, void* workspace,
+                            size_t workspace_bytes, ta_stream_t stream) {
+  ta_status st = validate_decode_shape(page_size, num_seqs, Hq, Hkv, d, max_pages, num_pages_total);
+  if (st != TA_OK) return st;
+  if (!std::isfinite(scale) || scale < 0.f) return TA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return TA_OK;
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !o || !workspace) return TA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return TA_ERR_INVALID_ARG;
+  DecodePlan plan;
+  if (!make_decode_plan(num_seqs, Hq, Hkv, d, max_pages, page_size, &plan)) return TA_ERR_UNSUPPORTED;
+  if (workspace_bytes < plan.bytes) return TA_ERR_INVALID_ARG;
+  return launch_paged_decode(q, k_cache, v_cache, block_table, seq_lens, page_size, num_seqs, Hq, Hkv, d, max_pages,
+                             num_pages_total, scale, o, lse, workspace, plan, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ta_status attn_paged_decode_check(const void* workspace, unsigned* flags, ta_stream_t stream) {
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return TA_ERR_INVALID_ARG;
+  unsigned w = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&w, workspace, sizeof(w), cudaMemcpyDeviceToHost, s) != cudaSuccess) return TA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TA_ERR_CUDA;
+  if (flags) *flags = w;
+  if (w & TA_DEV_TIMEOUT) return TA_ERR_DEVICE_TIMEOUT;
+  if (w & (TA_DEV_BAD_BLOCK_TABLE | TA_DEV_BAD_SEQ_LEN)) return TA_ERR_BAD_BLOCK_TABLE;
+  return TA_OK;
+}
+
+ta_status attn_paged_gather_debug(const void* k_cache, const void* v_cache, const int32_t* block_table,
+                                  const int32_t* seq_lens, int seq, int hkv, int page_size, int Hkv, int d,
+                                  int max_pages, int num_pages_total, void* k_out, void* v_out, ta_stream_t stream) {
+  ta_status st = validate_decode_shape(page_size, seq + 1, Hkv, Hkv, d, max_pages, num_pages_total);
+  if (st != TA_OK) return st;
+  if (seq < 0 || hkv < 0 || hkv >= Hkv) return TA_ERR_INVALID_ARG;
+  if (!k_cache || !v_cache || !block_table || !seq_lens || !k_out || !v_out) return TA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_out) || !aligned16(v_out) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return TA_ERR_INVALID_ARG;
+  return launch_gather_debug(k_cache, v_cache, block_table, seq_lens, seq, hkv, page_size, Hkv, d, max_pages,
+                             num_pages_total, k_out, v_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ta_status ta_device_status(unsigned* flags, int reset) {
+  unsigned* p = device_status_ptr();
+  if (!p) return TA_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return TA_ERR_CUDA;
+  unsigned w = 0;
+  if (cudaMemcpy(&w, p, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return TA_ERR_CUDA;
+  if (reset && cudaMemset(p, 0, sizeof(unsigned)) != cudaSuccess) return TA_ERR_CUDA;
+  if (flags) *flags = w;
+  if (w & TA_DEV_TIMEOUT) return TA_ERR_DEVICE_TIMEOUT;
+  if (w & (TA_DEV_BAD_BLOCK_TABLE | TA_DEV_BAD_SEQ_LEN)) return TA_ERR_BAD_BLOCK_TABLE;
+  return TA_OK;
+}
+
+ta_status ta_selftest_bounded_wait(unsigned limit_us, ta_stream_t stream) {
+  if (limit_us == 0 || limit_us > 1000000u) return TA_ERR_INVALID_ARG;
+  return launch_selftest_wait(limit_us, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,538 @@
+// Split-KV paged decode for sm_100a: one query token per sequence against a
+// paged KV cache, followed by a log-sum-exp combine of the splits.
+//
+// The pool holds fixed-size pages [num_pages_total, Hkv, page_size, d]; a
+// sequence's pages are listed in its block-table row (PagedAttention,
+// GPU-optimisation tag page).  The gather follows the paged gather article,
+// section 2:
+//   2.1  a CTA stages the scattered pages of its range into shared memory;
+//        here each (page, KV head) is one contiguous page_size*d*2-byte span,
+//        so one TMA bulk copy moves it and every byte read is used;
+//   2.3  the split's block-table entries are loaded into registers of the
+//        issuing warp before the gather loop (index prefetch);
+//   2.4  the gather is fused with the dot products q.k, the online softmax
+//        and the weighted sum of V; nothing gathered is written back.
+// Splits are merged by their log-sum-exp, which is exact because the online
+// softmax result does not depend on how the keys are grouped (FlashAttention
+// optimisation article, section 3.2.2).
+//
+// Kernel 1 (decode_split_kernel): one CTA per (split, KV head, sequence);
+//   the G = Hq/Hkv query heads of the KV head are handled together so every
+//   K/V byte is read from HBM once.  A 3-stage ring of 64-token chunks keeps
+//   up to 96 KB per CTA in flight.  Per chunk:
+//     A) scores: 16 lanes cover one 256-byte K row with 16-byte shared loads,
+//        dot with the G query slices held in registers, reduce across lanes;
+//     B) online softmax per head (one warp per head): chunk max, rescale
+//        factor e^(m_old - m_new), probabilities, running sum;
+//     C) O_partial = alpha * O_partial + sum_t p_t v_t.
+// Kernel 2 (decode_combine_kernel): one CTA per (query head, sequence).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "tiledattn_internal.h"
+
+namespace ta {
+
+constexpr int kDecThreads = 128;
+constexpr int kChunkTokens = 64;
+constexpr int kDecStages = 3;
+constexpr int kMaxG = 8;
+
+template <int D>
+struct DecodeLayout {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kChunkBytes = kChunkTokens * kRowBytes;
+  static constexpr int kStageBytes = 2 * kChunkBytes;   // K chunk then V chunk
+  static constexpr int kScores = kDecStages * kStageBytes;
+  static constexpr int kAlpha = kScores + kChunkTokens * kMaxG * 4;
+  static constexpr int kM = kAlpha + kMaxG * 4;
+  static constexpr int kL = kM + kMaxG * 4;
+  static constexpr int kBar = kL + kMaxG * 4;
+  static constexpr int kAbort = kBar + kDecStages * 8;
+  static constexpr int kBytes = kAbort + 16;
+  static constexpr int kLanesPerRow = D / 8;            // 16-byte slices per row
+  static constexpr int kRowGroups = kDecThreads / kLanesPerRow;
+  static_assert(kRowGroups * kMaxG * D * 4 <= kScores, "reduction buffer fits in the ring");
+};
+
+struct DecodeArgs {
+  const __nv_bfloat16* q;
+  const uint8_t* k_cache;
+  const uint8_t* v_cache;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  int page_size, num_seqs, Hq, Hkv, max_pages, num_pages_total;
+  int split_pages, max_splits;
+  float scale, scale_log2;
+  float* part_o;
+  float* part_lse;
+  unsigned* status;
+};
+
+__device__ __forceinline__ int clamp_len(int len, const DecodeArgs& a) {
+  const int cap = a.max_pages * a.page_size;
+  return len < 0 ? 0 : (len > cap ? cap : len);
+}
+
+// The page gather shared by decode and the gather-debug export.  Warp-wide:
+// every lane of the calling warp must call it.  Stages the `npg` pages
+// starting at split-local page `first` into dstK/dstV (consecutive, in page
+// order) and arms `bar` with their byte count.  tbl0/tbl1 hold the split's
+// prefetched block-table entries (entry i sits in lane i % 32, register i / 32).
+// Entries outside [0, num_pages_total) are replaced by page 0 and flagged.
+template <int D>
+__device__ __forceinline__ void gather_pages(const DecodeArgs& a, int hkv, int first, int npg, int tbl0, int tbl1,
+                                             uint32_t dstK, uint32_t dstV, uint32_t bar, unsigned* flag_word) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t page_bytes = static_cast<uint32_t>(a.page_size) * D * 2;
+  if (lane == 0) mbar_arrive_expect_tx(bar, 2u * npg * page_bytes);
+  __syncwarp();
+  const int idx = first + lane;
+  const int v0 = __shfl_sync(0xffffffffu, tbl0, idx & 31);
+  const int v1 = __shfl_sync(0xffffffffu, tbl1, idx & 31);
+  if (lane < npg) {
+    int pg = (idx < 32) ? v0 : v1;
+    if (pg < 0 || pg >= a.num_pages_total) {
+      atomicOr(flag_word, kDevBadBlockTable);
+      pg = 0;
+    }
+    const size_t off = (static_cast<size_t>(pg) * a.Hkv + hkv) * page_bytes;
+    bulk_load(dstK + lane * page_bytes, a.k_cache + off, page_bytes, bar);
+    bulk_load(dstV + lane * page_bytes, a.v_cache + off, page_bytes, bar);
+  }
+}
+
+// Loads the block-table entries of pages [first_page, first_page + npages)
+// of `seq` into two registers per lane (index prefetch).
+__device__ __forceinline__ void prefetch_table(const DecodeArgs& a, int seq, int first_page, int npages, int& tbl0,
+                                               int& tbl1) {
+  const int lane = threadIdx.x & 31;
+  const int32_t* row = a.block_table + static_cast<size_t>(seq) * a.max_pages + first_page;
+  tbl0 = lane < npages ? __ldg(row + lane) : -1;
+  tbl1 = lane + 32 < npages ? __ldg(row + lane + 32) : -1;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const DecodeArgs a) {
+  using L = DecodeLayout<D>;
+  constexpr int LPR = L::kLanesPerRow;
+  constexpr int RG = L::kRowGroups;
+  extern __shared__ __align__(128) uint8_t smem[];
+
+  const int split = blockIdx.x, hkv = blockIdx.y, seq = blockIdx.z;
+  const int raw_len = __ldg(a.seq_lens + seq);
+  const int len = clamp_len(raw_len, a);
+  if (raw_len != len && split == 0 && hkv == 0 && threadIdx.x == 0) atomicOr(a.status, kDevBadSeqLen);
+  const int split_tokens = a.split_pages * a.page_size;
+  const int t_begin = split * split_tokens;
+  if (t_begin >= len) return;  // CTA-uniform: nothing in this split
+  const int t_end = min(len, t_begin + split_tokens);
+  const int n_chunks = (t_end - t_begin + kChunkTokens - 1) / kChunkTokens;
+  const int split_first_page = split * a.split_pages;
+  const int split_npages = (t_end - t_begin + a.page_size - 1) / a.page_size;
+  const int pages_per_chunk = kChunkTokens / a.page_size;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sbase = smem_u32(smem);
+  float* sc = reinterpret_cast<float*>(smem + L::kScores);       // [64][kMaxG] scores, then probabilities
+  float* s_alpha = reinterpret_cast<float*>(smem + L::kAlpha);
+  float* s_m = reinterpret_cast<float*>(smem + L::kM);
+  float* s_l = reinterpret_cast<float*>(smem + L::kL);
+  const uint32_t bar0 = sbase + L::kBar;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+
+  if (tid == 0) {
+    for (int s = 0; s < kDecStages; ++s) mbar_init(bar0 + 8 * s, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // warp 0: prefetch the split's table entries, start the first stages
+  int tbl0 = -1, tbl1 = -1;
+  if (warp == 0) {
+    prefetch_table(a, seq, split_first_page, split_npages, tbl0, tbl1);
+    for (int c = 0; c < min(kDecStages, n_chunks); ++c) {
+      const int first = c * pages_per_chunk;
+      const int npg = min(pages_per_chunk, split_npages - first);
+      const uint32_t st = sbase + c * L::kStageBytes;
+      gather_pages<D>(a, hkv, first, npg, tbl0, tbl1, st, st + L::kChunkBytes, bar0 + 8 * c, a.status);
+    }
+  }
+
+  // this thread's slice of the G query vectors
+  const int lane_r = tid % LPR;   // 16-byte slice of a row
+  const int rg = tid / LPR;       // row group
+  float qf[G][8];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(seq) * a.Hq + hkv * G + g) * D) +
+                          lane_r);
+    unpack8(u, qf[g]);
+  }
+  float acc[G][8];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+  // running statistics, owned by warp (g % 4) for head g
+  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
+  const float c2 = a.scale_log2;
+  const uint32_t seg_mask = (LPR == 16) ? (0xFFFFu << (lane & 16)) : (0xFFu << (lane & 24));
+
+  int c = 0;
+  for (; c < n_chunks; ++c) {
+    const int stage = c % kDecStages;
+    const uint32_t st = sbase + stage * L::kStageBytes;
+    const uint8_t* sK = smem + stage * L::kStageBytes;
+    const uint8_t* sV = sK + L::kChunkBytes;
+    const bool ok = mbar_wait(bar0 + 8 * stage, (c / kDecStages) & 1u, a.status, abort_flag);
+    const int valid = min(kChunkTokens, t_end - (t_begin + c * kChunkTokens));
+
+    // ---- A: scores s[t][g] = q_g . k_t
+    for (int r = rg; r < valid; r += RG) {
+      float kf[8];
+      unpack8(*reinterpret_cast<const uint4*>(sK + r * L::kRowBytes + lane_r * 16), kf);
+      float part[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s = fmaf(qf[g][e], kf[e], s);
+        part[g] = s;
+      }
+      if constexpr (G == 4) {
+        // reduce-scatter over the LPR lanes of the row: each lane ends with one head's total
+        const bool hi = lane_r & (LPR / 2);
+        float ka = hi ? part[2] : part[0], kb = hi ? part[3] : part[1];
+        const float sa = hi ? part[0] : part[2], sb = hi ? part[1] : part[3];
+        ka += __shfl_xor_sync(seg_mask, sa, LPR / 2);
+        kb += __shfl_xor_sync(seg_mask, sb, LPR / 2);
+        const bool hi2 = lane_r & (LPR / 4);
+        float x = hi2 ? kb : ka;
+        x += __shfl_xor_sync(seg_mask, hi2 ? ka : kb, LPR / 4);
+#pragma unroll
+        for (int o = LPR / 8; o >= 1; o >>= 1) x += __shfl_xor_sync(seg_mask, x, o);
+        if ((lane_r & (LPR / 4 - 1)) == 0) sc[r * kMaxG + (hi ? 2 : 0) + (hi2 ? 1 : 0)] = x;
+      } else {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int o = LPR / 2; o >= 1; o >>= 1) part[g] += __shfl_xor_sync(seg_mask, part[g], o);
+        if (lane_r == 0) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) sc[r * kMaxG + g] = part[g];
+        }
+      }
+    }
+    if (__syncthreads_or(!ok)) break;
+
+    // ---- B: online softmax per head (warp g % 4 owns head g)
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+      const int g = warp + 4 * gi;
+      if (g < G) {
+        const float x0 = lane < valid ? sc[lane * kMaxG + g] : -INFINITY;
+        const float x1 = lane + 32 < valid ? sc[(lane + 32) * kMaxG + g] : -INFINITY;
+        float mx = fmaxf(x0, x1);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float m_new = fmaxf(m_r[gi], mx);
+        const float alpha = (m_r[gi] == -INFINITY) ? 0.f : ex2((m_r[gi] - m_new) * c2);
+        const float p0 = lane < valid ? ex2((x0 - m_new) * c2) : 0.f;
+        const float p1 = lane + 32 < valid ? ex2((x1 - m_new) * c2) : 0.f;
+        sc[lane * kMaxG + g] = p0;
+        sc[(lane + 32) * kMaxG + g] = p1;
+        float ps = p0 + p1;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        l_r[gi] = alpha * l_r[gi] + ps;
+        m_r[gi] = m_new;
+        if (lane == 0) s_alpha[g] = alpha;
+      }
+    }
+    __syncthreads();
+
+    // ---- C: acc = alpha * acc + sum_t p_t v_t
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float al = s_alpha[g];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[g][e] *= al;
+    }
+    for (int r = rg; r < valid; r += RG) {
+      float vf[8];
+      unpack8(*reinterpret_cast<const uint4*>(sV + r * L::kRowBytes + lane_r * 16), vf);
+      float p[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) p[g] = sc[r * kMaxG + g];
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(p[g], vf[e], acc[g][e]);
+    }
+    __syncthreads();  // stage and score buffer free
+
+    if (warp == 0 && c + kDecStages < n_chunks) {
+      const int cn = c + kDecStages;
+      const int first = cn * pages_per_chunk;
+      const int npg = min(pages_per_chunk, split_npages - first);
+      gather_pages<D>(a, hkv, first, npg, tbl0, tbl1, st, st + L::kChunkBytes, bar0 + 8 * stage, a.status);
+    }
+  }
+
+  if (c < n_chunks) {
+    // a wait gave up: drain what may still be in flight, then leave
+    if (tid == 0) {
+      for (int cc = c; cc < min(n_chunks, c + kDecStages); ++cc)
+        mbar_wait(bar0 + 8 * (cc % kDecStages), (cc / kDecStages) & 1u, nullptr, nullptr, kWaitLimitNs);
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ---- reduce the row groups' partial outputs, normalise, write the split's partials
+  float* red = reinterpret_cast<float*>(smem);
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[(rg * G + g) * D + lane_r * 8 + e] = acc[g][e];
+#pragma unroll
+  for (int gi = 0; gi < 2; ++gi) {
+    const int g = warp + 4 * gi;
+    if (g < G && lane == 0) {
+      s_m[g] = m_r[gi];
+      s_l[g] = l_r[gi];
+    }
+  }
+  __syncthreads();
+  const size_t row0 = (static_cast<size_t>(seq) * a.Hq + hkv * G) * a.max_splits + split;
+  for (int idx = tid; idx < G * D; idx += kDecThreads) {
+    const int g = idx / D, col = idx % D;
+    float s = 0.f;
+#pragma unroll 4
+    for (int r = 0; r < RG; ++r) s += red[(r * G + g) * D + col];
+    a.part_o[(row0 + static_cast<size_t>(g) * a.max_splits) * D + col] = s / s_l[g];
+  }
+  if (tid < G) {
+    a.part_lse[row0 + static_cast<size_t>(tid) * a.max_splits] =
+        fmaf(s_m[tid], a.scale, __logf(s_l[tid]));
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a, __nv_bfloat16* o, float* lse) {
+  const int hq = blockIdx.x, seq = blockIdx.y;
+  const int len = clamp_len(__ldg(a.seq_lens + seq), a);
+  const int split_tokens = a.split_pages * a.page_size;
+  const int ns = (len + split_tokens - 1) / split_tokens;
+  const size_t row0 = (static_cast<size_t>(seq) * a.Hq + hq) * a.max_splits;
+  const size_t orow = static_cast<size_t>(seq) * a.Hq + hq;
+  const int col = threadIdx.x;
+  if (ns == 0) {
+    if (col < D) o[orow * D + col] = __float2bfloat16(0.f);
+    if (col == 0 && lse) lse[orow] = -INFINITY;
+    return;
+  }
+  float mx = -INFINITY;
+  for (int s = 0; s < ns; ++s) mx = fmaxf(mx, a.part_lse[row0 + s]);
+  float tot = 0.f, acc = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const float w = __expf(a.part_lse[row0 + s] - mx);
+    tot += w;
+    if (col < D) acc = fmaf(w, a.part_o[(row0 + s) * D + col], acc);
+  }
+  if (col < D) o[orow * D + col] = __float2bfloat16(acc / tot);
+  if (col == 0 && lse) lse[orow] = mx + __logf(tot);
+}
+
+// Gather-debug: same gather routine, result written out contiguously.
+template <int D>
+__global__ void __launch_bounds__(kDecThreads) gather_debug_kernel(const DecodeArgs a, int seq, int hkv,
+                                                                   __nv_bfloat16* k_out, __nv_bfloat16* v_out) {
+  using L = DecodeLayout<D>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar = sbase + L::kBar;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int len = clamp_len(__ldg(a.seq_lens + seq), a);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int pages_per_chunk = kChunkTokens / a.page_size;
+  const int npages = (len + a.page_size - 1) / a.page_size;
+  int phase = 0;
+  for (int g0 = 0; g0 < npages; g0 += 64) {       // table prefetch covers 64 pages
+    const int gn = min(64, npages - g0);
+    int tbl0 = -1, tbl1 = -1;
+    if (warp == 0) prefetch_table(a, seq, g0, gn, tbl0, tbl1);
+    for (int first = 0; first < gn; first += pages_per_chunk) {
+      const int npg = min(pages_per_chunk, gn - first);
+      if (warp == 0)
+        gather_pages<D>(a, hkv, first, npg, tbl0, tbl1, sbase, sbase + L::kChunkBytes, bar, a.status);
+      const bool ok = mbar_wait(bar, phase & 1u, a.status, abort_flag);
+      phase++;
+      if (__syncthreads_or(!ok)) return;
+      const int t0 = (g0 + first) * a.page_size;
+      const int rows = min(npg * a.page_size, len - t0);
+      const int words = rows * D / 8;   // 16-byte words
+      for (int w = tid; w < words; w += kDecThreads) {
+        reinterpret_cast<uint4*>(k_out + static_cast<size_t>(t0) * D)[w] = reinterpret_cast<const uint4*>(smem)[w];
+        reinterpret_cast<uint4*>(v_out + static_cast<size_t>(t0) * D)[w] =
+            reinterpret_cast<const uint4*>(smem + L::kChunkBytes)[w];
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Bounded-wait self-test: nothing ever arrives on this barrier.
+__global__ void selftest_wait_kernel(unsigned* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  abort_flag = 0;
+  fence_mbar_init();
+  mbar_wait(b, 0, status, &abort_flag, limit_ns);
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+static DecodeArgs make_args(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                            const int32_t* seq_lens, int page_size, int num_seqs, int Hq, int Hkv, int max_pages,
+                            int num_pages_total, float scale, int split_pages, int max_splits, void* workspace,
+                            const DecodePlan* plan, unsigned* status) {
+  DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k_cache = static_cast<const uint8_t*>(k_cache);
+  a.v_cache = static_cast<const uint8_t*>(v_cache);
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.page_size = page_size;
+  a.num_seqs = num_seqs;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.max_pages = max_pages;
+  a.num_pages_total = num_pages_total;
+  a.split_pages = split_pages;
+  a.max_splits = max_splits;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.part_o = plan ? reinterpret_cast<float*>(ws + plan->partial_o_offset) : nullptr;
+  a.part_lse = plan ? reinterpret_cast<float*>(ws + plan->partial_lse_offset) : nullptr;
+  a.status = status;
+  return a;
+}
+
+template <int D, int G>
+static cudaError_t launch_split(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
+  using L = DecodeLayout<D>;
+  static int attr_done[64] = {0};
+  cudaError_t e = ensure_smem_limit(decode_split_kernel<D, G>, L::kBytes, attr_done);
+  if (e != cudaSuccess) return e;
+  decode_split_kernel<D, G><<<grid, kDecThreads, L::kBytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_split_g(const DecodeArgs& a, int G, dim3 grid, cudaStream_t stream) {
+  switch (G) {
+    case 1: return launch_split<D, 1>(a, grid, stream);
+    case 2: return launch_split<D, 2>(a, grid, stream);
+    case 4: return launch_split<D, 4>(a, grid, stream);
+    default: return launch_split<D, 8>(a, grid, stream);
+  }
+}
+
+ta_status launch_paged_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                              const int32_t* seq_lens, int page_size, int num_seqs, int Hq, int Hkv, int d,
+                              int max_pages, int num_pages_total, float scale, void* o, float* lse, void* workspace,
+                              const DecodePlan& plan, cudaStream_t stream) {
+  if (num_seqs == 0) return TA_OK;
+  unsigned* status = static_cast<unsigned*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned), stream) != cudaSuccess) return TA_ERR_CUDA;
+  DecodeArgs a = make_args(q, k_cache, v_cache, block_table, seq_lens, page_size, num_seqs, Hq, Hkv, max_pages,
+                           num_pages_total, scale, plan.split_pages, plan.max_splits, workspace, &plan, status);
+  const int G = Hq / Hkv;
+  dim3 grid(plan.max_splits, Hkv, num_seqs);
+  cudaError_t e = (d == 128) ? launch_split_g<128>(a, G, grid, stream) : launch_split_g<64>(a, G, grid, stream);
+  if (e != cudaSuccess) return TA_ERR_CUDA;
+  dim3 cgrid(Hq, num_seqs);
+  if (d == 128)
+    decode_combine_kernel<128><<<cgrid, 128, 0, stream>>>(a, static_cast<__nv_bfloat16*>(o), lse);
+  else
+    decode_combine_kernel<64><<<cgrid, 128, 0, stream>>>(a, static_cast<__nv_bfloat16*>(o), lse);
+  return cudaGetLastError() == cudaSuccess ? TA_OK : TA_ERR_CUDA;
+}
+
+ta_status launch_gather_debug(const void* k_cache, const void* v_cache, const int32_t* block_table,
+                              const int32_t* seq_lens, int seq, int hkv, int page_size, int Hkv, int d,
+                              int max_pages, int num_pages_total, void* k_out, void* v_out, cudaStream_t stream) {
+  unsigned* status = device_status_ptr();
+  if (!status) return TA_ERR_CUDA;
+  DecodeArgs a = make_args(nullptr, k_cache, v_cache, block_table, seq_lens, page_size, seq + 1, Hkv, Hkv, max_pages,
+                           num_pages_total, 1.f, 64, 1, nullptr, nullptr, status);
+  static int done128[64] = {0}, done64[64] = {0};
+  if (d == 128) {
+    if (ensure_smem_limit(gather_debug_kernel<128>, DecodeLayout<128>::kBytes, done128) != cudaSuccess)
+      return TA_ERR_CUDA;
+    gather_debug_kernel<128><<<1, kDecThreads, DecodeLayout<128>::kBytes, stream>>>(
+        a, seq, hkv, static_cast<__nv_bfloat16*>(k_out), static_cast<__nv_bfloat16*>(v_out));
+  } else {
+    if (ensure_smem_limit(gather_debug_kernel<64>, DecodeLayout<64>::kBytes, done64) != cudaSuccess)
+      return TA_ERR_CUDA;
+    gather_debug_kernel<64><<<1, kDecThreads, DecodeLayout<64>::kBytes, stream>>>(
+        a, seq, hkv, static_cast<__nv_bfloat16*>(k_out), static_cast<__nv_bfloat16*>(v_out));
+  }
+  return cudaGetLastError() == cudaSuccess ? TA_OK : TA_ERR_CUDA;
+}
+
+ta_status launch_selftest_wait(unsigned limit_us, cudaStream_t stream) {
+  unsigned* status = device_status_ptr();
+  if (!status) return TA_ERR_CUDA;
+  selftest_wait_kernel<<<1, 1, 0, stream>>>(status, static_cast<unsigned long long>(limit_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? TA_OK : TA_ERR_CUDA;
+}
+
+bool make_decode_plan(int num_seqs, int Hq, int Hkv, int d, int max_pages, int page_size, DecodePlan* plan) {
+  if (page_size != 8 && page_size != 16 && page_size != 32 && page_size != 64) return false;
+  if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || max_pages <= 0 || (d != 64 && d != 128)) return false;
+  const int chunk_pages = kChunkTokens / page_size;
+  int sp = 1024 / page_size;
+  if (sp > 64) sp = 64;                 // the table prefetch holds 64 entries per split
+  const long long target = 8LL * 148;   // enough CTAs to balance uneven lengths
+  auto splits_for = [&](int p) { return (max_pages + p - 1) / p; };
+  while (sp > chunk_pages && static_cast<long long>(num_seqs) * Hkv * splits_for(sp) < target) sp /= 2;
+  if (sp < chunk_pages) sp = chunk_pages;
+  plan->chunk_tokens = kChunkTokens;
+  plan->split_pages = sp;
+  plan->max_splits = splits_for(sp);
+  const size_t rows = static_cast<size_t>(num_seqs) * Hq * plan->max_splits;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  plan->partial_o_offset = 256;
+  plan->partial_lse_offset = up(plan->partial_o_offset + rows * d * sizeof(float));
+  plan->bytes = up(plan->partial_lse_offset + rows * sizeof(float));
+  return true;
+}
+
+}  // namespace ta

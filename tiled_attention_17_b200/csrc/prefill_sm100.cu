@@ -1,0 +1,469 @@
+// Fused, tiled attention forward for sm_100a (B200).
+//
+// O = softmax(scale * Q K^T [+ causal mask]) V computed in one pass over K/V
+// tiles with the online-softmax recurrence, so the score and probability
+// tiles live only in tensor memory and registers and never reach HBM
+// (Gemini 3 Flash kernel-fusion post, sections 1-3; FlashAttention
+// optimisation article, sections 3.1-3.2 and 7.1).
+//
+// CTA = two 128-row query tiles of one (batch, query head) sharing one K/V
+// stream.  Warp roles (320 threads):
+//   warp 0      TMA producer: Q tiles once, then K_j / V_j into a smem ring
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2-5   softmax warpgroup for query tile 0 (one thread per row)
+//   warps 6-9   softmax warpgroup for query tile 1
+// Tensor memory (512 columns): S0 | S1 | O0 | O1.  P (bf16) overwrites the
+// first half of its S tile and feeds the P.V product straight from TMEM.
+//
+// Per K/V tile j the MMA issue order is
+//   O0 += P0 V_j ; S0 = Q0 K_{j+1}^T ; O1 += P1 V_j ; S1 = Q1 K_{j+1}^T
+// so each softmax warpgroup works while the tensor pipe serves the other tile.
+// Softmax follows the recurrence of the article's section 3.2.1: running max
+// m and sum l per row, e^(m_old - m_new) rescaling of l and of the partial O.
+// The O rescale is skipped while the max has not grown by more than 2^8 in
+// exp2 units (the page's "rescale only when the max changes", with a margin);
+// the result is unchanged because numerator and denominator share the stale
+// max.  lse = m * scale + ln(l) is written per row (the row max and
+// normaliser kept for a recomputing backward, kernel-fusion post section 4).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "tiledattn_internal.h"
+
+namespace ta {
+
+constexpr int kBM = 128;      // query rows per tile
+constexpr int kBN = 128;      // keys per tile
+constexpr int kThreads = 320;
+constexpr int kSoftmaxWarp0 = 2;
+constexpr float kRescaleLog2 = 8.0f;   // skip O rescale while max grew by <= 2^8
+
+template <int D>
+struct PrefillLayout {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kChunks = D / 64;              // 64-column (128-byte) swizzle atoms along d
+  static constexpr int kTileBytes = 128 * D * 2;      // one 128-row bf16 tile
+  static constexpr int kChunkBytes = 128 * 128;       // 128 rows x 128 bytes
+  static constexpr int kStages = (D == 128) ? 2 : 3;  // K ring and V ring depth
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + 2 * kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kBar = kV + kStages * kTileBytes;
+  // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2], o_done[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 6;
+  static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base (4 B) + abort flag (4 B)
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;        // slack to align the base to 1024 B
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmS0 = 0, kTmS1 = 128, kTmO0 = 256, kTmO1 = 256 + D;
+};
+
+struct PrefillArgs {
+  __nv_bfloat16* o;
+  float* lse;
+  int B, Hq, Hkv, Nq, Nkv;
+  int n_pairs;       // ceil(Nq / 256)
+  int causal;
+  float scale;       // natural-log scale (for lse)
+  float scale_log2;  // scale * log2(e)
+  unsigned* status;
+};
+
+// Number of K/V tiles query tile [q0, q0+128) must visit (0 if it has no rows
+// or every row is fully masked).
+__device__ __forceinline__ int kv_tiles_for(int q0, const PrefillArgs& a) {
+  if (q0 >= a.Nq) return 0;
+  int kv_end = a.Nkv;
+  if (a.causal) {
+    int last = min(q0 + kBM, a.Nq) - 1;
+    kv_end = min(a.Nkv, last + (a.Nkv - a.Nq) + 1);
+  }
+  return kv_end <= 0 ? 0 : (kv_end + kBN - 1) / kBN;
+}
+
+template <int D>
+__global__ void __maxnreg__(200)
+    prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
+  using L = PrefillLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + L::kQ, sK = sbase + L::kK, sV = sbase + L::kV;
+  const uint32_t bar0 = sbase + L::kBar;
+  auto BAR_Q = [&]() { return bar0; };
+  auto BAR_KF = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto BAR_KE = [&](int s) { return bar0 + 8u * (1 + L::kStages + s); };
+  auto BAR_VF = [&](int s) { return bar0 + 8u * (1 + 2 * L::kStages + s); };
+  auto BAR_VE = [&](int s) { return bar0 + 8u * (1 + 3 * L::kStages + s); };
+  auto BAR_SF = [&](int t) { return bar0 + 8u * (1 + 4 * L::kStages + t); };
+  auto BAR_PR = [&](int t) { return bar0 + 8u * (3 + 4 * L::kStages + t); };
+  auto BAR_OD = [&](int t) { return bar0 + 8u * (5 + 4 * L::kStages + t); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: heavy (late) query pairs first so causal tails are short
+  const int bh_count = a.B * a.Hq;
+  const int pair = a.n_pairs - 1 - static_cast<int>(blockIdx.x) / bh_count;
+  const int bh = static_cast<int>(blockIdx.x) % bh_count;
+  const int b = bh / a.Hq, hq = bh % a.Hq;
+  const int hkv = hq / (a.Hq / a.Hkv);
+  const int q0_0 = pair * 2 * kBM, q0_1 = q0_0 + kBM;
+  const int nt_0 = kv_tiles_for(q0_0, a), nt_1 = kv_tiles_for(q0_1, a);
+  const int n_max = max(nt_0, nt_1);
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    mbar_init(BAR_Q(), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(BAR_KF(s), 1);
+      mbar_init(BAR_KE(s), 1);
+      mbar_init(BAR_VF(s), 1);
+      mbar_init(BAR_VE(s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(BAR_SF(t), 1);
+      mbar_init(BAR_PR(t), 128);
+      mbar_init(BAR_OD(t), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ======================= TMA producer =======================
+    if (lane == 0) {
+      const int zq = b * a.Hq + hq, zk = b * a.Hkv + hkv;
+      const uint32_t qbytes = static_cast<uint32_t>((q0_0 < a.Nq) + (q0_1 < a.Nq)) * L::kTileBytes;
+      mbar_arrive_expect_tx(BAR_Q(), qbytes);
+      for (int t = 0; t < 2; ++t) {
+        const int q0 = t ? q0_1 : q0_0;
+        if (q0 >= a.Nq) continue;
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * 64, q0, zq);
+      }
+      bool ok = true;
+      for (int j = 0; j < n_max && ok; ++j) {
+        const int s = j % L::kStages;
+        const uint32_t ph = (j / L::kStages) & 1u;
+        ok = mbar_wait(BAR_KE(s), ph ^ 1u, a.status, abort_flag);
+        if (!ok) break;
+        mbar_arrive_expect_tx(BAR_KF(s), L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sK + s * L::kTileBytes + c * L::kChunkBytes, &tmK, BAR_KF(s), c * 64, j * kBN, zk);
+        ok = mbar_wait(BAR_VE(s), ph ^ 1u, a.status, abort_flag);
+        if (!ok) break;
+        mbar_arrive_expect_tx(BAR_VF(s), L::kTileBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sV + s * L::kTileBytes + c * L::kChunkBytes, &tmV, BAR_VF(s), c * 64, j * kBN, zk);
+      }
+      // drain: make sure no copy into this CTA's smem is still in flight at exit
+      mbar_wait(BAR_Q(), 0, a.status, abort_flag);
+      for (int j = max(0, n_max - L::kStages); j < n_max; ++j) {
+        const int s = j % L::kStages;
+        const uint32_t ph = (j / L::kStages) & 1u;
+        mbar_wait(BAR_KF(s), ph, a.status, abort_flag);
+        mbar_wait(BAR_VF(s), ph, a.status, abort_flag);
+      }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+      auto tS = [&](int t) { return tmem + (t ? L::kTmS1 : L::kTmS0); };
+      auto tO = [&](int t) { return tmem + (t ? L::kTmO1 : L::kTmO0); };
+
+      // S_t = Q_t K^T over d in 16-wide steps (K-major operands, 128B swizzle)
+      auto issue_qk = [&](int t, int s) {
+        const uint32_t qa = sQ + t * L::kTileBytes;
+        const uint32_t kb = sK + s * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+          mma_ss(tS(t), smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), idesc_qk,
+                 kk > 0);
+        }
+      };
+      // O_t += P_t V over the 128 keys in 16-row steps (P from TMEM, V MN-major)
+      auto issue_pv = [&](int t, int s, bool acc) {
+        const uint32_t vb = sV + s * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_ts(tO(t), tS(t) + kk * 8, smem_desc_sw128(vb + kk * 16 * 128, L::kChunkBytes, 1024), idesc_pv,
+                 (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = mbar_wait(BAR_Q(), 0, a.status, abort_flag);
+      if (ok && n_max > 0) {
+        ok = mbar_wait(BAR_KF(0), 0, a.status, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t)
+            if ((t ? nt_1 : nt_0) > 0) {
+              issue_qk(t, 0);
+              mma_commit(BAR_SF(t));
+            }
+          if (L::kStages < n_max) mma_commit(BAR_KE(0));  // only if a later load reuses stage 0
+        }
+      }
+      for (int j = 0; j < n_max && ok; ++j) {
+        const int s = j % L::kStages;
+        const uint32_t ph = (j / L::kStages) & 1u;
+        const int s1 = (j + 1) % L::kStages;
+        const uint32_t ph1 = ((j + 1) / L::kStages) & 1u;
+        if (!(ok = mbar_wait(BAR_VF(s), ph, a.status, abort_flag))) break;
+        for (int t = 0; t < 2; ++t) {
+          const int ntt = t ? nt_1 : nt_0;
+          if (j >= ntt) continue;
+          if (!(ok = mbar_wait(BAR_PR(t), j & 1u, a.status, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(t, s, j > 0);
+          mma_commit(BAR_OD(t));
+          if (j + 1 < ntt) {
+            if (!(ok = mbar_wait(BAR_KF(s1), ph1, a.status, abort_flag))) break;
+            issue_qk(t, s1);
+            mma_commit(BAR_SF(t));
+          }
+        }
+        if (!ok) break;
+        // release a stage only when a later load will reuse it, so no commit
+        // is left pending on a barrier nobody waits for at exit
+        if (j + L::kStages < n_max) mma_commit(BAR_VE(s));
+        if (j + 1 + L::kStages < n_max) mma_commit(BAR_KE(s1));
+      }
+    }
+  } else {
+    // ======================= softmax warpgroups =======================
+    const int t = (warp - kSoftmaxWarp0) / 4;           // query tile of this warpgroup
+    const int quarter = warp & 3;                       // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;                // row within the tile
+    const int q0 = t ? q0_1 : q0_0;                     // first query row of the tile
+    const int qrow = q0 + row;                          // query index
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + (t == 0 ? L::kTmS0 : L::kTmS1) + lane_off;
+    const uint32_t tO = tmem + (t == 0 ? L::kTmO0 : L::kTmO1) + lane_off;
+    const int n = t ? nt_1 : nt_0;
+    const int off = a.Nkv - a.Nq;
+    // visible keys of this row: [0, vis_end)
+    const int vis_end = a.causal ? min(a.Nkv, qrow + off + 1) : a.Nkv;
+    const float c2 = a.scale_log2;
+
+    float m = -INFINITY;  // running max of the raw scores q.k
+    float l = 0.f;        // running sum of exp2((s - m) * c2)
+    bool ok = true;
+
+    for (int j = 0; j < n; ++j) {
+      ok = mbar_wait(BAR_SF(t), j & 1u, a.status, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+      tmem_wait_ld();
+      float* s = reinterpret_cast<float*>(&sr[0][0]);
+
+      // tile-uniform: does any row of this tile have masked keys in tile j?
+      const int kv0 = j * kBN;
+      const bool need_mask =
+          (kv0 + kBN > a.Nkv) || (a.causal && kv0 + kBN - 1 > q0 + off);
+      const int lim = vis_end - kv0;  // visible columns of this tile for this row: [0, lim)
+
+      float mx = -INFINITY;
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, c < lim ? s[c] : -INFINITY);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      }
+      const float m_new = fmaxf(m, mx);
+      const bool upd = (m == -INFINITY) || ((m_new - m) * c2 > kRescaleLog2);
+      const float m_use = upd ? m_new : m;
+      const float alpha = (upd && m != -INFINITY) ? ex2((m - m_use) * c2) : (m == -INFINITY ? 0.f : 1.f);
+      const float neg = (m_use == -INFINITY) ? 0.f : -m_use * c2;
+
+      // P (bf16 pairs) into the first 64 columns of this tile's S region, in
+      // two halves so only one half of the packed values is live at a time
+      float sum = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int c = h * 64 + 2 * i;
+          float p0 = ex2(fmaf(s[c], c2, neg));
+          float p1 = ex2(fmaf(s[c + 1], c2, neg));
+          if (need_mask) {
+            p0 = c < lim ? p0 : 0.f;
+            p1 = c + 1 < lim ? p1 : 0.f;
+          }
+          sum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + h * 32, pk);
+      }
+      l = alpha * l + sum;
+      m = m_use;
+
+      if (j > 0) {
+        // the previous P.V must have landed before O is rescaled
+        ok = mbar_wait(BAR_OD(t), (j - 1) & 1u, a.status, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(tO + c * 32, orr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+            tmem_st32(tO + c * 32, orr);
+          }
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR_PR(t));
+    }
+
+    // ---- epilogue: O / l -> bf16, lse = m * scale + ln(l)
+    const bool have = (n > 0) && ok;
+    if (have) {
+      ok = mbar_wait(BAR_OD(t), (n - 1) & 1u, a.status, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+    }
+    const bool store = qrow < a.Nq;
+    const size_t orow = (static_cast<size_t>(b) * a.Hq + hq) * a.Nq + qrow;
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    __nv_bfloat16* optr = a.o + orow * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t orr[32];
+      if (have && ok) {
+        tmem_ld32(tO + c * 32, orr);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) orr[e] = 0u;
+      }
+      if (store) {
+        uint4* dst = reinterpret_cast<uint4*>(optr + c * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(orr[8 * e + 0]) * inv, __uint_as_float(orr[8 * e + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(orr[8 * e + 2]) * inv, __uint_as_float(orr[8 * e + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(orr[8 * e + 4]) * inv, __uint_as_float(orr[8 * e + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(orr[8 * e + 6]) * inv, __uint_as_float(orr[8 * e + 7]) * inv);
+          dst[e] = w;
+        }
+      }
+    }
+    if (store && a.lse) {
+      a.lse[orow] = (l > 0.f) ? fmaf(m, a.scale, __log2f(l) * 0.69314718055994531f) : -INFINITY;
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// Output for shapes with no keys at all: O = 0, lse = -inf.
+__global__ void empty_keys_kernel(__nv_bfloat16* o, float* lse, size_t rows, int d) {
+  const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (i < rows * d) o[i] = __float2bfloat16(0.f);
+  if (lse && i < rows) lse[i] = -INFINITY;
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+static bool encode_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
+  PFN_encodeTiled enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slices)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+static ta_status launch_prefill_d(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                                  int Hkv, int Nq, int Nkv, float scale, int causal, cudaStream_t stream) {
+  using L = PrefillLayout<D>;
+  CUtensorMap tq, tk, tv;
+  if (!encode_3d(&tq, q, D, Nq, B * Hq) || !encode_3d(&tk, k, D, Nkv, B * Hkv) ||
+      !encode_3d(&tv, v, D, Nkv, B * Hkv))
+    return TA_ERR_CUDA;
+  static int attr_done[64] = {0};
+  if (ensure_smem_limit(prefill_fwd_kernel<D>, L::kAlloc, attr_done) != cudaSuccess) return TA_ERR_CUDA;
+  PrefillArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nq = Nq;
+  a.Nkv = Nkv;
+  a.n_pairs = (Nq + 2 * kBM - 1) / (2 * kBM);
+  a.causal = causal;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.status = device_status_ptr();
+  if (!a.status) return TA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(a.n_pairs) * static_cast<unsigned>(B * Hq);
+  prefill_fwd_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? TA_OK : TA_ERR_CUDA;
+}
+
+ta_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                         int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream) {
+  if (B == 0 || Nq == 0) return TA_OK;
+  if (Nkv == 0) {
+    const size_t rows = static_cast<size_t>(B) * Hq * Nq;
+    const size_t n = rows * d;
+    empty_keys_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+        static_cast<__nv_bfloat16*>(o), lse, rows, d);
+    return cudaGetLastError() == cudaSuccess ? TA_OK : TA_ERR_CUDA;
+  }
+  if (d == 128) return launch_prefill_d<128>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, stream);
+  return launch_prefill_d<64>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, stream);
+}
+
+}  // namespace ta

@@ -1,0 +1,56 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "tiledattn.h"
+
+namespace ta {
+
+using PFN_encodeTiled = PFN_cuTensorMapEncodeTiled_v12000;
+
+// cuTensorMapEncodeTiled fetched through the runtime (no libcuda link).
+PFN_encodeTiled get_encode_tiled();
+
+// Device address of the library status word on the current device.
+unsigned* device_status_ptr();
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+// `slot` identifies the kernel (each caller passes its own static int array).
+template <typename Kernel>
+inline cudaError_t ensure_smem_limit(Kernel kernel, int bytes, int (&done)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
+  return e;
+}
+
+// Split-KV plan for paged decode (pure host arithmetic).
+struct DecodePlan {
+  int chunk_tokens;   // tokens staged per pipeline step (64)
+  int split_pages;    // pages handled by one CTA
+  int max_splits;     // ceil(max_pages / split_pages)
+  size_t partial_o_offset, partial_lse_offset, bytes;
+};
+bool make_decode_plan(int num_seqs, int Hq, int Hkv, int d, int max_pages, int page_size, DecodePlan* plan);
+
+ta_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                         int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);
+
+ta_status launch_paged_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                              const int32_t* seq_lens, int page_size, int num_seqs, int Hq, int Hkv, int d,
+                              int max_pages, int num_pages_total, float scale, void* o, float* lse, void* workspace,
+                              const DecodePlan& plan, cudaStream_t stream);
+
+ta_status launch_gather_debug(const void* k_cache, const void* v_cache, const int32_t* block_table,
+                              const int32_t* seq_lens, int seq, int hkv, int page_size, int Hkv, int d,
+                              int max_pages, int num_pages_total, void* k_out, void* v_out, cudaStream_t stream);
+
+ta_status launch_selftest_wait(unsigned limit_us, cudaStream_t stream);
+
+}  // namespace ta
