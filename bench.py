@@ -469,7 +469,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-stride", type=int, default=4, help="oracle baseline: every n-th query row")
+    ap.add_argument("--cpu-stride", type=int, default=1, help="oracle baseline: every n-th query row")
     ap.add_argument("--no-clocks", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

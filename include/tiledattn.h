@@ -68,6 +68,13 @@ const char *ta_status_string(ta_status status);
 int ta_version(void);
 
 /*
+ * Description of the last host-side failure on the calling thread (which step
+ * failed and the CUDA error name), or "" if none.  Static thread-local
+ * storage, never NULL; overwritten by the next failure.
+ */
+const char *ta_last_error(void);
+
+/*
  * attn_fwd - fused attention forward (prefill).
  *
  *   q   [B, Hq,  Nq,  d]  bf16     o   [B, Hq, Nq, d] bf16 (written)

@@ -24,15 +24,16 @@ TA_DEV_TIMEOUT = 1
 TA_DEV_BAD_BLOCK_TABLE = 2
 TA_DEV_BAD_SEQ_LEN = 4
 
-EXPORTS = ["ta_status_string", "ta_version", "attn_fwd", "attn_paged_decode_workspace_size",
+EXPORTS = ["ta_status_string", "ta_version", "ta_last_error", "attn_fwd", "attn_paged_decode_workspace_size",
            "attn_paged_decode", "attn_paged_decode_check", "attn_paged_gather_debug",
            "ta_device_status", "ta_selftest_bounded_wait"]
 
 
 class TiledAttnError(RuntimeError):
-    def __init__(self, fn, code):
+    def __init__(self, fn, code, detail=""):
         self.code = code
-        super().__init__(f"{fn} returned {STATUS_NAMES.get(code, code)}")
+        msg = f"{fn} returned {STATUS_NAMES.get(code, code)}"
+        super().__init__(msg + (f": {detail}" if detail else ""))
 
 
 _lib = None
@@ -52,6 +53,7 @@ def load(path: str | None = None):
     L.ta_status_string.argtypes = [i32]
     L.ta_status_string.restype = ctypes.c_char_p
     L.ta_version.restype = i32
+    L.ta_last_error.restype = ctypes.c_char_p
     L.attn_fwd.argtypes = [vp, vp, vp, vp, vp] + [i32] * 6 + [f32, i32, vp]
     L.attn_fwd.restype = i32
     L.attn_paged_decode_workspace_size.argtypes = [i32] * 6
@@ -90,7 +92,7 @@ def _stream(stream):
 
 def _check(fn, code):
     if code != TA_OK:
-        raise TiledAttnError(fn, code)
+        raise TiledAttnError(fn, code, ta_last_error())
 
 
 # ---------------------------------------------------------------------------
@@ -103,6 +105,10 @@ def ta_status_string(code: int) -> str:
 
 def ta_version() -> int:
     return load().ta_version()
+
+
+def ta_last_error() -> str:
+    return load().ta_last_error().decode()
 
 
 def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream=None, check=True) -> int:

@@ -6,6 +6,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <mutex>
 
 #include "ptx.cuh"
@@ -49,6 +50,21 @@ PFN_encodeTiled get_encode_tiled() {
   return fn;
 }
 
+static thread_local char g_last_error[256] = "";
+
+ta_status fail(ta_status code, const char* where, cudaError_t err) {
+  if (err != cudaSuccess)
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", where, cudaGetErrorName(err), cudaGetErrorString(err));
+  else
+    snprintf(g_last_error, sizeof g_last_error, "%s", where);
+  return code;
+}
+
+ta_status fail_cu(ta_status code, const char* where, int cu_result) {
+  snprintf(g_last_error, sizeof g_last_error, "%s: CUresult %d", where, cu_result);
+  return code;
+}
+
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace ta
@@ -70,6 +86,8 @@ const char* ta_status_string(ta_status s) {
 }
 
 int ta_version(void) { return 10000; }
+
+const char* ta_last_error(void) { return g_last_error; }
 
 ta_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
                    int Nkv, int d, float scale, int causal, ta_stream_t stream) {

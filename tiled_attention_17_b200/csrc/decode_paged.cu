@@ -470,19 +470,21 @@ ta_status launch_paged_decode(const void* q, const void* k_cache, const void* v_
                               const DecodePlan& plan, cudaStream_t stream) {
   if (num_seqs == 0) return TA_OK;
   unsigned* status = static_cast<unsigned*>(workspace);
-  if (cudaMemsetAsync(status, 0, sizeof(unsigned), stream) != cudaSuccess) return TA_ERR_CUDA;
+  cudaError_t me = cudaMemsetAsync(status, 0, sizeof(unsigned), stream);
+  if (me != cudaSuccess) return fail(TA_ERR_CUDA, "decode: status reset", me);
   DecodeArgs a = make_args(q, k_cache, v_cache, block_table, seq_lens, page_size, num_seqs, Hq, Hkv, max_pages,
                            num_pages_total, scale, plan.split_pages, plan.max_splits, workspace, &plan, status);
   const int G = Hq / Hkv;
   dim3 grid(plan.max_splits, Hkv, num_seqs);
   cudaError_t e = (d == 128) ? launch_split_g<128>(a, G, grid, stream) : launch_split_g<64>(a, G, grid, stream);
-  if (e != cudaSuccess) return TA_ERR_CUDA;
+  if (e != cudaSuccess) return fail(TA_ERR_CUDA, "decode: split kernel launch", e);
   dim3 cgrid(Hq, num_seqs);
   if (d == 128)
     decode_combine_kernel<128><<<cgrid, 128, 0, stream>>>(a, static_cast<__nv_bfloat16*>(o), lse);
   else
     decode_combine_kernel<64><<<cgrid, 128, 0, stream>>>(a, static_cast<__nv_bfloat16*>(o), lse);
-  return cudaGetLastError() == cudaSuccess ? TA_OK : TA_ERR_CUDA;
+  e = cudaGetLastError();
+  return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "decode: combine kernel launch", e);
 }
 
 ta_status launch_gather_debug(const void* k_cache, const void* v_cache, const int32_t* block_table,

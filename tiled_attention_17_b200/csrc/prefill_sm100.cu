@@ -7,11 +7,16 @@
 // optimisation article, sections 3.1-3.2 and 7.1).
 //
 // CTA = two 128-row query tiles of one (batch, query head) sharing one K/V
-// stream.  Warp roles (320 threads):
+// stream.  Warp roles (384 threads, three warpgroups):
 //   warp 0      TMA producer: Q tiles once, then K_j / V_j into a smem ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2-5   softmax warpgroup for query tile 0 (one thread per row)
-//   warps 6-9   softmax warpgroup for query tile 1
+//   warps 2-3   idle after setup
+//   warps 4-7   softmax warpgroup for query tile 0 (one thread per row)
+//   warps 8-11  softmax warpgroup for query tile 1
+// The block launches at 168 registers per thread (the per-sub-partition
+// register file holds three warps of that size); the first warpgroup then
+// releases registers (setmaxnreg.dec to 56) and the softmax warpgroups take
+// them (setmaxnreg.inc to 224): 128*56 + 256*224 = 384*168.
 // Tensor memory (512 columns): S0 | S1 | O0 | O1.  P (bf16) overwrites the
 // first half of its S tile and feeds the P.V product straight from TMEM.
 //
@@ -38,8 +43,13 @@ namespace ta {
 
 constexpr int kBM = 128;      // query rows per tile
 constexpr int kBN = 128;      // keys per tile
-constexpr int kThreads = 320;
-constexpr int kSoftmaxWarp0 = 2;
+constexpr int kThreads = 384;
+constexpr int kSoftmaxWarp0 = 4;
+constexpr int kLaunchRegs = 168;     // what ptxas must report for this kernel
+constexpr int kRegsControl = 56;     // warpgroup 0 after setmaxnreg.dec
+constexpr int kRegsSoftmax = 224;    // warpgroups 1-2 after setmaxnreg.inc
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
+static_assert(kRegsControl + 2 * kRegsSoftmax <= 512, "per sub-partition: one warp of each warpgroup");
 constexpr float kRescaleLog2 = 8.0f;   // skip O rescale while max grew by <= 2^8
 
 template <int D>
@@ -86,7 +96,7 @@ __device__ __forceinline__ int kv_tiles_for(int q0, const PrefillArgs& a) {
 }
 
 template <int D>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
   using L = PrefillLayout<D>;
@@ -150,9 +160,10 @@ __global__ void __maxnreg__(200)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp < kSoftmaxWarp0) {
+    setmaxnreg_dec<kRegsControl>();
+    if (warp == 0 && lane == 0) {
     // ======================= TMA producer =======================
-    if (lane == 0) {
       const int zq = b * a.Hq + hq, zk = b * a.Hkv + hkv;
       const uint32_t qbytes = static_cast<uint32_t>((q0_0 < a.Nq) + (q0_1 < a.Nq)) * L::kTileBytes;
       mbar_arrive_expect_tx(BAR_Q(), qbytes);
@@ -185,10 +196,8 @@ __global__ void __maxnreg__(200)
         mbar_wait(BAR_KF(s), ph, a.status, abort_flag);
         mbar_wait(BAR_VF(s), ph, a.status, abort_flag);
       }
-    }
-  } else if (warp == 1) {
+    } else if (warp == 1 && lane == 0) {
     // ======================= MMA issuer =======================
-    if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
       auto tS = [&](int t) { return tmem + (t ? L::kTmS1 : L::kTmS0); };
@@ -255,6 +264,7 @@ __global__ void __maxnreg__(200)
       }
     }
   } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ======================= softmax warpgroups =======================
     const int t = (warp - kSoftmaxWarp0) / 4;           // query tile of this warpgroup
     const int quarter = warp & 3;                       // TMEM lane quarter this warp may access
@@ -410,9 +420,9 @@ __global__ void empty_keys_kernel(__nv_bfloat16* o, float* lse, size_t rows, int
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-static bool encode_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
+static ta_status encode_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
   PFN_encodeTiled enc = get_encode_tiled();
-  if (!enc) return false;
+  if (!enc) return fail(TA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slices)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
   cuuint32_t box[3] = {64, 128, 1};
@@ -420,7 +430,7 @@ static bool encode_3d(CUtensorMap* map, const void* base, int d, int rows, int s
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return r == CUDA_SUCCESS ? TA_OK : fail_cu(TA_ERR_CUDA, "cuTensorMapEncodeTiled", static_cast<int>(r));
 }
 
 template <int D>
@@ -428,11 +438,13 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
                                   int Hkv, int Nq, int Nkv, float scale, int causal, cudaStream_t stream) {
   using L = PrefillLayout<D>;
   CUtensorMap tq, tk, tv;
-  if (!encode_3d(&tq, q, D, Nq, B * Hq) || !encode_3d(&tk, k, D, Nkv, B * Hkv) ||
-      !encode_3d(&tv, v, D, Nkv, B * Hkv))
-    return TA_ERR_CUDA;
+  ta_status st;
+  if ((st = encode_3d(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
+  if ((st = encode_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
   static int attr_done[64] = {0};
-  if (ensure_smem_limit(prefill_fwd_kernel<D>, L::kAlloc, attr_done) != cudaSuccess) return TA_ERR_CUDA;
+  cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D>, L::kAlloc, attr_done);
+  if (e != cudaSuccess) return fail(TA_ERR_CUDA, "prefill: shared-memory limit", e);
   PrefillArgs a;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
@@ -446,10 +458,11 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.status = device_status_ptr();
-  if (!a.status) return TA_ERR_CUDA;
+  if (!a.status) return fail(TA_ERR_CUDA, "prefill: device status word");
   const unsigned grid = static_cast<unsigned>(a.n_pairs) * static_cast<unsigned>(B * Hq);
   prefill_fwd_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
-  return cudaGetLastError() == cudaSuccess ? TA_OK : TA_ERR_CUDA;
+  e = cudaGetLastError();
+  return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "prefill: launch", e);
 }
 
 ta_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,

@@ -14,11 +14,16 @@ using PFN_encodeTiled = PFN_cuTensorMapEncodeTiled_v12000;
 // cuTensorMapEncodeTiled fetched through the runtime (no libcuda link).
 PFN_encodeTiled get_encode_tiled();
 
+// Records a description of the last host-side failure of this thread
+// (returned by ta_last_error) and returns `code`.
+ta_status fail(ta_status code, const char* where, cudaError_t err = cudaSuccess);
+ta_status fail_cu(ta_status code, const char* where, int cu_result);
+
 // Device address of the library status word on the current device.
 unsigned* device_status_ptr();
 
 // Raise a kernel's dynamic shared-memory limit once per device.
-// `slot` identifies the kernel (each caller passes its own static int array).
+// `done` is the caller's per-kernel, per-device record.
 template <typename Kernel>
 inline cudaError_t ensure_smem_limit(Kernel kernel, int bytes, int (&done)[64]) {
   int dev = 0;
