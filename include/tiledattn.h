@@ -131,6 +131,35 @@ ta_status attn_paged_decode(const void *q, const void *k_cache, const void *v_ca
                             void *workspace, size_t workspace_bytes, ta_stream_t stream);
 
 /*
+ * attn_paged_decode_noalloc - attn_paged_decode for callers that cannot
+ * allocate device memory.  (The source pages have no counterpart; this is a
+ * library convenience.)  Some callers have no way to obtain a workspace: a
+ * plugin inside a host framework that owns all device memory and passes the
+ * plugin only its inputs and outputs, or code on a latency-critical path where
+ * cudaMalloc's implicit device synchronisation is not acceptable.
+ *
+ * Same arguments, layouts, limits and results as attn_paged_decode, without
+ * `workspace`/`workspace_bytes`: the split partials go to a fixed 64 MiB scratch
+ * array in the library's own device memory (a file-scope __device__ array;
+ * every GPU that loads the library's code holds it until the process exits).
+ * The call allocates nothing.  Sizes whose attn_paged_decode_workspace_size
+ * exceeds 64 MiB return TA_ERR_UNSUPPORTED before anything is enqueued (the
+ * reason is in ta_last_error).  The first call on each device looks up the
+ * scratch array's device address (with that device current) and caches it;
+ * make that first call before any stream capture.  Every call on a device
+ * shares the one array: calls that may overlap on the GPU (different streams,
+ * no ordering between them) race and give wrong results; serialise them.  The
+ * status word that attn_paged_decode_check reads lives in that shared array
+ * and is not exposed for this entry point; bad table entries and lengths are
+ * still clamped on the device.
+ */
+ta_status attn_paged_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                    const int32_t *block_table, const int32_t *seq_lens, int page_size,
+                                    int num_seqs, int Hq, int Hkv, int d, int max_pages,
+                                    int num_pages_total, float scale, void *o, float *lse,
+                                    ta_stream_t stream);
+
+/*
  * Checked mode for paged decode: waits for `stream`, reads the status word the
  * last attn_paged_decode wrote into `workspace`, stores it in *flags (host
  * pointer, may be NULL) and returns TA_ERR_BAD_BLOCK_TABLE or

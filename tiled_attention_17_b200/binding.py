@@ -25,7 +25,7 @@ TA_DEV_BAD_BLOCK_TABLE = 2
 TA_DEV_BAD_SEQ_LEN = 4
 
 EXPORTS = ["ta_status_string", "ta_version", "ta_last_error", "attn_fwd", "attn_paged_decode_workspace_size",
-           "attn_paged_decode", "attn_paged_decode_check", "attn_paged_gather_debug",
+           "attn_paged_decode", "attn_paged_decode_noalloc", "attn_paged_decode_check", "attn_paged_gather_debug",
            "ta_device_status", "ta_selftest_bounded_wait"]
 
 
@@ -60,6 +60,8 @@ def load(path: str | None = None):
     L.attn_paged_decode_workspace_size.restype = sz
     L.attn_paged_decode.argtypes = [vp, vp, vp, vp, vp] + [i32] * 7 + [f32, vp, vp, vp, sz, vp]
     L.attn_paged_decode.restype = i32
+    L.attn_paged_decode_noalloc.argtypes = [vp, vp, vp, vp, vp] + [i32] * 7 + [f32, vp, vp, vp]
+    L.attn_paged_decode_noalloc.restype = i32
     L.attn_paged_decode_check.argtypes = [vp, ctypes.POINTER(u32), vp]
     L.attn_paged_decode_check.restype = i32
     L.attn_paged_gather_debug.argtypes = [vp, vp, vp, vp] + [i32] * 7 + [vp, vp, vp]
@@ -131,6 +133,19 @@ def attn_paged_decode(q, k_cache, v_cache, block_table, seq_lens, page_size, num
                                     _ptr(o), _ptr(lse), _ptr(workspace), int(workspace_bytes), _stream(stream))
     if check:
         _check("attn_paged_decode", code)
+    return code
+
+
+def attn_paged_decode_noalloc(q, k_cache, v_cache, block_table, seq_lens, page_size, num_seqs, Hq, Hkv, d,
+                              max_pages, num_pages_total, scale, o, lse, stream=None, check=True) -> int:
+    """attn_paged_decode without a workspace argument, for callers that cannot
+    allocate device memory: the library uses its own fixed 64 MiB scratch array
+    (shared by all calls on a device; overlapping calls race)."""
+    code = load().attn_paged_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                            _ptr(seq_lens), page_size, num_seqs, Hq, Hkv, d, max_pages,
+                                            num_pages_total, float(scale), _ptr(o), _ptr(lse), _stream(stream))
+    if check:
+        _check("attn_paged_decode_noalloc", code)
     return code
 
 
