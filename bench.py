@@ -460,6 +460,42 @@ def timed(torch, stream, fn, steps):
     return e0.elapsed_time(e1) / steps
 
 
+def run_ncu_case(args):
+    """A small, self-contained case for a profiler capture of one kernel:
+    prefill = the causal workload (about 270 MB on the device); decode = 16
+    sequences with the benchmark's length distribution (about 1.1 GB, larger
+    than L2).  Runs `--reps` launches and exits."""
+    import torch
+    from tiled_attention_17_b200 import binding
+    binding.load()
+    dev = torch.device("cuda", 0)
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    if args.ncu_case == "prefill":
+        c = PREFILL
+        q_h, k_h, v_h = inputs.prefill_inputs(c)
+        q, k, v = dev_bf16(q_h), dev_bf16(k_h), dev_bf16(v_h)
+        o = torch.empty_like(q)
+        lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+        for _ in range(args.reps):
+            binding.attn_fwd(q, k, v, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nkv, c.d, c.scale, 1)
+    else:
+        import dataclasses
+        D = dataclasses.replace(DECODE, num_seqs=16)
+        dinp = inputs.paged_inputs(D)
+        dq, dkc, dvc = dev_bf16(dinp.q), dev_bf16(dinp.k_cache), dev_bf16(dinp.v_cache)
+        dbt = torch.from_numpy(dinp.block_table).to(dev)
+        dsl = torch.from_numpy(dinp.seq_lens).to(dev)
+        ws = None
+        for _ in range(args.reps):
+            _o, _l, ws = binding.paged_decode(dq, dkc, dvc, dbt, dsl, workspace=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"ncu_case": args.ncu_case, "reps": args.reps, "ok": True}))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -471,7 +507,12 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-stride", type=int, default=1, help="oracle baseline: every n-th query row")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--ncu-case", choices=["prefill", "decode"], default=None,
+                    help="run a small single-kernel case for a profiler capture and exit")
+    ap.add_argument("--reps", type=int, default=4)
     args = ap.parse_args(argv)
+    if args.ncu_case:
+        return run_ncu_case(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

@@ -36,9 +36,12 @@
 
 namespace ta {
 
-constexpr int kDecThreads = 128;
-constexpr int kChunkTokens = 64;
-constexpr int kDecStages = 3;
+constexpr int kChunkTokens = 64;           // tokens staged per pipeline step
+constexpr int kDecStages = 3;              // ring depth
+constexpr int kConsumerWarps = 8;          // each owns 8 rows of every chunk
+constexpr int kRowsPerWarp = kChunkTokens / kConsumerWarps;
+constexpr int kSplitThreads = 32 * (kConsumerWarps + 1);   // + one TMA producer warp
+constexpr int kGatherThreads = 128;        // gather-debug kernel
 constexpr int kMaxG = 8;
 
 template <int D>
@@ -47,16 +50,18 @@ struct DecodeLayout {
   static constexpr int kRowBytes = D * 2;
   static constexpr int kChunkBytes = kChunkTokens * kRowBytes;
   static constexpr int kStageBytes = 2 * kChunkBytes;   // K chunk then V chunk
-  static constexpr int kScores = kDecStages * kStageBytes;
-  static constexpr int kAlpha = kScores + kChunkTokens * kMaxG * 4;
-  static constexpr int kM = kAlpha + kMaxG * 4;
-  static constexpr int kL = kM + kMaxG * 4;
-  static constexpr int kBar = kL + kMaxG * 4;
-  static constexpr int kAbort = kBar + kDecStages * 8;
-  static constexpr int kBytes = kAbort + 16;
+  static constexpr int kRing = kDecStages * kStageBytes;
   static constexpr int kLanesPerRow = D / 8;            // 16-byte slices per row
-  static constexpr int kRowGroups = kDecThreads / kLanesPerRow;
-  static_assert(kRowGroups * kMaxG * D * 4 <= kScores, "reduction buffer fits in the ring");
+  static constexpr int kSegs = 32 / kLanesPerRow;       // rows a warp covers per pass
+  static constexpr int kPasses = kRowsPerWarp / kSegs;
+  // end-of-split merge of the per-segment states (reuses the ring's space)
+  static constexpr int kStates = kConsumerWarps * kSegs;
+  template <int G>
+  static constexpr int merge_bytes() { return kStates * G * (D + 2) * 4; }
+  static constexpr int kArea = kRing > kStates * kMaxG * (D + 2) * 4 ? kRing : kStates * kMaxG * (D + 2) * 4;
+  static constexpr int kBar = kArea;                    // full[S], empty[S]
+  static constexpr int kAbort = kBar + 2 * kDecStages * 8;
+  static constexpr int kBytes = kAbort + 16;
 };
 
 struct DecodeArgs {
@@ -125,12 +130,48 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
   }
 }
 
+// Sum each head's partial dot product over the LPR lanes that share a row, so
+// that every lane of the row segment ends with all G totals.  For G = 4 a
+// reduce-scatter followed by an all-gather needs 8 shuffles instead of 16.
+template <int G, int LPR>
+__device__ __forceinline__ void segment_allreduce(float (&v)[G], uint32_t mask, int lane_r) {
+  if constexpr (G == 4) {
+    constexpr int H1 = LPR / 2, H2 = LPR / 4;
+    const bool b1 = lane_r & H1, b2 = lane_r & H2;
+    float k0 = b1 ? v[2] : v[0], k1 = b1 ? v[3] : v[1];
+    const float s0 = b1 ? v[0] : v[2], s1 = b1 ? v[1] : v[3];
+    k0 += __shfl_xor_sync(mask, s0, H1);
+    k1 += __shfl_xor_sync(mask, s1, H1);
+    float x = b2 ? k1 : k0;
+    x += __shfl_xor_sync(mask, b2 ? k0 : k1, H2);
+#pragma unroll
+    for (int o = H2 / 2; o >= 1; o >>= 1) x += __shfl_xor_sync(mask, x, o);
+    // x = total of head (b1 ? 2 : 0) + (b2 ? 1 : 0); gather the other three
+    const float xo = __shfl_xor_sync(mask, x, H2);
+    const float lo = b2 ? xo : x, hi = b2 ? x : xo;
+    const float lo2 = __shfl_xor_sync(mask, lo, H1), hi2 = __shfl_xor_sync(mask, hi, H1);
+    v[0] = b1 ? lo2 : lo;
+    v[1] = b1 ? hi2 : hi;
+    v[2] = b1 ? lo : lo2;
+    v[3] = b1 ? hi : hi2;
+  } else {
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int o = LPR / 2; o >= 1; o >>= 1) v[g] += __shfl_xor_sync(mask, v[g], o);
+  }
+}
+
+constexpr float kDecRescaleLog2 = 8.0f;   // keep a stale max until it is exceeded by 2^8
+
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kSplitThreads, (G <= 4 ? 2 : 1)) decode_split_kernel(const DecodeArgs a) {
   using L = DecodeLayout<D>;
   constexpr int LPR = L::kLanesPerRow;
-  constexpr int RG = L::kRowGroups;
-  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int SEGS = L::kSegs;
+  constexpr int PASSES = L::kPasses;
+  static_assert(L::template merge_bytes<G>() <= L::kArea, "merge area fits");
+  extern __shared__ __align__(1024) uint8_t smem[];
 
   const int split = blockIdx.x, hkv = blockIdx.y, seq = blockIdx.z;
   const int raw_len = __ldg(a.seq_lens + seq);
@@ -147,189 +188,167 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = smem_u32(smem);
-  float* sc = reinterpret_cast<float*>(smem + L::kScores);       // [64][kMaxG] scores, then probabilities
-  float* s_alpha = reinterpret_cast<float*>(smem + L::kAlpha);
-  float* s_m = reinterpret_cast<float*>(smem + L::kM);
-  float* s_l = reinterpret_cast<float*>(smem + L::kL);
-  const uint32_t bar0 = sbase + L::kBar;
+  auto FULL = [&](int s) { return sbase + L::kBar + 8u * s; };
+  auto EMPTY = [&](int s) { return sbase + L::kBar + 8u * (kDecStages + s); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
 
   if (tid == 0) {
-    for (int s = 0; s < kDecStages; ++s) mbar_init(bar0 + 8 * s, 1);
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(FULL(s), 1);
+      mbar_init(EMPTY(s), kConsumerWarps);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
-  // warp 0: prefetch the split's table entries, start the first stages
-  int tbl0 = -1, tbl1 = -1;
-  if (warp == 0) {
-    prefetch_table(a, seq, split_first_page, split_npages, tbl0, tbl1);
-    for (int c = 0; c < min(kDecStages, n_chunks); ++c) {
-      const int first = c * pages_per_chunk;
-      const int npg = min(pages_per_chunk, split_npages - first);
-      const uint32_t st = sbase + c * L::kStageBytes;
-      gather_pages<D>(a, hkv, first, npg, tbl0, tbl1, st, st + L::kChunkBytes, bar0 + 8 * c, a.status);
-    }
-  }
-
-  // this thread's slice of the G query vectors
-  const int lane_r = tid % LPR;   // 16-byte slice of a row
-  const int rg = tid / LPR;       // row group
-  float qf[G][8];
+  // per-segment online-softmax state (a segment = the LPR lanes of one row)
+  const int lane_r = lane % LPR;   // 16-byte slice of a row
+  const int seg = lane / LPR;
+  float m[G], l[G];
+  float2 acc[G][4];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(seq) * a.Hq + hkv * G + g) * D) +
-                          lane_r);
-    unpack8(u, qf[g]);
+    m[g] = -INFINITY;
+    l[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[g][e] = make_float2(0.f, 0.f);
   }
-  float acc[G][8];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-  // running statistics, owned by warp (g % 4) for head g
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-  const float c2 = a.scale_log2;
-  const uint32_t seg_mask = (LPR == 16) ? (0xFFFFu << (lane & 16)) : (0xFFu << (lane & 24));
 
-  int c = 0;
-  for (; c < n_chunks; ++c) {
-    const int stage = c % kDecStages;
-    const uint32_t st = sbase + stage * L::kStageBytes;
-    const uint8_t* sK = smem + stage * L::kStageBytes;
-    const uint8_t* sV = sK + L::kChunkBytes;
-    const bool ok = mbar_wait(bar0 + 8 * stage, (c / kDecStages) & 1u, a.status, abort_flag);
-    const int valid = min(kChunkTokens, t_end - (t_begin + c * kChunkTokens));
-
-    // ---- A: scores s[t][g] = q_g . k_t
-    for (int r = rg; r < valid; r += RG) {
-      float kf[8];
-      unpack8(*reinterpret_cast<const uint4*>(sK + r * L::kRowBytes + lane_r * 16), kf);
-      float part[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float s = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) s = fmaf(qf[g][e], kf[e], s);
-        part[g] = s;
-      }
-      if constexpr (G == 4) {
-        // reduce-scatter over the LPR lanes of the row: each lane ends with one head's total
-        const bool hi = lane_r & (LPR / 2);
-        float ka = hi ? part[2] : part[0], kb = hi ? part[3] : part[1];
-        const float sa = hi ? part[0] : part[2], sb = hi ? part[1] : part[3];
-        ka += __shfl_xor_sync(seg_mask, sa, LPR / 2);
-        kb += __shfl_xor_sync(seg_mask, sb, LPR / 2);
-        const bool hi2 = lane_r & (LPR / 4);
-        float x = hi2 ? kb : ka;
-        x += __shfl_xor_sync(seg_mask, hi2 ? ka : kb, LPR / 4);
-#pragma unroll
-        for (int o = LPR / 8; o >= 1; o >>= 1) x += __shfl_xor_sync(seg_mask, x, o);
-        if ((lane_r & (LPR / 4 - 1)) == 0) sc[r * kMaxG + (hi ? 2 : 0) + (hi2 ? 1 : 0)] = x;
-      } else {
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int o = LPR / 2; o >= 1; o >>= 1) part[g] += __shfl_xor_sync(seg_mask, part[g], o);
-        if (lane_r == 0) {
-#pragma unroll
-          for (int g = 0; g < G; ++g) sc[r * kMaxG + g] = part[g];
-        }
-      }
+  if (warp == kConsumerWarps) {
+    // ======================= producer warp =======================
+    int tbl0, tbl1;
+    prefetch_table(a, seq, split_first_page, split_npages, tbl0, tbl1);   // index prefetch
+    int c = 0;
+    for (; c < n_chunks; ++c) {
+      const int stage = c % kDecStages;
+      bool ok = mbar_wait(EMPTY(stage), ((c / kDecStages) & 1u) ^ 1u, a.status, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int first = c * pages_per_chunk;
+      const int npg = min(pages_per_chunk, split_npages - first);
+      const uint32_t st = sbase + stage * L::kStageBytes;
+      gather_pages<D>(a, hkv, first, npg, tbl0, tbl1, st, st + L::kChunkBytes, FULL(stage), a.status);
     }
-    if (__syncthreads_or(!ok)) break;
-
-    // ---- B: online softmax per head (warp g % 4 owns head g)
-#pragma unroll
-    for (int gi = 0; gi < 2; ++gi) {
-      const int g = warp + 4 * gi;
-      if (g < G) {
-        const float x0 = lane < valid ? sc[lane * kMaxG + g] : -INFINITY;
-        const float x1 = lane + 32 < valid ? sc[(lane + 32) * kMaxG + g] : -INFINITY;
-        float mx = fmaxf(x0, x1);
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float m_new = fmaxf(m_r[gi], mx);
-        const float alpha = (m_r[gi] == -INFINITY) ? 0.f : ex2((m_r[gi] - m_new) * c2);
-        const float p0 = lane < valid ? ex2((x0 - m_new) * c2) : 0.f;
-        const float p1 = lane + 32 < valid ? ex2((x1 - m_new) * c2) : 0.f;
-        sc[lane * kMaxG + g] = p0;
-        sc[(lane + 32) * kMaxG + g] = p1;
-        float ps = p0 + p1;
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-        l_r[gi] = alpha * l_r[gi] + ps;
-        m_r[gi] = m_new;
-        if (lane == 0) s_alpha[g] = alpha;
-      }
-    }
-    __syncthreads();
-
-    // ---- C: acc = alpha * acc + sum_t p_t v_t
+    // drain: no copy into this CTA's shared memory may be in flight at exit
+    if (lane == 0)
+      for (int cc = max(0, c - kDecStages); cc < c; ++cc)
+        mbar_wait(FULL(cc % kDecStages), (cc / kDecStages) & 1u, nullptr, nullptr, kWaitLimitNs);
+  } else {
+    // ======================= consumer warps =======================
+    const uint32_t seg_mask = (LPR == 32 ? 0xffffffffu : ((1u << LPR) - 1u) << (seg * LPR));
+    float2 qf[G][4];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float al = s_alpha[g];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[g][e] *= al;
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(seq) * a.Hq + hkv * G + g) * D) +
+                            lane_r);
+      qf[g][0] = bf16x2_to_f2(u.x);
+      qf[g][1] = bf16x2_to_f2(u.y);
+      qf[g][2] = bf16x2_to_f2(u.z);
+      qf[g][3] = bf16x2_to_f2(u.w);
     }
-    for (int r = rg; r < valid; r += RG) {
-      float vf[8];
-      unpack8(*reinterpret_cast<const uint4*>(sV + r * L::kRowBytes + lane_r * 16), vf);
-      float p[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) p[g] = sc[r * kMaxG + g];
-#pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(p[g], vf[e], acc[g][e]);
-    }
-    __syncthreads();  // stage and score buffer free
+    const float c2 = a.scale_log2;
+    const float thr = c2 > 0.f ? kDecRescaleLog2 / c2 : INFINITY;   // raw-score margin for a stale max
 
-    if (warp == 0 && c + kDecStages < n_chunks) {
-      const int cn = c + kDecStages;
-      const int first = cn * pages_per_chunk;
-      const int npg = min(pages_per_chunk, split_npages - first);
-      gather_pages<D>(a, hkv, first, npg, tbl0, tbl1, st, st + L::kChunkBytes, bar0 + 8 * stage, a.status);
+    for (int c = 0; c < n_chunks; ++c) {
+      const int stage = c % kDecStages;
+      bool ok = mbar_wait(FULL(stage), (c / kDecStages) & 1u, a.status, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const uint8_t* sK = smem + stage * L::kStageBytes;
+      const uint8_t* sV = sK + L::kChunkBytes;
+      const int valid = min(kChunkTokens, t_end - (t_begin + c * kChunkTokens));
+#pragma unroll
+      for (int p = 0; p < PASSES; ++p) {
+        const int row0 = warp * kRowsPerWarp + p * SEGS;
+        if (row0 >= valid) break;                          // warp-uniform
+        const int row = row0 + seg;
+        const bool rv = row < valid;
+        // ---- q . k for the G heads (16-byte slice per lane), summed over the row's lanes
+        const uint4 ku = *reinterpret_cast<const uint4*>(sK + row * L::kRowBytes + lane_r * 16);
+        const float2 k0 = bf16x2_to_f2(ku.x), k1 = bf16x2_to_f2(ku.y);
+        const float2 k2 = bf16x2_to_f2(ku.z), k3 = bf16x2_to_f2(ku.w);
+        float s[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float2 t = fmul2(qf[g][0], k0);
+          t = ffma2(qf[g][1], k1, t);
+          t = ffma2(qf[g][2], k2, t);
+          t = ffma2(qf[g][3], k3, t);
+          s[g] = t.x + t.y;
+        }
+        segment_allreduce<G, LPR>(s, seg_mask, lane_r);
+        // ---- online softmax, per segment, with a stale max kept within 2^8
+        bool need = false;
+#pragma unroll
+        for (int g = 0; g < G; ++g) need |= rv && (m[g] == -INFINITY || s[g] > m[g] + thr);
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            if (rv && (m[g] == -INFINITY || s[g] > m[g] + thr)) {
+              const float alpha = (m[g] == -INFINITY) ? 0.f : ex2((m[g] - s[g]) * c2);
+              l[g] *= alpha;
+              const float2 al = make_float2(alpha, alpha);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[g][e] = fmul2(acc[g][e], al);
+              m[g] = s[g];
+            }
+          }
+        }
+        if (rv) {
+          const uint4 vu = *reinterpret_cast<const uint4*>(sV + row * L::kRowBytes + lane_r * 16);
+          const float2 v0 = bf16x2_to_f2(vu.x), v1 = bf16x2_to_f2(vu.y);
+          const float2 v2 = bf16x2_to_f2(vu.z), v3 = bf16x2_to_f2(vu.w);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float pg = ex2(fmaf(s[g], c2, -m[g] * c2));
+            l[g] += pg;
+            const float2 p2 = make_float2(pg, pg);
+            acc[g][0] = ffma2(p2, v0, acc[g][0]);
+            acc[g][1] = ffma2(p2, v1, acc[g][1]);
+            acc[g][2] = ffma2(p2, v2, acc[g][2]);
+            acc[g][3] = ffma2(p2, v3, acc[g][3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(EMPTY(stage));
     }
   }
+  __syncthreads();   // ring no longer in use (the producer drained its copies)
 
-  if (c < n_chunks) {
-    // a wait gave up: drain what may still be in flight, then leave
-    if (tid == 0) {
-      for (int cc = c; cc < min(n_chunks, c + kDecStages); ++cc)
-        mbar_wait(bar0 + 8 * (cc % kDecStages), (cc / kDecStages) & 1u, nullptr, nullptr, kWaitLimitNs);
-    }
-    __syncthreads();
-    return;
-  }
-
-  // ---- reduce the row groups' partial outputs, normalise, write the split's partials
-  float* red = reinterpret_cast<float*>(smem);
+  // ---- merge the per-segment states by log-sum-exp and write the split's partials
+  float* ms = reinterpret_cast<float*>(smem);                 // [kStates][G] maxima
+  float* ls = ms + L::kStates * G;                            // [kStates][G] sums
+  float* os = ls + L::kStates * G;                            // [kStates][G][D] outputs
+  if (warp < kConsumerWarps) {
+    const int st = warp * SEGS + seg;
 #pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) red[(rg * G + g) * D + lane_r * 8 + e] = acc[g][e];
-#pragma unroll
-  for (int gi = 0; gi < 2; ++gi) {
-    const int g = warp + 4 * gi;
-    if (g < G && lane == 0) {
-      s_m[g] = m_r[gi];
-      s_l[g] = l_r[gi];
+    for (int g = 0; g < G; ++g) {
+      if (lane_r == 0) {
+        ms[st * G + g] = m[g];
+        ls[st * G + g] = l[g];
+      }
+      float* dst = os + (static_cast<size_t>(st) * G + g) * D + lane_r * 8;
+      reinterpret_cast<float4*>(dst)[0] = make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
+      reinterpret_cast<float4*>(dst)[1] = make_float4(acc[g][2].x, acc[g][2].y, acc[g][3].x, acc[g][3].y);
     }
   }
   __syncthreads();
+  if (*abort_flag) return;
+  const float c2 = a.scale_log2;
   const size_t row0 = (static_cast<size_t>(seq) * a.Hq + hkv * G) * a.max_splits + split;
-  for (int idx = tid; idx < G * D; idx += kDecThreads) {
+  for (int idx = tid; idx < G * D; idx += kSplitThreads) {
     const int g = idx / D, col = idx % D;
-    float s = 0.f;
-#pragma unroll 4
-    for (int r = 0; r < RG; ++r) s += red[(r * G + g) * D + col];
-    a.part_o[(row0 + static_cast<size_t>(g) * a.max_splits) * D + col] = s / s_l[g];
-  }
-  if (tid < G) {
-    a.part_lse[row0 + static_cast<size_t>(tid) * a.max_splits] =
-        fmaf(s_m[tid], a.scale, __logf(s_l[tid]));
+    float M = -INFINITY;
+    for (int e = 0; e < L::kStates; ++e) M = fmaxf(M, ms[e * G + g]);
+    float tot = 0.f, o = 0.f;
+    for (int e = 0; e < L::kStates; ++e) {
+      const float me = ms[e * G + g];
+      const float w = (me == -INFINITY) ? 0.f : ex2((me - M) * c2);
+      tot = fmaf(w, ls[e * G + g], tot);
+      o = fmaf(w, os[(static_cast<size_t>(e) * G + g) * D + col], o);
+    }
+    a.part_o[(row0 + static_cast<size_t>(g) * a.max_splits) * D + col] = o / tot;
+    if (col == 0) a.part_lse[row0 + static_cast<size_t>(g) * a.max_splits] = fmaf(M, a.scale, __logf(tot));
   }
 }
 
@@ -361,7 +380,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a,
 
 // Gather-debug: same gather routine, result written out contiguously.
 template <int D>
-__global__ void __launch_bounds__(kDecThreads) gather_debug_kernel(const DecodeArgs a, int seq, int hkv,
+__global__ void __launch_bounds__(kGatherThreads) gather_debug_kernel(const DecodeArgs a, int seq, int hkv,
                                                                    __nv_bfloat16* k_out, __nv_bfloat16* v_out) {
   using L = DecodeLayout<D>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -393,7 +412,7 @@ __global__ void __launch_bounds__(kDecThreads) gather_debug_kernel(const DecodeA
       const int t0 = (g0 + first) * a.page_size;
       const int rows = min(npg * a.page_size, len - t0);
       const int words = rows * D / 8;   // 16-byte words
-      for (int w = tid; w < words; w += kDecThreads) {
+      for (int w = tid; w < words; w += kGatherThreads) {
         reinterpret_cast<uint4*>(k_out + static_cast<size_t>(t0) * D)[w] = reinterpret_cast<const uint4*>(smem)[w];
         reinterpret_cast<uint4*>(v_out + static_cast<size_t>(t0) * D)[w] =
             reinterpret_cast<const uint4*>(smem + L::kChunkBytes)[w];
@@ -450,7 +469,7 @@ static cudaError_t launch_split(const DecodeArgs& a, dim3 grid, cudaStream_t str
   static int attr_done[64] = {0};
   cudaError_t e = ensure_smem_limit(decode_split_kernel<D, G>, L::kBytes, attr_done);
   if (e != cudaSuccess) return e;
-  decode_split_kernel<D, G><<<grid, kDecThreads, L::kBytes, stream>>>(a);
+  decode_split_kernel<D, G><<<grid, kSplitThreads, L::kBytes, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -498,12 +517,12 @@ ta_status launch_gather_debug(const void* k_cache, const void* v_cache, const in
   if (d == 128) {
     if (ensure_smem_limit(gather_debug_kernel<128>, DecodeLayout<128>::kBytes, done128) != cudaSuccess)
       return TA_ERR_CUDA;
-    gather_debug_kernel<128><<<1, kDecThreads, DecodeLayout<128>::kBytes, stream>>>(
+    gather_debug_kernel<128><<<1, kGatherThreads, DecodeLayout<128>::kBytes, stream>>>(
         a, seq, hkv, static_cast<__nv_bfloat16*>(k_out), static_cast<__nv_bfloat16*>(v_out));
   } else {
     if (ensure_smem_limit(gather_debug_kernel<64>, DecodeLayout<64>::kBytes, done64) != cudaSuccess)
       return TA_ERR_CUDA;
-    gather_debug_kernel<64><<<1, kDecThreads, DecodeLayout<64>::kBytes, stream>>>(
+    gather_debug_kernel<64><<<1, kGatherThreads, DecodeLayout<64>::kBytes, stream>>>(
         a, seq, hkv, static_cast<__nv_bfloat16*>(k_out), static_cast<__nv_bfloat16*>(v_out));
   }
   return cudaGetLastError() == cudaSuccess ? TA_OK : TA_ERR_CUDA;

@@ -35,6 +35,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "ptx.cuh"
 #include "tiledattn_internal.h"
@@ -51,6 +52,11 @@ constexpr int kRegsSoftmax = 224;    // warpgroups 1-2 after setmaxnreg.inc
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
 static_assert(kRegsControl + 2 * kRegsSoftmax <= 512, "per sub-partition: one warp of each warpgroup");
 constexpr float kRescaleLog2 = 8.0f;   // skip O rescale while max grew by <= 2^8
+// Column pairs whose index i has bit (i % 8) set in kPolyMask compute 2^x on
+// the FMA pipe instead of the MUFU unit (3 of every 8 pairs): the two softmax
+// warpgroups of an SM would otherwise need as many MUFU cycles as the tensor
+// pipe needs for the four MMAs of a K/V tile.
+constexpr unsigned kPolyMask = 0x52u;   // pairs 1, 4, 6 of each group of 8
 
 template <int D>
 struct PrefillLayout {
@@ -63,8 +69,9 @@ struct PrefillLayout {
   static constexpr int kK = kQ + 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kBar = kV + kStages * kTileBytes;
-  // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2], o_done[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 6;
+  // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2], o_done[2],
+  // p_half[2] (first 64 keys of P written)
+  static constexpr int kNumBars = 1 + 4 * kStages + 8;
   static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base (4 B) + abort flag (4 B)
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;        // slack to align the base to 1024 B
@@ -113,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto BAR_SF = [&](int t) { return bar0 + 8u * (1 + 4 * L::kStages + t); };
   auto BAR_PR = [&](int t) { return bar0 + 8u * (3 + 4 * L::kStages + t); };
   auto BAR_OD = [&](int t) { return bar0 + 8u * (5 + 4 * L::kStages + t); };
+  auto BAR_PH = [&](int t) { return bar0 + 8u * (7 + 4 * L::kStages + t); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -142,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(BAR_SF(t), 1);
       mbar_init(BAR_PR(t), 128);
       mbar_init(BAR_OD(t), 1);
+      mbar_init(BAR_PH(t), 128);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -203,23 +212,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto tS = [&](int t) { return tmem + (t ? L::kTmS1 : L::kTmS0); };
       auto tO = [&](int t) { return tmem + (t ? L::kTmO1 : L::kTmO0); };
 
+      // Shared-memory descriptors are built once; a K step or a ring stage
+      // only moves the start-address field (address >> 4), so the issue loop
+      // adds compile-time offsets instead of rebuilding descriptors.
+      const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dK = smem_desc_sw128(sK, 16, 1024);
+      const uint64_t dV = smem_desc_sw128(sV, L::kChunkBytes, 1024);
+      constexpr uint64_t kTileStep = L::kTileBytes >> 4;
+
       // S_t = Q_t K^T over d in 16-wide steps (K-major operands, 128B swizzle)
       auto issue_qk = [&](int t, int s) {
-        const uint32_t qa = sQ + t * L::kTileBytes;
-        const uint32_t kb = sK + s * L::kTileBytes;
+        uint64_t a0 = dQ + static_cast<uint64_t>(t) * kTileStep;
+        uint64_t b0 = dK + static_cast<uint64_t>(s) * kTileStep;
+        const uint32_t d = tS(t);
+        // 16-element K steps: +32 B within a 128-byte swizzle row, then the next 64-column chunk
+#pragma unroll 1
+        for (int c = 0; c < L::kChunks; ++c) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-          mma_ss(tS(t), smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), idesc_qk,
-                 kk > 0);
+          for (int k4 = 0; k4 < 4; ++k4)
+            mma_ss(d, a0 + 2 * k4, b0 + 2 * k4, idesc_qk, (c | k4) != 0);
+          a0 += L::kChunkBytes >> 4;
+          b0 += L::kChunkBytes >> 4;
         }
       };
-      // O_t += P_t V over the 128 keys in 16-row steps (P from TMEM, V MN-major)
-      auto issue_pv = [&](int t, int s, bool acc) {
-        const uint32_t vb = sV + s * L::kTileBytes;
+      // O_t += P_t V over one half (64 keys) of the tile in 16-row steps
+      // (P from TMEM, V MN-major)
+      auto issue_pv_half = [&](int t, int s, int half, bool acc) {
+        const uint64_t b0 = dV + static_cast<uint64_t>(s) * kTileStep;
+        const uint32_t d = tO(t), a = tS(t);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(tO(t), tS(t) + kk * 8, smem_desc_sw128(vb + kk * 16 * 128, L::kChunkBytes, 1024), idesc_pv,
+        for (int k4 = 0; k4 < kBN / 32; ++k4) {
+          const int kk = half * (kBN / 32) + k4;
+          mma_ts(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
                  (acc || kk > 0) ? 1u : 0u);
         }
       };
@@ -246,9 +270,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t) {
           const int ntt = t ? nt_1 : nt_0;
           if (j >= ntt) continue;
+          if (!(ok = mbar_wait(BAR_PH(t), j & 1u, a.status, abort_flag))) break;
+          tc_fence_after();
+          issue_pv_half(t, s, 0, j > 0);
           if (!(ok = mbar_wait(BAR_PR(t), j & 1u, a.status, abort_flag))) break;
           tc_fence_after();
-          issue_pv(t, s, j > 0);
+          issue_pv_half(t, s, 1, true);
           mma_commit(BAR_OD(t));
           if (j + 1 < ntt) {
             if (!(ok = mbar_wait(BAR_KF(s1), ph1, a.status, abort_flag))) break;
@@ -300,62 +327,99 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool need_mask =
           (kv0 + kBN > a.Nkv) || (a.causal && kv0 + kBN - 1 > q0 + off);
       const int lim = vis_end - kv0;  // visible columns of this tile for this row: [0, lim)
-
-      float mx = -INFINITY;
       if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, c < lim ? s[c] : -INFINITY);
-      } else {
+        for (int c = 0; c < 128; ++c) s[c] = c < lim ? s[c] : -INFINITY;
+      }
+
+      // exp2((s - m) * c2) for 32 column pairs [64h, 64h + 64), packed to bf16
+      // pairs; masked columns get exactly 0.  Returns the sum of the values.
+      // The masked form is a separate specialisation so unmasked tiles carry
+      // no per-element compare/select.
+      auto exp_half = [&](auto masked, int h, float negm, uint32_t (&pk)[32]) -> float {
+        constexpr bool kMasked = decltype(masked)::value;
+        const float2 c2v = make_float2(c2, c2), negv = make_float2(negm, negm);
+        float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int i = 0; i < 32; ++i) {
+          const int c = h * 64 + 2 * i;
+          const float2 x = ffma2(make_float2(s[c], s[c + 1]), c2v, negv);
+          float2 pp;
+          if ((kPolyMask >> (i & 7)) & 1u) {
+            pp = exp2_poly2(x);
+          } else {
+            pp.x = ex2(x.x);
+            pp.y = ex2(x.y);
+          }
+          if constexpr (kMasked) {
+            pp.x = c < lim ? pp.x : 0.f;
+            pp.y = c + 1 < lim ? pp.y : 0.f;
+          }
+          if (i & 1) sb = fadd2(sb, pp); else sa = fadd2(sa, pp);
+          pk[i] = pack_bf16x2(pp.x, pp.y);
+        }
+        return (sa.x + sb.x) + (sa.y + sb.y);
+      };
+      auto exp_half_any = [&](int h, float negm, uint32_t (&pk)[32]) -> float {
+        return need_mask ? exp_half(std::true_type{}, h, negm, pk) : exp_half(std::false_type{}, h, negm, pk);
+      };
+
+      // row max of the tile, then the running max with a stale-max margin:
+      // the max is only moved (and O rescaled) when it grows by more than
+      // 2^8 in exp2 units; weights stay below 2^8 either way.
+      float mx;
+      {
+        float r0 = -INFINITY, r1 = -INFINITY, r2 = -INFINITY, r3 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 8) {
+          r0 = fmax3(r0, s[c + 0], s[c + 1]);
+          r1 = fmax3(r1, s[c + 2], s[c + 3]);
+          r2 = fmax3(r2, s[c + 4], s[c + 5]);
+          r3 = fmax3(r3, s[c + 6], s[c + 7]);
+        }
+        mx = fmaxf(fmax3(r0, r1, r2), r3);
       }
       const float m_new = fmaxf(m, mx);
       const bool upd = (m == -INFINITY) || ((m_new - m) * c2 > kRescaleLog2);
       const float m_use = upd ? m_new : m;
       const float alpha = (upd && m != -INFINITY) ? ex2((m - m_use) * c2) : (m == -INFINITY ? 0.f : 1.f);
-      const float neg = (m_use == -INFINITY) ? 0.f : -m_use * c2;
-
-      // P (bf16 pairs) into the first 64 columns of this tile's S region, in
-      // two halves so only one half of the packed values is live at a time
-      float sum = 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int c = h * 64 + 2 * i;
-          float p0 = ex2(fmaf(s[c], c2, neg));
-          float p1 = ex2(fmaf(s[c + 1], c2, neg));
-          if (need_mask) {
-            p0 = c < lim ? p0 : 0.f;
-            p1 = c + 1 < lim ? p1 : 0.f;
-          }
-          sum += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + h * 32, pk);
-      }
-      l = alpha * l + sum;
+      const float negm = (m_use == -INFINITY) ? 0.f : -m_use * c2;
       m = m_use;
 
-      if (j > 0) {
-        // the previous P.V must have landed before O is rescaled
-        ok = mbar_wait(BAR_OD(t), (j - 1) & 1u, a.status, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      // Rescale O before any of this tile's P.V lands on it.  The previous
+      // P.V has completed: the commit that signalled this S tile was issued
+      // after it and covers every earlier MMA.
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t orr[32];
-            tmem_ld32(tO + c * 32, orr);
-            tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(tO + c * 32, orr);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-            tmem_st32(tO + c * 32, orr);
-          }
+          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+          tmem_st32(tO + c * 32, orr);
         }
       }
+
+      // P (bf16 pairs) into the first 64 columns of this tile's S region, one
+      // half (64 keys) at a time; the MMA warp starts P.V on the first half
+      // while the second is computed.
+      float psum;
+      {
+        uint32_t pk[32];
+        psum = exp_half_any(0, negm, pk);
+        tmem_st32(tS, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR_PH(t));
+      {
+        uint32_t pk[32];
+        psum += exp_half_any(1, negm, pk);
+        tmem_st32(tS + 32, pk);
+      }
+      l = alpha * l + psum;
+
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR_PR(t));
