@@ -352,6 +352,314 @@ __global__ void __launch_bounds__(kSplitThreads, (G <= 4 ? 2 : 1)) decode_split_
   }
 }
 
+// ---------------------------------------------------------------------------
+// Specialised split kernel for head dim 128 with 4 query heads per KV head
+// (the common GQA shape).  Same work decomposition and results as
+// decode_split_kernel, restructured to cut instructions per gathered byte:
+//  * 8 warps, no dedicated producer: the last warp to finish a ring stage
+//    (an acquire-release counter in shared memory) issues the stage's next
+//    page copies, so every warp computes;
+//  * each 16-lane row segment accumulates the partial q.k of its 4 rows of a
+//    chunk before reducing: one reduce-scatter of 16 values leaves each lane
+//    with exactly one (row, head) score, so each lane computes one
+//    exponential per chunk and the stale-max check runs once per chunk;
+//  * probabilities reach the P.V step through shared memory (one store, one
+//    16-byte load per row) instead of shuffles;
+//  * full chunks take a path without per-row validity checks.
+// ---------------------------------------------------------------------------
+constexpr int kG4Warps = 8;
+constexpr int kG4Threads = 32 * kG4Warps;
+
+struct G4Layout {
+  static constexpr int D = 128;
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kChunkBytes = kChunkTokens * kRowBytes;   // 16 KB
+  static constexpr int kStageBytes = 2 * kChunkBytes;            // K then V
+  static constexpr int kRing = kDecStages * kStageBytes;         // 96 KB
+  static constexpr int kStates = kG4Warps * 2;                   // (warp, segment) softmax states
+  static constexpr int kMerge = kStates * 4 * (D + 2) * 4;       // 33 KB, reuses the ring
+  static constexpr int kProb = kRing;                            // [8 warps][2 seg][16] floats
+  static constexpr int kTable = kProb + kG4Warps * 2 * 16 * 4;   // split's block-table entries
+  static constexpr int kBar = kTable + 64 * 4;                   // full[3]
+  static constexpr int kCnt = kBar + kDecStages * 8;             // per-stage finish counters
+  static constexpr int kMisc = kCnt + kDecStages * 4;            // abort flag, issued-chunk count
+  static constexpr int kBytes = kMisc + 16;
+  static_assert(kMerge <= kRing, "merge area fits in the ring");
+};
+
+__device__ __forceinline__ uint32_t atom_add_acq_rel_shared(uint32_t addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Page copies for one chunk, page ids read from the shared-memory table.
+// Warp-wide; lane i < npg copies page i of the chunk.
+__device__ __forceinline__ void gather_chunk_g4(const DecodeArgs& a, int hkv, const int* tbl, int first, int npg,
+                                                uint32_t dstK, uint32_t dstV, uint32_t bar) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t page_bytes = static_cast<uint32_t>(a.page_size) * G4Layout::kRowBytes;
+  if (lane == 0) mbar_arrive_expect_tx(bar, 2u * npg * page_bytes);
+  __syncwarp();
+  if (lane < npg) {
+    const size_t off = (static_cast<size_t>(tbl[first + lane]) * a.Hkv + hkv) * page_bytes;
+    bulk_load(dstK + lane * page_bytes, a.k_cache + off, page_bytes, bar);
+    bulk_load(dstV + lane * page_bytes, a.v_cache + off, page_bytes, bar);
+  }
+}
+
+__global__ void __launch_bounds__(kG4Threads, 2) decode_split_g4_kernel(const DecodeArgs a) {
+  using L = G4Layout;
+  constexpr int D = 128, LPR = 16;
+  extern __shared__ __align__(1024) uint8_t smem[];
+
+  const int split = blockIdx.x, hkv = blockIdx.y, seq = blockIdx.z;
+  const int raw_len = __ldg(a.seq_lens + seq);
+  const int len = clamp_len(raw_len, a);
+  if (raw_len != len && split == 0 && hkv == 0 && threadIdx.x == 0) atomicOr(a.status, kDevBadSeqLen);
+  const int split_tokens = a.split_pages * a.page_size;
+  const int t_begin = split * split_tokens;
+  if (t_begin >= len) return;  // CTA-uniform: nothing in this split
+  const int t_end = min(len, t_begin + split_tokens);
+  const int n_chunks = (t_end - t_begin + kChunkTokens - 1) / kChunkTokens;
+  const int split_first_page = split * a.split_pages;
+  const int split_npages = (t_end - t_begin + a.page_size - 1) / a.page_size;
+  const int pages_per_chunk = kChunkTokens / a.page_size;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int seg = lane >> 4, lane_r = lane & 15;
+  const uint32_t sbase = smem_u32(smem);
+  int* tbl = reinterpret_cast<int*>(smem + L::kTable);
+  float* sp = reinterpret_cast<float*>(smem + L::kProb) + (warp * 2 + seg) * 16;   // this segment's 16 weights
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
+  int* issued = reinterpret_cast<int*>(smem + L::kMisc + 4);   // chunks whose copies were issued
+  auto FULL = [&](int s) { return sbase + L::kBar + 8u * s; };
+  auto CNT = [&](int s) { return sbase + L::kCnt + 4u * s; };
+
+  // index prefetch: the split's block-table entries, checked once
+  if (tid == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(FULL(s), 1);
+      reinterpret_cast<volatile uint32_t*>(smem + L::kCnt)[s] = 0;
+    }
+    *abort_flag = 0;
+    *issued = min(kDecStages, n_chunks);
+    fence_mbar_init();
+  }
+  if (tid < split_npages) {
+    int pg = __ldg(a.block_table + static_cast<size_t>(seq) * a.max_pages + split_first_page + tid);
+    if (pg < 0 || pg >= a.num_pages_total) {
+      atomicOr(a.status, kDevBadBlockTable);
+      pg = 0;
+    }
+    tbl[tid] = pg;
+  }
+  __syncthreads();
+  if (warp < kDecStages && warp < n_chunks) {
+    const int first = warp * pages_per_chunk;
+    const uint32_t st = sbase + warp * L::kStageBytes;
+    gather_chunk_g4(a, hkv, tbl, first, min(pages_per_chunk, split_npages - first), st, st + L::kChunkBytes,
+                    FULL(warp));
+  }
+
+  // q slices (16-byte slice lane_r of each of the 4 heads), fp32 pairs
+  float2 qf[4][4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<size_t>(seq) * a.Hq + hkv * 4 + g) * D) +
+                          lane_r);
+    qf[g][0] = bf16x2_to_f2(u.x);
+    qf[g][1] = bf16x2_to_f2(u.y);
+    qf[g][2] = bf16x2_to_f2(u.z);
+    qf[g][3] = bf16x2_to_f2(u.w);
+  }
+  // this lane's softmax state is that of head gh = lane_r & 3 of its segment;
+  // acc holds the segment's partial output for all 4 heads on this d-slice
+  const int gh = lane_r & 3, ph = lane_r >> 2;
+  float m = -INFINITY, negmc = 0.f, l = 0.f;
+  float2 acc[4][4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[g][e] = make_float2(0.f, 0.f);
+  const float c2 = a.scale_log2;
+  const float thr = c2 > 0.f ? kDecRescaleLog2 / c2 : INFINITY;
+  const uint32_t seg_mask = 0xFFFFu << (seg * 16);
+  const int row_base = warp * 8 + seg;   // rows row_base + 2p, p = 0..3
+
+  int c = 0;
+  for (; c < n_chunks; ++c) {
+    const int stage = c % kDecStages;
+    const bool ok = mbar_wait(FULL(stage), (c / kDecStages) & 1u, a.status, abort_flag);
+    if (!__all_sync(0xffffffffu, ok)) break;
+    const int valid = min(kChunkTokens, t_end - (t_begin + c * kChunkTokens));
+    const uint8_t* sK = smem + stage * L::kStageBytes + lane_r * 16;
+    const uint8_t* sV = sK + L::kChunkBytes;
+    if (warp * 8 < valid) {
+      // ---- q . k of this segment's 4 rows, partial over this lane's 8 dims
+      float v[16];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const uint4 ku = *reinterpret_cast<const uint4*>(sK + (row_base + 2 * p) * L::kRowBytes);
+        const float2 k0 = bf16x2_to_f2(ku.x), k1 = bf16x2_to_f2(ku.y);
+        const float2 k2 = bf16x2_to_f2(ku.z), k3 = bf16x2_to_f2(ku.w);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float2 t = fmul2(qf[g][0], k0);
+          t = ffma2(qf[g][1], k1, t);
+          t = ffma2(qf[g][2], k2, t);
+          t = ffma2(qf[g][3], k3, t);
+          v[p * 4 + g] = t.x + t.y;
+        }
+      }
+      // ---- reduce-scatter the 16 (row, head) partials over the 16 lanes:
+      // lane_r ends with the full score of (row p = lane_r >> 2, head lane_r & 3)
+#pragma unroll
+      for (int o = 8, n = 16; o >= 1; o >>= 1, n >>= 1) {
+        const bool hi = lane_r & o;
+#pragma unroll
+        for (int k = 0; k < n / 2; ++k) {
+          const float keep = hi ? v[k + n / 2] : v[k];
+          const float send = hi ? v[k] : v[k + n / 2];
+          v[k] = keep + __shfl_xor_sync(seg_mask, send, o);
+        }
+      }
+      float sc = v[0];
+      if (row_base + 2 * ph >= valid) sc = -INFINITY;
+      // ---- online softmax for head gh over the chunk's 4 rows of this segment
+      float cm = fmaxf(sc, __shfl_xor_sync(seg_mask, sc, 4));
+      cm = fmaxf(cm, __shfl_xor_sync(seg_mask, cm, 8));
+      const bool need = (cm != -INFINITY) && (m == -INFINITY || cm > m + thr);
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ((m == -INFINITY) ? 0.f : ex2((m - cm) * c2)) : 1.f;
+        if (need) {
+          m = cm;
+          negmc = -cm * c2;
+        }
+        l *= alpha;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float ah = __shfl_sync(0xffffffffu, alpha, seg * 16 + h);
+          const float2 a2 = make_float2(ah, ah);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[h][e] = fmul2(acc[h][e], a2);
+        }
+      }
+      const float pv = (sc == -INFINITY) ? 0.f : ex2(fmaf(sc, c2, negmc));
+      l += pv;
+      sp[lane_r] = pv;
+      __syncwarp();
+      // ---- acc += p * v for the 4 rows
+      if (valid == kChunkTokens) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float4 w4 = *reinterpret_cast<const float4*>(sp + 4 * p);
+          const uint4 vu = *reinterpret_cast<const uint4*>(sV + (row_base + 2 * p) * L::kRowBytes);
+          const float2 v0 = bf16x2_to_f2(vu.x), v1 = bf16x2_to_f2(vu.y);
+          const float2 v2 = bf16x2_to_f2(vu.z), v3 = bf16x2_to_f2(vu.w);
+          const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float2 w2 = make_float2(wv[h], wv[h]);
+            acc[h][0] = ffma2(w2, v0, acc[h][0]);
+            acc[h][1] = ffma2(w2, v1, acc[h][1]);
+            acc[h][2] = ffma2(w2, v2, acc[h][2]);
+            acc[h][3] = ffma2(w2, v3, acc[h][3]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          if (row_base + 2 * p < valid) {
+            const float4 w4 = *reinterpret_cast<const float4*>(sp + 4 * p);
+            const uint4 vu = *reinterpret_cast<const uint4*>(sV + (row_base + 2 * p) * L::kRowBytes);
+            const float2 v0 = bf16x2_to_f2(vu.x), v1 = bf16x2_to_f2(vu.y);
+            const float2 v2 = bf16x2_to_f2(vu.z), v3 = bf16x2_to_f2(vu.w);
+            const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float2 w2 = make_float2(wv[h], wv[h]);
+              acc[h][0] = ffma2(w2, v0, acc[h][0]);
+              acc[h][1] = ffma2(w2, v1, acc[h][1]);
+              acc[h][2] = ffma2(w2, v2, acc[h][2]);
+              acc[h][3] = ffma2(w2, v3, acc[h][3]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+    }
+    // ---- release the stage; the last warp to finish it issues its next copies
+    uint32_t last = 0;
+    if (lane == 0) last = (atom_add_acq_rel_shared(CNT(stage), 1u) == kG4Warps - 1) ? 1u : 0u;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      if (lane == 0) reinterpret_cast<volatile uint32_t*>(smem + L::kCnt)[stage] = 0;
+      const int cn = c + kDecStages;
+      if (cn < n_chunks) {
+        fence_proxy_async_shared();   // generic reads of the stage before the async copies into it
+        const int first = cn * pages_per_chunk;
+        const uint32_t st = sbase + stage * L::kStageBytes;
+        gather_chunk_g4(a, hkv, tbl, first, min(pages_per_chunk, split_npages - first), st, st + L::kChunkBytes,
+                        FULL(stage));
+        if (lane == 0) atomicMax(issued, cn + 1);
+      }
+    }
+  }
+  const bool aborted = c < n_chunks;
+  __syncthreads();
+  if (aborted || *abort_flag) {
+    // a wait gave up: let whatever copies may be in flight land, then leave
+    if (tid == 0) {
+      const int hi = *reinterpret_cast<volatile int*>(issued);
+      for (int cc = max(0, hi - kDecStages); cc < hi; ++cc)
+        mbar_wait(FULL(cc % kDecStages), (cc / kDecStages) & 1u, nullptr, nullptr, kWaitLimitNs);
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ---- merge the 16 segment states by log-sum-exp, write the split's partials
+  float* ms = reinterpret_cast<float*>(smem);
+  float* ls = ms + L::kStates * 4;
+  float* os = ls + L::kStates * 4;
+  {
+    const int st = warp * 2 + seg;
+    float lt = l + __shfl_xor_sync(0xffffffffu, l, 4);
+    lt += __shfl_xor_sync(0xffffffffu, lt, 8);
+    if (ph == 0) {
+      ms[st * 4 + gh] = m;
+      ls[st * 4 + gh] = lt;
+    }
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float* dst = os + (static_cast<size_t>(st) * 4 + h) * D + lane_r * 8;
+      reinterpret_cast<float4*>(dst)[0] = make_float4(acc[h][0].x, acc[h][0].y, acc[h][1].x, acc[h][1].y);
+      reinterpret_cast<float4*>(dst)[1] = make_float4(acc[h][2].x, acc[h][2].y, acc[h][3].x, acc[h][3].y);
+    }
+  }
+  __syncthreads();
+  const size_t row0 = (static_cast<size_t>(seq) * a.Hq + hkv * 4) * a.max_splits + split;
+  for (int idx = tid; idx < 4 * D; idx += kG4Threads) {
+    const int g = idx / D, col = idx % D;
+    float M = -INFINITY;
+    for (int e = 0; e < L::kStates; ++e) M = fmaxf(M, ms[e * 4 + g]);
+    float tot = 0.f, o = 0.f;
+    for (int e = 0; e < L::kStates; ++e) {
+      const float me = ms[e * 4 + g];
+      const float w = (me == -INFINITY) ? 0.f : ex2((me - M) * c2);
+      tot = fmaf(w, ls[e * 4 + g], tot);
+      o = fmaf(w, os[(static_cast<size_t>(e) * 4 + g) * D + col], o);
+    }
+    a.part_o[(row0 + static_cast<size_t>(g) * a.max_splits) * D + col] = o / tot;
+    if (col == 0) a.part_lse[row0 + static_cast<size_t>(g) * a.max_splits] = fmaf(M, a.scale, __logf(tot));
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a, __nv_bfloat16* o, float* lse) {
   const int hq = blockIdx.x, seq = blockIdx.y;
@@ -473,8 +781,17 @@ static cudaError_t launch_split(const DecodeArgs& a, dim3 grid, cudaStream_t str
   return cudaGetLastError();
 }
 
+static cudaError_t launch_split_g4(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
+  static int attr_done[64] = {0};
+  cudaError_t e = ensure_smem_limit(decode_split_g4_kernel, G4Layout::kBytes, attr_done);
+  if (e != cudaSuccess) return e;
+  decode_split_g4_kernel<<<grid, kG4Threads, G4Layout::kBytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
 template <int D>
 static cudaError_t launch_split_g(const DecodeArgs& a, int G, dim3 grid, cudaStream_t stream) {
+  if (D == 128 && G == 4) return launch_split_g4(a, grid, stream);
   switch (G) {
     case 1: return launch_split<D, 1>(a, grid, stream);
     case 2: return launch_split<D, 2>(a, grid, stream);
