@@ -352,7 +352,7 @@ def run_ours(args):
             "prefill": {"ms": t_pre, "tflops": tflops, "flops_per_step_per_gpu": pre_flops},
             "decode": {"value": gbs, "unit": "GB/s", "ms": t_dec, "bytes_per_step_per_gpu": dec_bytes,
                        "roofline": roofline("hbm", dec_per_gpu, peaks["hbm_gbs"], "GB/s",
-                                            recorded_traffic("decode_split_kernel", "decode_paged.cu",
+                                            recorded_traffic("decode_split_g4_kernel", "decode_paged.cu",
                                                              float(dinp.seq_lens.sum()))),
                        "e2e": dec_e2e},
             "roofline": roofline("tensor", pre_per_gpu, peaks["bf16_tflops"], "TFLOP/s",
