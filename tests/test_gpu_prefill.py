@@ -49,6 +49,10 @@ CASES = [
     (1, 1, 1, 1, 700, 128, False),        # one query row
     (1, 1, 1, 1, 700, 128, True),
     (1, 1, 1, 513, 129, 128, False),
+    # more CTAs than SMs, several waves
+    (2, 40, 8, 512, 512, 128, True),
+    (1, 64, 16, 600, 200, 128, True),     # items with no visible key mixed in
+    (2, 40, 40, 384, 384, 64, False),
 ]
 
 
