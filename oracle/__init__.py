@@ -1,4 +1,4 @@
-"""fp64 CPU oracle for exact attention and its paged-decode form.
+"""fp64 CPU oracle for exact attention, its paged-decode form and its gradients.
 
 TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
 benchmark's CPU-baseline leg import this package; the library under
@@ -33,6 +33,9 @@ def _bind(path):
     L.oracle_paged_decode.argtypes = [c_u16p, c_u16p, c_u16p, c_i32p, c_i32p] + [ctypes.c_int] * 6 + [
         ctypes.c_int64, ctypes.c_double, c_i32p, ctypes.c_int, c_dp, c_dp]
     L.oracle_paged_decode.restype = ctypes.c_int
+    L.oracle_attn_bwd.argtypes = [c_u16p, c_u16p, c_u16p, c_u16p] + [ctypes.c_int] * 6 + [
+        ctypes.c_double, ctypes.c_int, c_i64p, ctypes.c_int64, c_dp, c_dp, c_dp]
+    L.oracle_attn_bwd.restype = ctypes.c_int
     L.oracle_num_threads.restype = ctypes.c_int
     L.oracle_set_num_threads.argtypes = [ctypes.c_int]
     return L
@@ -151,6 +154,41 @@ def paged_decode(q, k_cache, v_cache, block_table, seq_lens, scale: float | None
     return o[:n], lse[:n]
 
 
+def attn_bwd(q, k, v, dout, causal: bool, scale: float | None = None, groups=None, _L=None):
+    """Gradients (dq, dk, dv) of attention in fp64 for the loss gradient dout.
+
+    q, dout [B,Hq,Nq,d]; k, v [B,Hkv,Nkv,d] as uint16 bf16 bit arrays.
+    groups: optional flat KV-head ids b*Hkv + hkv to evaluate (with all rows of
+    their query heads); gradients of other heads are returned as zeros.
+    Returns dq [B,Hq,Nq,d], dk [B,Hkv,Nkv,d], dv [B,Hkv,Nkv,d] as float64.
+    """
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    dout = np.ascontiguousarray(dout, dtype=np.uint16)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nkv, _ = k.shape
+    if dout.shape != q.shape:
+        raise OracleError("dout must have the shape of q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if groups is None:
+        n, gp = B * Hkv, None
+    else:
+        groups = np.ascontiguousarray(groups, dtype=np.int64)
+        n, gp = groups.size, _p(groups, ctypes.c_int64)
+    dq = np.zeros((B, Hq, Nq, d), dtype=np.float64)
+    dk = np.zeros((B, Hkv, Nkv, d), dtype=np.float64)
+    dv = np.zeros((B, Hkv, Nkv, d), dtype=np.float64)
+    err = (_L or lib()).oracle_attn_bwd(_p(q, ctypes.c_uint16), _p(k, ctypes.c_uint16), _p(v, ctypes.c_uint16),
+                                        _p(dout, ctypes.c_uint16), B, Hq, Hkv, Nq, Nkv, d, float(scale),
+                                        int(bool(causal)), gp, n, _p(dq, ctypes.c_double),
+                                        _p(dk, ctypes.c_double), _p(dv, ctypes.c_double))
+    if err:
+        raise OracleError(f"oracle_attn_bwd failed with code {err}")
+    return dq, dk, dv
+
+
 class Variant:
     """The same wrappers bound to another build of oracle.c (used by the
     tests that check the pins catch planted mistakes)."""
@@ -166,3 +204,6 @@ class Variant:
 
     def paged_decode(self, *a, **kw):
         return paged_decode(*a, _L=self._L, **kw)
+
+    def attn_bwd(self, *a, **kw):
+        return attn_bwd(*a, _L=self._L, **kw)

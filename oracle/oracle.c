@@ -274,3 +274,113 @@ int oracle_paged_decode(const uint16_t *q, const uint16_t *k_cache, const uint16
     }
     return err;
 }
+
+/*
+ * Gradients of attention (the backward pass), plain chain rule in fp64.
+ *
+ * The kernel-fusion post (section 4, recomputation) fixes the strategy of the
+ * backward pass -- keep only each row's max and normaliser, recompute the
+ * Q K^T blocks, stream the gradients -- but prints no formulas, so this is
+ * the derivative of the definition above, written out:
+ *
+ *   S = scale Q K^T (+ mask),  P = softmax_rows(S),  O = P V,  loss gradient dO
+ *   dV = P^T dO
+ *   dP = dO V^T
+ *   dS_ij = P_ij (dP_ij - sum_t P_it dP_it)          (softmax Jacobian)
+ *   dQ = scale dS K,   dK = scale dS^T Q
+ *
+ * With grouped heads a KV head's dK and dV sum the contributions of every
+ * query head that reads it.  Masked entries have P = 0 and contribute
+ * nothing; a row with no visible key contributes nothing.
+ *
+ * groups: optional list of flat KV-head ids g = b*Hkv + hkv to evaluate (each
+ * needs all rows of its query heads); NULL = all.  dq [B,Hq,Nq,d],
+ * dk/dv [B,Hkv,Nkv,d] (fp64) are written for the listed groups only and must
+ * be zero-initialised by the caller.
+ */
+int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                    int B, int Hq, int Hkv, int Nq, int Nkv, int d, double scale, int causal,
+                    const int64_t *groups, int64_t ngroups, double *dq, double *dk, double *dv)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nkv < 0 || d <= 0 || Hq % Hkv)
+        return ORACLE_ERR_ARG;
+    const int64_t total = (int64_t)B * Hkv;
+    if (!groups)
+        ngroups = total;
+    const int G = Hq / Hkv;
+    int err = ORACLE_OK;
+#pragma omp parallel
+    {
+        size_t n = (size_t)(Nkv > 0 ? Nkv : 1);
+        double *s = (double *)malloc(sizeof(double) * n);
+        double *p = (double *)malloc(sizeof(double) * n);
+        double *dp = (double *)malloc(sizeof(double) * n);
+        if (!s || !p || !dp) {
+#pragma omp atomic write
+            err = ORACLE_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t gi = 0; gi < ngroups; ++gi) {
+            if (!s || !p || !dp)
+                continue;
+            int64_t gid = groups ? groups[gi] : gi;
+            if (gid < 0 || gid >= total) {
+#pragma omp atomic write
+                err = ORACLE_ERR_ARG;
+                continue;
+            }
+            int b = (int)(gid / Hkv), hkv = (int)(gid % Hkv);
+            const uint16_t *kb = k + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
+            const uint16_t *vb = v + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
+            double *dkb = dk + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
+            double *dvb = dv + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
+            for (int hq = hkv * G; hq < (hkv + 1) * G; ++hq) {
+                for (int i = 0; i < Nq; ++i) {
+                    size_t row = (((size_t)b * Hq + hq) * (size_t)Nq + i);
+                    const uint16_t *qi = q + row * d;
+                    const uint16_t *doi = dout + row * d;
+                    double *dqi = dq + row * d;
+                    int visible = visible_keys(i, Nq, Nkv, causal);
+                    if (visible == 0)
+                        continue;
+                    /* scores over the visible keys, then the three-sweep softmax */
+                    double m = -INFINITY;
+                    for (int j = 0; j < visible; ++j) {
+                        double acc = 0.0;
+                        for (int t = 0; t < d; ++t)
+                            acc += bf16_to_f64(qi[t]) * bf16_to_f64(kb[(size_t)j * d + t]);
+                        s[j] = scale * acc;
+                        if (s[j] > m)
+                            m = s[j];
+                    }
+                    double l = 0.0;
+                    for (int j = 0; j < visible; ++j)
+                        l += exp(s[j] - m);
+                    for (int j = 0; j < visible; ++j)
+                        p[j] = exp(s[j] - m) / l;
+                    /* dP_ij = dO_i . v_j and the Jacobian's row term */
+                    double rowterm = 0.0;
+                    for (int j = 0; j < visible; ++j) {
+                        double acc = 0.0;
+                        for (int t = 0; t < d; ++t)
+                            acc += bf16_to_f64(doi[t]) * bf16_to_f64(vb[(size_t)j * d + t]);
+                        dp[j] = acc;
+                        rowterm += p[j] * dp[j];
+                    }
+                    for (int j = 0; j < visible; ++j) {
+                        double ds = p[j] * (dp[j] - rowterm);
+                        for (int t = 0; t < d; ++t) {
+                            dqi[t] += scale * ds * bf16_to_f64(kb[(size_t)j * d + t]);
+                            dkb[(size_t)j * d + t] += scale * ds * bf16_to_f64(qi[t]);
+                            dvb[(size_t)j * d + t] += p[j] * bf16_to_f64(doi[t]);
+                        }
+                    }
+                }
+            }
+        }
+        free(s);
+        free(p);
+        free(dp);
+    }
+    return err;
+}

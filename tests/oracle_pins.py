@@ -301,7 +301,149 @@ def pin_paged_decode(orc):
             _close(lse[s, h], lb, what=f"decode lse seq {s} head {h}")
 
 
+# ---------------------------------------------------------------------------
+# Backward pass (gradients of attention)
+# ---------------------------------------------------------------------------
+
+def _forward_f64(Q, K, V, scale, causal):
+    """Attention written out in fp64 on float inputs (not bf16 bits), independent
+    of the oracle: explicit mask, softmax with the row max subtracted, O = P V.
+    Q [B,Hq,Nq,d], K/V [B,Hkv,Nkv,d]."""
+    B, Hq, Nq, d = Q.shape
+    Hkv, Nkv = K.shape[1], K.shape[2]
+    G = Hq // Hkv
+    O = np.zeros_like(Q)
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // G
+            S = scale * (Q[b, h] @ K[b, kv].T)
+            for i in range(Nq):
+                vis = _visible(i, Nq, Nkv, causal)
+                if vis == 0:
+                    continue
+                srow = S[i, :vis]
+                e = np.exp(srow - srow.max())
+                O[b, h, i] = (e / e.sum()) @ V[b, kv, :vis]
+    return O
+
+
+def pin_bwd_finite_differences(orc):
+    # directional derivatives of L = sum(dO * O) by central differences of an
+    # independent fp64 forward, against <grad, direction> from the oracle
+    rng = np.random.Generator(np.random.PCG64(21))
+    for (B, Hq, Hkv, Nq, Nkv, d) in [(1, 2, 1, 5, 6, 3), (1, 1, 1, 4, 4, 2), (2, 4, 2, 3, 7, 2)]:
+        for causal in (False, True):
+            scale = 0.8
+            q, k, v, do = (_bf16(rng, (B, Hq, Nq, d)), _bf16(rng, (B, Hkv, Nkv, d)),
+                           _bf16(rng, (B, Hkv, Nkv, d)), _bf16(rng, (B, Hq, Nq, d)))
+            dq, dk, dv = orc.attn_bwd(q, k, v, do, causal, scale=scale)
+            X = [widen(q), widen(k), widen(v)]
+            dO = widen(do)
+            grads = [dq, dk, dv]
+            eps = 1e-5
+            for which in range(3):
+                for trial in range(3):
+                    E = rng.standard_normal(X[which].shape)
+                    Xp = [x.copy() for x in X]
+                    Xm = [x.copy() for x in X]
+                    Xp[which] += eps * E
+                    Xm[which] -= eps * E
+                    fd = (np.sum(dO * _forward_f64(*Xp, scale, causal)) -
+                          np.sum(dO * _forward_f64(*Xm, scale, causal))) / (2 * eps)
+                    an = float(np.sum(grads[which] * E))
+                    if abs(fd - an) > 1e-6 * max(1.0, abs(fd)):
+                        raise AssertionError(f"bwd finite differences ({'qkv'[which]}) {B,Hq,Hkv,Nq,Nkv,d} "
+                                             f"c={causal}: {an} vs {fd}")
+
+
+def pin_bwd_single_key(orc):
+    # one key: P = 1 for every row that sees it, so dQ = dK = 0 and
+    # dV_0 = sum of dO over those rows (all query heads of the group)
+    rng = np.random.Generator(np.random.PCG64(22))
+    for (B, Hq, Hkv, Nq) in [(1, 2, 1, 5), (2, 4, 2, 3)]:
+        for causal in (False, True):
+            q, k, v, do = (_bf16(rng, (B, Hq, Nq, 4)), _bf16(rng, (B, Hkv, 1, 4)),
+                           _bf16(rng, (B, Hkv, 1, 4)), _bf16(rng, (B, Hq, Nq, 4)))
+            dq, dk, dv = orc.attn_bwd(q, k, v, do, causal, scale=1.1)
+            _close(dq, np.zeros_like(dq), what="single key dq")
+            _close(dk, np.zeros_like(dk), what="single key dk")
+            G = Hq // Hkv
+            want = np.zeros_like(dv)
+            for b in range(B):
+                for h in range(Hq):
+                    for i in range(Nq):
+                        if _visible(i, Nq, 1, causal) > 0:
+                            want[b, h // G, 0] += widen(do[b, h, i])
+            _close(dv, want, what="single key dv")
+
+
+def pin_bwd_scale_zero(orc):
+    # scale 0: uniform weights over the visible keys, no gradient reaches Q or K
+    rng = np.random.Generator(np.random.PCG64(23))
+    B, Hq, Hkv, Nq, Nkv, d = 1, 2, 1, 6, 4, 3
+    for causal in (False, True):
+        q, k, v, do = (_bf16(rng, (B, Hq, Nq, d)), _bf16(rng, (B, Hkv, Nkv, d)),
+                       _bf16(rng, (B, Hkv, Nkv, d)), _bf16(rng, (B, Hq, Nq, d)))
+        dq, dk, dv = orc.attn_bwd(q, k, v, do, causal, scale=0.0)
+        _close(dq, np.zeros_like(dq), what="scale 0 dq")
+        _close(dk, np.zeros_like(dk), what="scale 0 dk")
+        want = np.zeros_like(dv)
+        for h in range(Hq):
+            for i in range(Nq):
+                n = _visible(i, Nq, Nkv, causal)
+                for j in range(n):
+                    want[0, 0, j] += widen(do[0, h, i]) / n
+        _close(dv, want, what="scale 0 dv")
+
+
+def pin_bwd_key_gradients_sum_to_zero(orc):
+    # each row of dS sums to zero (softmax is shift invariant), hence
+    # sum_j dK_j = 0 for every KV head
+    rng = np.random.Generator(np.random.PCG64(24))
+    for (B, Hq, Hkv, Nq, Nkv, d) in [(1, 2, 1, 9, 9, 5), (2, 3, 3, 4, 11, 4)]:
+        for causal in (False, True):
+            q, k, v, do = (_bf16(rng, (B, Hq, Nq, d)), _bf16(rng, (B, Hkv, Nkv, d)),
+                           _bf16(rng, (B, Hkv, Nkv, d)), _bf16(rng, (B, Hq, Nq, d)))
+            _, dk, _ = orc.attn_bwd(q, k, v, do, causal, scale=0.9)
+            _close(dk.sum(axis=2), np.zeros((B, Hkv, d)), tol=1e-11, what="sum of dK")
+
+
+def pin_bwd_permutation(orc):
+    # non-causal: permuting the (k_j, v_j) pairs permutes dK and dV the same
+    # way and leaves dQ unchanged
+    rng = np.random.Generator(np.random.PCG64(25))
+    B, Hq, Hkv, Nq, Nkv, d = 1, 2, 2, 5, 8, 4
+    q, k, v, do = (_bf16(rng, (B, Hq, Nq, d)), _bf16(rng, (B, Hkv, Nkv, d)),
+                   _bf16(rng, (B, Hkv, Nkv, d)), _bf16(rng, (B, Hq, Nq, d)))
+    perm = rng.permutation(Nkv)
+    dq, dk, dv = orc.attn_bwd(q, k, v, do, False, scale=0.6)
+    dq2, dk2, dv2 = orc.attn_bwd(q, k[:, :, perm], v[:, :, perm], do, False, scale=0.6)
+    _close(dq2, dq, tol=1e-11, what="perm dq")
+    _close(dk2, dk[:, :, perm], tol=1e-11, what="perm dk")
+    _close(dv2, dv[:, :, perm], tol=1e-11, what="perm dv")
+
+
+def pin_bwd_grouped_heads(orc):
+    # a KV head shared by G query heads gets the sum of the gradients it would
+    # get as G separate copies (one per query head)
+    rng = np.random.Generator(np.random.PCG64(26))
+    B, Hq, Hkv, Nq, Nkv, d = 2, 4, 2, 5, 6, 3
+    G = Hq // Hkv
+    for causal in (False, True):
+        q, k, v, do = (_bf16(rng, (B, Hq, Nq, d)), _bf16(rng, (B, Hkv, Nkv, d)),
+                       _bf16(rng, (B, Hkv, Nkv, d)), _bf16(rng, (B, Hq, Nq, d)))
+        dq, dk, dv = orc.attn_bwd(q, k, v, do, causal, scale=0.7)
+        kr, vr = np.repeat(k, G, axis=1), np.repeat(v, G, axis=1)
+        dq1, dk1, dv1 = orc.attn_bwd(q, kr, vr, do, causal, scale=0.7)
+        _close(dq1, dq, tol=1e-11, what="gqa dq")
+        _close(dk1.reshape(B, Hkv, G, Nkv, d).sum(axis=2), dk, tol=1e-11, what="gqa dk")
+        _close(dv1.reshape(B, Hkv, G, Nkv, d).sum(axis=2), dv, tol=1e-11, what="gqa dv")
+
+
+BWD_PINS = [pin_bwd_finite_differences, pin_bwd_single_key, pin_bwd_scale_zero,
+            pin_bwd_key_gradients_sum_to_zero, pin_bwd_permutation, pin_bwd_grouped_heads]
+
 ALL_PINS = [pin_brute_force, pin_large_scores, pin_handpicked, pin_rows_of_p_sum_to_one,
             pin_constant_v, pin_permutation_invariance, pin_single_key, pin_scale_zero,
             pin_causal_row0, pin_identical_keys, pin_online_recurrence, pin_paged_gather,
-            pin_paged_decode]
+            pin_paged_decode] + BWD_PINS

@@ -24,6 +24,18 @@ MUTANTS = {
     "page_row_index": ("(size_t)(t % page_size)) * d;", "(size_t)(t / page_size)) * d;"),
     "sum_without_max": ("l += exp(s[j] - m);", "l += exp(s[j]);"),
     "decode_head_mapping": ("int hq = hkv * G + g;", "int hq = g * Hkv + hkv;"),
+    # backward pass
+    "bwd_dq_without_scale": ("dqi[t] += scale * ds *", "dqi[t] += ds *"),
+    "bwd_no_jacobian_row_term": ("double ds = p[j] * (dp[j] - rowterm);", "double ds = p[j] * dp[j];"),
+    "bwd_dv_from_q": ("dvb[(size_t)j * d + t] += p[j] * bf16_to_f64(doi[t]);",
+                      "dvb[(size_t)j * d + t] += p[j] * bf16_to_f64(qi[t]);"),
+    "bwd_dk_from_do": ("dkb[(size_t)j * d + t] += scale * ds * bf16_to_f64(qi[t]);",
+                       "dkb[(size_t)j * d + t] += scale * ds * bf16_to_f64(doi[t]);"),
+    "bwd_one_head_per_group": ("for (int hq = hkv * G; hq < (hkv + 1) * G; ++hq)",
+                               "for (int hq = hkv * G; hq < hkv * G + 1; ++hq)"),
+    "bwd_dp_from_k": ("acc += bf16_to_f64(doi[t]) * bf16_to_f64(vb[", "acc += bf16_to_f64(doi[t]) * bf16_to_f64(kb["),
+    "bwd_dk_transposed_ds": ("dkb[(size_t)j * d + t] += scale * ds * bf16_to_f64(qi[t]);",
+                             "dkb[(size_t)j * d + t] += scale * p[j] * dp[j] * bf16_to_f64(qi[t]);"),
 }
 
 
