@@ -92,6 +92,42 @@ ta_status attn_fwd(const void *q, const void *k, const void *v, void *o, float *
                    float scale, int causal, ta_stream_t stream);
 
 /*
+ * Bytes of device workspace attn_bwd needs (256-byte multiple): two fp32
+ * values per query row, rows padded to a multiple of 128 per head.  Pure
+ * host arithmetic; returns 0 for invalid sizes.
+ */
+size_t attn_bwd_workspace_size(int B, int Hq, int Nq);
+
+/*
+ * attn_bwd - gradients of attn_fwd by recomputation.  (The kernel-fusion
+ * post, section 4, states the strategy: keep only each row's max and
+ * normaliser from the forward pass, recompute the Q K^T blocks during the
+ * backward pass and stream the gradients; it prints no formulas.  This call
+ * computes the chain rule through the softmax:
+ *     dV = P^T dO,  dS = P o (dO V^T - rowsum(dO o O)),
+ *     dQ = scale dS K,  dK = scale dS^T Q,
+ * with P = exp(scale Q K^T [+ mask] - lse) rebuilt tile by tile.)
+ *
+ *   q, o, dout, dq   [B, Hq,  Nq,  d]  bf16 (o and lse as written by attn_fwd
+ *   k, v, dk, dv     [B, Hkv, Nkv, d]  bf16  for the same q, k, v, scale and
+ *   lse              [B, Hq,  Nq]      fp32  causal; dout is the gradient of
+ *                                            the loss with respect to o)
+ *   workspace        >= attn_bwd_workspace_size(B, Hq, Nq) bytes, 256-byte
+ *                    aligned; overwritten.
+ *
+ * dq, dk, dv are written (not accumulated) in bf16.  With grouped heads a KV
+ * head's dk and dv sum the contributions of all Hq / Hkv query heads that read
+ * it.  Rows with no visible key (lse = -inf) contribute nothing.  Same
+ * supported shapes and conventions as attn_fwd; outputs must not overlap the
+ * inputs.  Nq == 0 writes dk = dv = 0 and Nkv == 0 writes dq = 0.  The
+ * result does not depend on scheduling: no atomics are used.
+ */
+ta_status attn_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                   const float *lse, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                   int B, int Hq, int Hkv, int Nq, int Nkv, int d, float scale, int causal,
+                   ta_stream_t stream);
+
+/*
  * Bytes of device workspace attn_paged_decode needs for these sizes (256-byte
  * aligned).  Pure host arithmetic; returns 0 for invalid sizes.
  */

@@ -293,11 +293,26 @@ int oracle_paged_decode(const uint16_t *q, const uint16_t *k_cache, const uint16
  * query head that reads it.  Masked entries have P = 0 and contribute
  * nothing; a row with no visible key contributes nothing.
  *
+ * Evaluation order (plain loops, parallel over independent outputs):
+ *   sweep 1, per query row i: scores, the three-sweep softmax, dP_i., the
+ *            Jacobian row term r_i = sum_t P_it dP_it, and dQ_i; keeps the
+ *            row's max m_i and normaliser l_i;
+ *   sweep 2, per key j: P_ij = exp(s_ij - m_i) / l_i and dP_ij recomputed for
+ *            every row i that sees j, then dV_j and dK_j.
+ *
  * groups: optional list of flat KV-head ids g = b*Hkv + hkv to evaluate (each
- * needs all rows of its query heads); NULL = all.  dq [B,Hq,Nq,d],
+ * with all rows of its query heads); NULL = all.  dq [B,Hq,Nq,d] and
  * dk/dv [B,Hkv,Nkv,d] (fp64) are written for the listed groups only and must
  * be zero-initialised by the caller.
  */
+static double dot_bf16(const uint16_t *a, const uint16_t *b, int d)
+{
+    double acc = 0.0;
+    for (int t = 0; t < d; ++t)
+        acc += bf16_to_f64(a[t]) * bf16_to_f64(b[t]);
+    return acc;
+}
+
 int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
                     int B, int Hq, int Hkv, int Nq, int Nkv, int d, double scale, int causal,
                     const int64_t *groups, int64_t ngroups, double *dq, double *dk, double *dv)
@@ -307,8 +322,24 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
     const int64_t total = (int64_t)B * Hkv;
     if (!groups)
         ngroups = total;
+    for (int64_t gi = 0; gi < ngroups; ++gi)
+        if (groups && (groups[gi] < 0 || groups[gi] >= total))
+            return ORACLE_ERR_ARG;
     const int G = Hq / Hkv;
+    const int64_t rows_per_group = (int64_t)G * Nq;
+    /* per row of the listed groups: softmax max, normaliser, Jacobian row term */
+    double *rm = (double *)malloc(sizeof(double) * (size_t)(ngroups * rows_per_group + 1));
+    double *rl = (double *)malloc(sizeof(double) * (size_t)(ngroups * rows_per_group + 1));
+    double *rr = (double *)malloc(sizeof(double) * (size_t)(ngroups * rows_per_group + 1));
+    if (!rm || !rl || !rr) {
+        free(rm);
+        free(rl);
+        free(rr);
+        return ORACLE_ERR_NOMEM;
+    }
     int err = ORACLE_OK;
+
+    /* sweep 1: one query row at a time */
 #pragma omp parallel
     {
         size_t n = (size_t)(Nkv > 0 ? Nkv : 1);
@@ -319,68 +350,83 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
 #pragma omp atomic write
             err = ORACLE_ERR_NOMEM;
         }
-#pragma omp for schedule(dynamic, 1)
-        for (int64_t gi = 0; gi < ngroups; ++gi) {
+#pragma omp for schedule(dynamic, 8)
+        for (int64_t x = 0; x < ngroups * rows_per_group; ++x) {
             if (!s || !p || !dp)
                 continue;
-            int64_t gid = groups ? groups[gi] : gi;
-            if (gid < 0 || gid >= total) {
-#pragma omp atomic write
-                err = ORACLE_ERR_ARG;
-                continue;
-            }
+            int64_t gid = groups ? groups[x / rows_per_group] : x / rows_per_group;
             int b = (int)(gid / Hkv), hkv = (int)(gid % Hkv);
+            int hq = hkv * G + (int)((x % rows_per_group) / Nq);
+            int i = (int)(x % Nq);
+            size_t row = ((size_t)b * Hq + hq) * (size_t)Nq + i;
+            const uint16_t *qi = q + row * d, *doi = dout + row * d;
             const uint16_t *kb = k + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
             const uint16_t *vb = v + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
-            double *dkb = dk + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
-            double *dvb = dv + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
-            for (int hq = hkv * G; hq < (hkv + 1) * G; ++hq) {
-                for (int i = 0; i < Nq; ++i) {
-                    size_t row = (((size_t)b * Hq + hq) * (size_t)Nq + i);
-                    const uint16_t *qi = q + row * d;
-                    const uint16_t *doi = dout + row * d;
-                    double *dqi = dq + row * d;
-                    int visible = visible_keys(i, Nq, Nkv, causal);
-                    if (visible == 0)
-                        continue;
-                    /* scores over the visible keys, then the three-sweep softmax */
-                    double m = -INFINITY;
-                    for (int j = 0; j < visible; ++j) {
-                        double acc = 0.0;
-                        for (int t = 0; t < d; ++t)
-                            acc += bf16_to_f64(qi[t]) * bf16_to_f64(kb[(size_t)j * d + t]);
-                        s[j] = scale * acc;
-                        if (s[j] > m)
-                            m = s[j];
-                    }
-                    double l = 0.0;
-                    for (int j = 0; j < visible; ++j)
-                        l += exp(s[j] - m);
-                    for (int j = 0; j < visible; ++j)
-                        p[j] = exp(s[j] - m) / l;
-                    /* dP_ij = dO_i . v_j and the Jacobian's row term */
-                    double rowterm = 0.0;
-                    for (int j = 0; j < visible; ++j) {
-                        double acc = 0.0;
-                        for (int t = 0; t < d; ++t)
-                            acc += bf16_to_f64(doi[t]) * bf16_to_f64(vb[(size_t)j * d + t]);
-                        dp[j] = acc;
-                        rowterm += p[j] * dp[j];
-                    }
-                    for (int j = 0; j < visible; ++j) {
-                        double ds = p[j] * (dp[j] - rowterm);
-                        for (int t = 0; t < d; ++t) {
-                            dqi[t] += scale * ds * bf16_to_f64(kb[(size_t)j * d + t]);
-                            dkb[(size_t)j * d + t] += scale * ds * bf16_to_f64(qi[t]);
-                            dvb[(size_t)j * d + t] += p[j] * bf16_to_f64(doi[t]);
-                        }
-                    }
-                }
+            int visible = visible_keys(i, Nq, Nkv, causal);
+            rm[x] = -INFINITY;
+            rl[x] = 0.0;
+            rr[x] = 0.0;
+            if (visible == 0)
+                continue;
+            double m = -INFINITY;
+            for (int j = 0; j < visible; ++j) {
+                s[j] = scale * dot_bf16(qi, kb + (size_t)j * d, d);
+                if (s[j] > m)
+                    m = s[j];
             }
+            double l = 0.0;
+            for (int j = 0; j < visible; ++j)
+                l += exp(s[j] - m);
+            double rowterm = 0.0;
+            for (int j = 0; j < visible; ++j) {
+                p[j] = exp(s[j] - m) / l;
+                dp[j] = dot_bf16(doi, vb + (size_t)j * d, d);
+                rowterm += p[j] * dp[j];
+            }
+            double *dqi = dq + row * d;
+            for (int j = 0; j < visible; ++j) {
+                double ds = p[j] * (dp[j] - rowterm);
+                for (int t = 0; t < d; ++t)
+                    dqi[t] += scale * ds * bf16_to_f64(kb[(size_t)j * d + t]);
+            }
+            rm[x] = m;
+            rl[x] = l;
+            rr[x] = rowterm;
         }
         free(s);
         free(p);
         free(dp);
     }
+
+    /* sweep 2: one key at a time, over every row of the group that sees it */
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int64_t y = 0; y < ngroups * (int64_t)Nkv; ++y) {
+        int64_t gi = y / Nkv;
+        int64_t gid = groups ? groups[gi] : gi;
+        int b = (int)(gid / Hkv), hkv = (int)(gid % Hkv);
+        int j = (int)(y % Nkv);
+        const uint16_t *kj = k + (((size_t)b * Hkv + hkv) * (size_t)Nkv + j) * d;
+        const uint16_t *vj = v + (((size_t)b * Hkv + hkv) * (size_t)Nkv + j) * d;
+        double *dkj = dk + (((size_t)b * Hkv + hkv) * (size_t)Nkv + j) * d;
+        double *dvj = dv + (((size_t)b * Hkv + hkv) * (size_t)Nkv + j) * d;
+        for (int hq = hkv * G; hq < (hkv + 1) * G; ++hq) {
+            for (int i = 0; i < Nq; ++i) {
+                if (j >= visible_keys(i, Nq, Nkv, causal))
+                    continue;
+                int64_t x = gi * rows_per_group + (int64_t)(hq - hkv * G) * Nq + i;
+                size_t row = ((size_t)b * Hq + hq) * (size_t)Nq + i;
+                const uint16_t *qi = q + row * d, *doi = dout + row * d;
+                double p = exp(scale * dot_bf16(qi, kj, d) - rm[x]) / rl[x];
+                double ds = p * (dot_bf16(doi, vj, d) - rr[x]);
+                for (int t = 0; t < d; ++t) {
+                    dkj[t] += scale * ds * bf16_to_f64(qi[t]);
+                    dvj[t] += p * bf16_to_f64(doi[t]);
+                }
+            }
+        }
+    }
+    free(rm);
+    free(rl);
+    free(rr);
     return err;
 }

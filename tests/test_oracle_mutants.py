@@ -27,15 +27,15 @@ MUTANTS = {
     # backward pass
     "bwd_dq_without_scale": ("dqi[t] += scale * ds *", "dqi[t] += ds *"),
     "bwd_no_jacobian_row_term": ("double ds = p[j] * (dp[j] - rowterm);", "double ds = p[j] * dp[j];"),
-    "bwd_dv_from_q": ("dvb[(size_t)j * d + t] += p[j] * bf16_to_f64(doi[t]);",
-                      "dvb[(size_t)j * d + t] += p[j] * bf16_to_f64(qi[t]);"),
-    "bwd_dk_from_do": ("dkb[(size_t)j * d + t] += scale * ds * bf16_to_f64(qi[t]);",
-                       "dkb[(size_t)j * d + t] += scale * ds * bf16_to_f64(doi[t]);"),
+    "bwd_key_sweep_no_row_term": ("double ds = p * (dot_bf16(doi, vj, d) - rr[x]);", "double ds = p * dot_bf16(doi, vj, d);"),
+    "bwd_dv_from_q": ("dvj[t] += p * bf16_to_f64(doi[t]);", "dvj[t] += p * bf16_to_f64(qi[t]);"),
+    "bwd_dk_from_do": ("dkj[t] += scale * ds * bf16_to_f64(qi[t]);", "dkj[t] += scale * ds * bf16_to_f64(doi[t]);"),
     "bwd_one_head_per_group": ("for (int hq = hkv * G; hq < (hkv + 1) * G; ++hq)",
                                "for (int hq = hkv * G; hq < hkv * G + 1; ++hq)"),
-    "bwd_dp_from_k": ("acc += bf16_to_f64(doi[t]) * bf16_to_f64(vb[", "acc += bf16_to_f64(doi[t]) * bf16_to_f64(kb["),
-    "bwd_dk_transposed_ds": ("dkb[(size_t)j * d + t] += scale * ds * bf16_to_f64(qi[t]);",
-                             "dkb[(size_t)j * d + t] += scale * p[j] * dp[j] * bf16_to_f64(qi[t]);"),
+    "bwd_dp_from_k": ("dp[j] = dot_bf16(doi, vb + (size_t)j * d, d);", "dp[j] = dot_bf16(doi, kb + (size_t)j * d, d);"),
+    "bwd_key_sweep_dp_from_k": ("double ds = p * (dot_bf16(doi, vj, d) - rr[x]);", "double ds = p * (dot_bf16(doi, kj, d) - rr[x]);"),
+    "bwd_key_sweep_unnormalised": ("- rm[x]) / rl[x];", "- rm[x]);"),
+    "bwd_key_sweep_mask_ignored": ("if (j >= visible_keys(i, Nq, Nkv, causal))\n                    continue;", "if (0)\n                    continue;"),
 }
 
 

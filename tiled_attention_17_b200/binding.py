@@ -24,7 +24,8 @@ TA_DEV_TIMEOUT = 1
 TA_DEV_BAD_BLOCK_TABLE = 2
 TA_DEV_BAD_SEQ_LEN = 4
 
-EXPORTS = ["ta_status_string", "ta_version", "ta_last_error", "attn_fwd", "attn_paged_decode_workspace_size",
+EXPORTS = ["ta_status_string", "ta_version", "ta_last_error", "attn_fwd", "attn_bwd_workspace_size", "attn_bwd",
+           "attn_paged_decode_workspace_size",
            "attn_paged_decode", "attn_paged_decode_noalloc", "attn_paged_decode_check", "attn_paged_gather_debug",
            "ta_device_status", "ta_selftest_bounded_wait"]
 
@@ -56,6 +57,10 @@ def load(path: str | None = None):
     L.ta_last_error.restype = ctypes.c_char_p
     L.attn_fwd.argtypes = [vp, vp, vp, vp, vp] + [i32] * 6 + [f32, i32, vp]
     L.attn_fwd.restype = i32
+    L.attn_bwd_workspace_size.argtypes = [i32] * 3
+    L.attn_bwd_workspace_size.restype = sz
+    L.attn_bwd.argtypes = [vp] * 10 + [sz] + [i32] * 6 + [f32, i32, vp]
+    L.attn_bwd.restype = i32
     L.attn_paged_decode_workspace_size.argtypes = [i32] * 6
     L.attn_paged_decode_workspace_size.restype = sz
     L.attn_paged_decode.argtypes = [vp, vp, vp, vp, vp] + [i32] * 7 + [f32, vp, vp, vp, sz, vp]
@@ -118,6 +123,20 @@ def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream=None
                            float(scale), int(causal), _stream(stream))
     if check:
         _check("attn_fwd", code)
+    return code
+
+
+def attn_bwd_workspace_size(B, Hq, Nq) -> int:
+    return load().attn_bwd_workspace_size(B, Hq, Nq)
+
+
+def attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, Nq, Nkv, d, scale,
+             causal, stream=None, check=True) -> int:
+    code = load().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                           _ptr(workspace), int(workspace_bytes), B, Hq, Hkv, Nq, Nkv, d, float(scale), int(causal),
+                           _stream(stream))
+    if check:
+        _check("attn_bwd", code)
     return code
 
 
@@ -194,6 +213,27 @@ def attention(q, k, v, causal: bool, scale: float | None = None, out=None, lse=N
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream)
     return o, lse
+
+
+def attention_backward(q, k, v, o, lse, dout, causal: bool, scale: float | None = None, workspace=None,
+                       stream=None):
+    """Gradients (dq, dk, dv) of `attention` for the loss gradient dout (all bf16
+    CUDA tensors; o and lse from the forward call with the same arguments)."""
+    import torch
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nkv, _ = k.shape
+    for t in (q, k, v, o, dout):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v, o, dout must be contiguous bf16 CUDA tensors")
+    if scale is None:
+        scale = d ** -0.5
+    ws_bytes = attn_bwd_workspace_size(B, Hq, Nq)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace.numel(), B, Hq, Hkv, Nq, Nkv, d, scale,
+             causal, stream)
+    return dq, dk, dv
 
 
 def paged_decode(q, k_cache, v_cache, block_table, seq_lens, scale: float | None = None, workspace=None,

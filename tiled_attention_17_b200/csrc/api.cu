@@ -50,6 +50,19 @@ PFN_encodeTiled get_encode_tiled() {
   return fn;
 }
 
+ta_status encode_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
+  PFN_encodeTiled enc = get_encode_tiled();
+  if (!enc) return fail(TA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slices)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TA_OK : fail_cu(TA_ERR_CUDA, "cuTensorMapEncodeTiled", static_cast<int>(r));
+}
+
 static thread_local char g_last_error[256] = "";
 
 ta_status fail(ta_status code, const char* where, cudaError_t err) {
@@ -106,6 +119,50 @@ ta_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* 
   const long long pairs = (static_cast<long long>(Nq) + 255) / 256;
   if (pairs * B * Hq > INT32_MAX) return TA_ERR_UNSUPPORTED;
   return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Nq) {
+  if (B < 0 || Hq <= 0 || Nq < 0) return 0;
+  if (static_cast<long long>(B) * Hq > INT32_MAX / 2 || Nq > (1 << 30)) return 0;
+  return bwd_workspace_bytes(B, Hq, Nq);
+}
+
+ta_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                   int Nq, int Nkv, int d, float scale, int causal, ta_stream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nkv < 0 || d <= 0) return TA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return TA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return TA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return TA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return TA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq > INT32_MAX / 2 || Nq > (1 << 30) || Nkv > (1 << 30)) return TA_ERR_UNSUPPORTED;
+  const long long q_tiles = (static_cast<long long>(Nq) + 127) / 128, k_tiles = (static_cast<long long>(Nkv) + 127) / 128;
+  if (q_tiles * B * Hq > INT32_MAX || k_tiles * B * Hkv > INT32_MAX) return TA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t q_bytes = static_cast<size_t>(B) * Hq * Nq * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(B) * Hkv * Nkv * d * 2;
+  if (q_bytes == 0 && kv_bytes == 0) return TA_OK;
+  if ((q_bytes && (!q || !o || !dout || !lse || !dq)) || (kv_bytes && (!k || !v || !dk || !dv)))
+    return TA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return TA_ERR_INVALID_ARG;
+  // no queries: no gradient reaches K or V; no keys: none reaches Q
+  if (q_bytes == 0 || kv_bytes == 0) {
+    cudaError_t e = cudaSuccess;
+    if (kv_bytes) {
+      if ((e = cudaMemsetAsync(dk, 0, kv_bytes, st)) == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, st);
+    }
+    if (q_bytes && e == cudaSuccess) e = cudaMemsetAsync(dq, 0, q_bytes, st);
+    return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "attn_bwd: zero fill", e);
+  }
+  const size_t need = bwd_workspace_bytes(B, Hq, Nq);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) {
+    char msg[160];
+    snprintf(msg, sizeof msg, "attn_bwd: workspace needs %zu bytes, 256-byte aligned", need);
+    return fail(TA_ERR_INVALID_ARG, msg);
+  }
+  return launch_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nkv, d, scale, causal, st);
 }
 
 size_t attn_paged_decode_workspace_size(int num_seqs, int Hq, int Hkv, int d, int max_pages, int page_size) {

@@ -1,0 +1,742 @@
+// Attention backward for sm_100a (B200): gradients dQ, dK, dV of
+// O = softmax(scale * Q K^T [+ causal mask]) V, by recomputation.
+//
+// The forward pass keeps only each row's log-sum-exp; the backward pass
+// recomputes the Q K^T blocks from it and streams the gradients tile by tile,
+// so neither S nor P is ever stored (Gemini 3 Flash kernel-fusion post,
+// section 4, recomputation strategy).  With P = exp(S - lse) per row:
+//
+//   dV = P^T dO,  dP = dO V^T,  dS = P o (dP - delta),  delta_i = dO_i . O_i
+//   dQ = scale dS K,  dK = scale dS^T Q
+//
+// (delta_i equals sum_j P_ij dP_ij, the softmax Jacobian's row term, because
+// O_i = sum_j P_ij v_j.)  Three kernels:
+//   bwd_prep_kernel    delta and lse (in log2 units, +inf for rows with no
+//                      visible key) per query row, into a padded workspace
+//   bwd_dkdv_kernel    one CTA per 128-key tile of one (batch, KV head); loops
+//                      over the query heads of the group and the query tiles
+//                      that see the keys; dK, dV accumulate in TMEM
+//   bwd_dq_kernel      one CTA per 128-row query tile; loops over key tiles;
+//                      dQ accumulates in TMEM
+// Splitting dQ from dK/dV recomputes S and dP once more (7 tile GEMMs instead
+// of 5) but needs no atomics, so the gradients are deterministic.
+//
+// Warp roles (256 threads): warp 0 TMA producer, warp 1 TMEM allocator and
+// single-thread tcgen05.mma issuer, warps 4-7 one thread per tile row for the
+// elementwise work and the epilogue.  All operand forms are the forward
+// kernel's: K-major A and B from shared memory for the score-like products,
+// bf16 probabilities from TMEM as A with an MN-major B for the accumulating
+// ones.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "tiledattn_internal.h"
+
+namespace ta {
+namespace {
+
+constexpr int kT = 128;          // rows per tile (queries or keys)
+constexpr int kBwdThreads = 256;
+constexpr int kWorkWarp0 = 4;    // warps 4-7: one thread per tile row
+
+template <int D>
+struct BwdTiles {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kChunks = D / 64;              // 64-column (128-byte) swizzle atoms
+  static constexpr int kTileBytes = kT * D * 2;
+  static constexpr int kChunkBytes = kT * 128;
+};
+
+struct BwdArgs {
+  int B, Hq, Hkv, Nq, Nkv;
+  int n_qt, n_kt;              // query / key tiles per head
+  int causal;
+  float scale;                 // multiplies dQ and dK
+  float scale_log2;            // scale * log2(e)
+  const float* delta;          // [B*Hq][n_qt*128]
+  const float* lse2;           // [B*Hq][n_qt*128], log2 units, +inf = no visible key
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  unsigned* status;
+};
+
+// K-major operand tile (128 rows x D, 128-byte swizzle): descriptor of the
+// tile, +2 per 16-element step inside a 64-column chunk, +chunk to the next.
+__device__ __forceinline__ void mma_kmajor_tile(uint32_t d_tmem, uint64_t a0, uint64_t b0, int chunks,
+                                                uint32_t idesc, bool acc) {
+#pragma unroll 1
+  for (int c = 0; c < chunks; ++c) {
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) mma_ss(d_tmem, a0 + 2 * k4, b0 + 2 * k4, idesc, (acc || (c | k4) != 0));
+    a0 += (kT * 128) >> 4;
+    b0 += (kT * 128) >> 4;
+  }
+}
+
+// D += A B with A = 128 x 128 bf16 in TMEM (64 columns of packed pairs) and
+// B = an MN-major 128-row x D tile in shared memory (K = its rows).
+__device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc, bool acc) {
+#pragma unroll
+  for (int kk = 0; kk < kT / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc,
+           (acc || kk > 0) ? 1u : 0u);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ---------------------------------------------------------------------------
+// delta_i = dO_i . O_i and lse in log2 units per (padded) query row
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ dout,
+                                                       const float* __restrict__ lse, float* __restrict__ delta,
+                                                       float* __restrict__ lse2, int Nq, int n_rows_pad,
+                                                       long long total_pad) {
+  // 8 lanes per row, each covering D/8 contiguous elements
+  constexpr int kPer = D / 8;
+  const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long r = gt >> 3;
+  const int part = static_cast<int>(gt & 7);
+  if (r >= total_pad) return;   // whole 8-lane groups leave together
+  const long long bh = r / n_rows_pad;
+  const int i = static_cast<int>(r - bh * n_rows_pad);
+  float acc = 0.f;
+  if (i < Nq) {
+    const size_t off = (static_cast<size_t>(bh) * Nq + i) * D + part * kPer;
+    const uint4* po = reinterpret_cast<const uint4*>(o + off);
+    const uint4* pd = reinterpret_cast<const uint4*>(dout + off);
+#pragma unroll
+    for (int v = 0; v < kPer / 8; ++v) {
+      const uint4 a = po[v], b = pd[v];
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc += bf16lo(aw[e]) * bf16lo(bw[e]) + bf16hi(aw[e]) * bf16hi(bw[e]);
+    }
+  }
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+  if (part == 0) {
+    delta[r] = acc;
+    float l2 = INFINITY;
+    if (i < Nq) {
+      const float l = lse[static_cast<size_t>(bh) * Nq + i];
+      if (l != -INFINITY) l2 = l * 1.4426950408889634f;
+    }
+    lse2[r] = l2;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV: one CTA per (key tile, batch, KV head)
+// ---------------------------------------------------------------------------
+template <int D>
+struct DkdvLayout {
+  using T = BwdTiles<D>;
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + T::kTileBytes;
+  static constexpr int kQ = kV + T::kTileBytes;              // 2 stages
+  static constexpr int kDO = kQ + 2 * T::kTileBytes;         // 2 stages
+  static constexpr int kVec = kDO + 2 * T::kTileBytes;       // 2 stages x {lse2, delta} x 128 floats
+  static constexpr int kBar = kVec + 2 * 2 * kT * 4;
+  // kv_full, q_full[2], q_empty[2], s_full, p_full, dp_full, ds_full, acc_done
+  static constexpr int kNumBars = 10;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kAlloc = kMisc + 16 + 1024;
+  static_assert(kAlloc <= 232448, "dynamic shared memory per block");
+  // TMEM: S^T | dP^T | dV | dK
+  static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDV = 256, kTmDK = 256 + D;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+// First query tile whose rows see key tile kt (bottom-right causal alignment:
+// query q sees key k iff k <= q + Nkv - Nq).
+__device__ __forceinline__ int first_query_tile(int kt, const BwdArgs& a) {
+  if (!a.causal) return 0;
+  const int q_min = kt * kT - (a.Nkv - a.Nq);   // smallest query that sees the tile's first key
+  return q_min <= 0 ? 0 : q_min / kT;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const BwdArgs a) {
+  using T = BwdTiles<D>;
+  using L = DkdvLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t sK = sb + L::kK, sV = sb + L::kV, sQ = sb + L::kQ, sDO = sb + L::kDO;
+  const float* vec = reinterpret_cast<const float*>(smem + L::kVec);
+  const uint32_t bar0 = sb + L::kBar;
+  const uint32_t BAR_KV = bar0;
+  auto BAR_QF = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto BAR_QE = [&](int s) { return bar0 + 8u * (3 + s); };
+  const uint32_t BAR_SF = bar0 + 8u * 5, BAR_PF = bar0 + 8u * 6, BAR_DPF = bar0 + 8u * 7,
+                 BAR_DSF = bar0 + 8u * 8, BAR_ACC = bar0 + 8u * 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // key tiles that more query tiles see come first (causal: the early ones)
+  const int bh_count = a.B * a.Hkv;
+  const int kt = static_cast<int>(blockIdx.x) / bh_count;
+  const int bhk = static_cast<int>(blockIdx.x) % bh_count;
+  const int b = bhk / a.Hkv, hkv = bhk % a.Hkv;
+  const int G = a.Hq / a.Hkv;
+  const int i0 = first_query_tile(kt, a);
+  const int per_head = i0 < a.n_qt ? a.n_qt - i0 : 0;
+  const int n_items = G * per_head;   // (query head of the group, query tile) pairs
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR_KV, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR_QF(s), 1);
+      mbar_init(BAR_QE(s), 1);
+    }
+    mbar_init(BAR_SF, 1);
+    mbar_init(BAR_PF, 128);
+    mbar_init(BAR_DPF, 1);
+    mbar_init(BAR_DSF, 128);
+    mbar_init(BAR_ACC, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmDO);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (n_items > 0 && warp == 0 && lane == 0) {
+    // ======================= TMA producer =======================
+    const int zk = b * a.Hkv + hkv;
+    mbar_arrive_expect_tx(BAR_KV, 2 * T::kTileBytes);
+    for (int c = 0; c < T::kChunks; ++c) {
+      tma_load_3d(sK + c * T::kChunkBytes, &tmK, BAR_KV, c * 64, kt * kT, zk);
+      tma_load_3d(sV + c * T::kChunkBytes, &tmV, BAR_KV, c * 64, kt * kT, zk);
+    }
+    for (int it = 0; it < n_items; ++it) {
+      const int s = it & 1;
+      if (!mbar_wait(BAR_QE(s), ((it >> 1) & 1u) ^ 1u, a.status, abort_flag)) break;
+      const int hq = hkv * G + it / per_head, qt = i0 + it % per_head;
+      const int zq = b * a.Hq + hq;
+      mbar_arrive_expect_tx(BAR_QF(s), 2 * T::kTileBytes + 2 * kT * 4);
+      for (int c = 0; c < T::kChunks; ++c) {
+        tma_load_3d(sQ + s * T::kTileBytes + c * T::kChunkBytes, &tmQ, BAR_QF(s), c * 64, qt * kT, zq);
+        tma_load_3d(sDO + s * T::kTileBytes + c * T::kChunkBytes, &tmDO, BAR_QF(s), c * 64, qt * kT, zq);
+      }
+      const size_t vrow = static_cast<size_t>(zq) * (a.n_qt * kT) + qt * kT;
+      bulk_load(sb + L::kVec + (s * 2 + 0) * kT * 4, a.lse2 + vrow, kT * 4, BAR_QF(s));
+      bulk_load(sb + L::kVec + (s * 2 + 1) * kT * 4, a.delta + vrow, kT * 4, BAR_QF(s));
+    }
+  } else if (n_items > 0 && warp == 1 && lane == 0) {
+    // ======================= MMA issuer =======================
+    constexpr uint32_t idesc_s = idesc_bf16_f32(kT, kT, false);   // 128 x 128, K-major B
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(kT, D, true);   // 128 x D, MN-major B
+    const uint64_t dK = smem_desc_sw128(sK, 16, 1024), dV = smem_desc_sw128(sV, 16, 1024);
+    const uint64_t dQk = smem_desc_sw128(sQ, 16, 1024), dDOk = smem_desc_sw128(sDO, 16, 1024);
+    const uint64_t dQm = smem_desc_sw128(sQ, T::kChunkBytes, 1024), dDOm = smem_desc_sw128(sDO, T::kChunkBytes, 1024);
+    constexpr uint64_t kStep = T::kTileBytes >> 4;
+    bool ok = mbar_wait(BAR_KV, 0, a.status, abort_flag);
+    ok = ok && mbar_wait(BAR_QF(0), 0, a.status, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      // S^T = K Q^T and dP^T = V dO^T for the first item
+      mma_kmajor_tile(tmem + L::kTmS, dK, dQk, T::kChunks, idesc_s, false);
+      mma_commit(BAR_SF);
+      mma_kmajor_tile(tmem + L::kTmDP, dV, dDOk, T::kChunks, idesc_s, false);
+      mma_commit(BAR_DPF);
+    }
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int s = it & 1, s1 = s ^ 1;
+      const uint32_t ph = it & 1u;
+      // dV += P^T dO once P^T is in TMEM
+      if (!(ok = mbar_wait(BAR_PF, ph, a.status, abort_flag))) break;
+      tc_fence_after();
+      mma_tmem_a(tmem + L::kTmDV, tmem + L::kTmS, dDOm + s * kStep, idesc_acc, it > 0);
+      // next item's S^T: the S buffer is free once the dV product above has read P^T
+      if (it + 1 < n_items) {
+        if (!(ok = mbar_wait(BAR_QF(s1), ((it + 1) >> 1) & 1u, a.status, abort_flag))) break;
+        tc_fence_after();
+        mma_kmajor_tile(tmem + L::kTmS, dK, dQk + s1 * kStep, T::kChunks, idesc_s, false);
+        mma_commit(BAR_SF);
+      }
+      // dK += dS^T Q once dS^T is in TMEM
+      if (!(ok = mbar_wait(BAR_DSF, ph, a.status, abort_flag))) break;
+      tc_fence_after();
+      mma_tmem_a(tmem + L::kTmDK, tmem + L::kTmDP, dQm + s * kStep, idesc_acc, it > 0);
+      mma_commit(BAR_QE(s));   // this stage's Q, dO, lse and delta are read once these land
+      if (it + 1 < n_items) {
+        mma_kmajor_tile(tmem + L::kTmDP, dV, dDOk + s1 * kStep, T::kChunks, idesc_s, false);
+        mma_commit(BAR_DPF);
+      }
+    }
+    if (ok) mma_commit(BAR_ACC);
+  } else if (warp >= kWorkWarp0) {
+    // ======================= per-key-row work + epilogue =======================
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;             // key row within the tile
+    const int key = kt * kT + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float c2 = a.scale_log2;
+    const int off = a.Nkv - a.Nq;
+    bool ok = true;
+    for (int it = 0; it < n_items; ++it) {
+      const int s = it & 1;
+      const uint32_t ph = it & 1u;
+      const int qt = i0 + it % per_head;
+      const int q0 = qt * kT;
+      // query columns c with key > q0 + c + off are masked: c < lim
+      const int lim = (a.causal ? key - off - q0 : 0);
+      const bool row_ok = key < a.Nkv;
+      const bool need_mask = !row_ok || lim > 0;
+      ok = mbar_wait(BAR_QF(s), (it >> 1) & 1u, a.status, abort_flag);
+      ok = ok && mbar_wait(BAR_SF, ph, a.status, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const float* l2v = vec + (s * 2 + 0) * kT;
+      const float* dlv = vec + (s * 2 + 1) * kT;
+      // P^T = exp2(S^T c2 - lse2[query]) for this key row, in two 64-column halves
+      uint32_t pk[2][32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sr[2][32];
+        tmem_ld32(tmem + L::kTmS + lane_off + h * 64, sr[0]);
+        tmem_ld32(tmem + L::kTmS + lane_off + h * 64 + 32, sr[1]);
+        tmem_wait_ld();
+        const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = h * 64 + 2 * e;
+          const float4 l4 = *reinterpret_cast<const float4*>(l2v + (c & ~3));
+          const float la = (c & 2) ? l4.z : l4.x, lb = (c & 2) ? l4.w : l4.y;
+          float p0 = ex2(fmaf(sv[2 * e], c2, -la));
+          float p1 = ex2(fmaf(sv[2 * e + 1], c2, -lb));
+          if (need_mask) {
+            p0 = (row_ok && c >= lim) ? p0 : 0.f;
+            p1 = (row_ok && c + 1 >= lim) ? p1 : 0.f;
+          }
+          pk[h][e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tmem + L::kTmS + lane_off + h * 32, pk[h]);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR_PF);
+      // dS^T = P^T o (dP^T - delta[query])
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_DPF, ph, a.status, abort_flag)))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t dr[2][32];
+        tmem_ld32(tmem + L::kTmDP + lane_off + h * 64, dr[0]);
+        tmem_ld32(tmem + L::kTmDP + lane_off + h * 64 + 32, dr[1]);
+        tmem_wait_ld();
+        const float* dpv = reinterpret_cast<const float*>(&dr[0][0]);
+        uint32_t dk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = h * 64 + 2 * e;
+          const float4 d4 = *reinterpret_cast<const float4*>(dlv + (c & ~3));
+          const float da = (c & 2) ? d4.z : d4.x, db = (c & 2) ? d4.w : d4.y;
+          dk[e] = pack_bf16x2(bf16lo(pk[h][e]) * (dpv[2 * e] - da), bf16hi(pk[h][e]) * (dpv[2 * e + 1] - db));
+        }
+        tmem_st32(tmem + L::kTmDP + lane_off + h * 32, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR_DSF);
+    }
+    // ---- epilogue: dK (times scale) and dV rows of this key tile
+    const bool have = ok && n_items > 0;
+    if (have) {
+      ok = __all_sync(0xffffffffu, mbar_wait(BAR_ACC, 0, a.status, abort_flag));
+      tc_fence_after();
+    }
+    // TMEM loads are warp-collective: every lane loads, only rows < Nkv store
+    const bool store = key < a.Nkv;
+    const size_t orow = (static_cast<size_t>(b) * a.Hkv + hkv) * a.Nkv + (store ? key : 0);
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      __nv_bfloat16* dst_row = (which ? a.dv : a.dk) + orow * D;
+      const float mul = which ? 1.f : a.scale;
+      const uint32_t src = tmem + (which ? L::kTmDV : L::kTmDK) + lane_off;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        if (have && ok) {
+          tmem_ld32(src + c * 32, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * mul, __uint_as_float(v[8 * e + 1]) * mul);
+            w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * mul, __uint_as_float(v[8 * e + 3]) * mul);
+            w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * mul, __uint_as_float(v[8 * e + 5]) * mul);
+            w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * mul, __uint_as_float(v[8 * e + 7]) * mul);
+            dst[e] = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ: one CTA per (query tile, batch, query head)
+// ---------------------------------------------------------------------------
+template <int D>
+struct DqLayout {
+  using T = BwdTiles<D>;
+  static constexpr int kQ = 0;
+  static constexpr int kDO = kQ + T::kTileBytes;
+  static constexpr int kK = kDO + T::kTileBytes;     // 2 stages
+  static constexpr int kV = kK + 2 * T::kTileBytes;  // 2 stages
+  static constexpr int kBar = kV + 2 * T::kTileBytes;
+  // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full, s_free, dp_full, ds_full, acc_done
+  static constexpr int kNumBars = 14;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kAlloc = kMisc + 16 + 1024;
+  static_assert(kAlloc <= 232448, "dynamic shared memory per block");
+  // TMEM: S | dP | dQ
+  static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDQ = 256;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+// Key tiles query tile [q0, q0 + 128) must visit (0 if no row sees a key).
+__device__ __forceinline__ int key_tiles_for(int q0, const BwdArgs& a) {
+  int kv_end = a.Nkv;
+  if (a.causal) kv_end = min(a.Nkv, min(q0 + kT, a.Nq) - 1 + (a.Nkv - a.Nq) + 1);
+  return kv_end <= 0 ? 0 : (kv_end + kT - 1) / kT;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const BwdArgs a) {
+  using T = BwdTiles<D>;
+  using L = DqLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t sQ = sb + L::kQ, sDO = sb + L::kDO, sK = sb + L::kK, sV = sb + L::kV;
+  const uint32_t bar0 = sb + L::kBar;
+  const uint32_t BAR_Q = bar0;
+  auto BAR_KF = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto BAR_KE = [&](int s) { return bar0 + 8u * (3 + s); };
+  auto BAR_VF = [&](int s) { return bar0 + 8u * (5 + s); };
+  auto BAR_VE = [&](int s) { return bar0 + 8u * (7 + s); };
+  const uint32_t BAR_SF = bar0 + 8u * 9, BAR_SFREE = bar0 + 8u * 10, BAR_DPF = bar0 + 8u * 11,
+                 BAR_DSF = bar0 + 8u * 12, BAR_ACC = bar0 + 8u * 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // later query tiles (more visible keys under causal masking) first
+  const int bh_count = a.B * a.Hq;
+  const int qt = a.n_qt - 1 - static_cast<int>(blockIdx.x) / bh_count;
+  const int bh = static_cast<int>(blockIdx.x) % bh_count;
+  const int b = bh / a.Hq, hq = bh % a.Hq;
+  const int hkv = hq / (a.Hq / a.Hkv);
+  const int q0 = qt * kT;
+  const int n = key_tiles_for(q0, a);
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR_Q, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR_KF(s), 1);
+      mbar_init(BAR_KE(s), 1);
+      mbar_init(BAR_VF(s), 1);
+      mbar_init(BAR_VE(s), 1);
+    }
+    mbar_init(BAR_SF, 1);
+    mbar_init(BAR_SFREE, 128);
+    mbar_init(BAR_DPF, 1);
+    mbar_init(BAR_DSF, 128);
+    mbar_init(BAR_ACC, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmDO);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (n > 0 && warp == 0 && lane == 0) {
+    // ======================= TMA producer =======================
+    const int zq = b * a.Hq + hq, zk = b * a.Hkv + hkv;
+    mbar_arrive_expect_tx(BAR_Q, 2 * T::kTileBytes);
+    for (int c = 0; c < T::kChunks; ++c) {
+      tma_load_3d(sQ + c * T::kChunkBytes, &tmQ, BAR_Q, c * 64, q0, zq);
+      tma_load_3d(sDO + c * T::kChunkBytes, &tmDO, BAR_Q, c * 64, q0, zq);
+    }
+    for (int j = 0; j < n; ++j) {
+      const int s = j & 1;
+      const uint32_t ph = ((j >> 1) & 1u) ^ 1u;
+      if (!mbar_wait(BAR_KE(s), ph, a.status, abort_flag)) break;
+      mbar_arrive_expect_tx(BAR_KF(s), T::kTileBytes);
+      for (int c = 0; c < T::kChunks; ++c)
+        tma_load_3d(sK + s * T::kTileBytes + c * T::kChunkBytes, &tmK, BAR_KF(s), c * 64, j * kT, zk);
+      if (!mbar_wait(BAR_VE(s), ph, a.status, abort_flag)) break;
+      mbar_arrive_expect_tx(BAR_VF(s), T::kTileBytes);
+      for (int c = 0; c < T::kChunks; ++c)
+        tma_load_3d(sV + s * T::kTileBytes + c * T::kChunkBytes, &tmV, BAR_VF(s), c * 64, j * kT, zk);
+    }
+  } else if (n > 0 && warp == 1 && lane == 0) {
+    // ======================= MMA issuer =======================
+    constexpr uint32_t idesc_s = idesc_bf16_f32(kT, kT, false);
+    constexpr uint32_t idesc_acc = idesc_bf16_f32(kT, D, true);
+    const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024), dDO = smem_desc_sw128(sDO, 16, 1024);
+    const uint64_t dKk = smem_desc_sw128(sK, 16, 1024), dVk = smem_desc_sw128(sV, 16, 1024);
+    const uint64_t dKm = smem_desc_sw128(sK, T::kChunkBytes, 1024);
+    constexpr uint64_t kStep = T::kTileBytes >> 4;
+    bool ok = mbar_wait(BAR_Q, 0, a.status, abort_flag);
+    ok = ok && mbar_wait(BAR_KF(0), 0, a.status, abort_flag);
+    ok = ok && mbar_wait(BAR_VF(0), 0, a.status, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      mma_kmajor_tile(tmem + L::kTmS, dQ, dKk, T::kChunks, idesc_s, false);     // S = Q K_0^T
+      mma_commit(BAR_SF);
+      mma_kmajor_tile(tmem + L::kTmDP, dDO, dVk, T::kChunks, idesc_s, false);   // dP = dO V_0^T
+      mma_commit(BAR_DPF);
+      if (n > 2) mma_commit(BAR_VE(0));   // release a stage only when a later load reuses it
+    }
+    for (int j = 0; j < n && ok; ++j) {
+      const int s = j & 1, s1 = s ^ 1;
+      const uint32_t ph = j & 1u, ph1 = ((j + 1) >> 1) & 1u;
+      // next S once the work warps hold this one in registers
+      if (j + 1 < n) {
+        if (!(ok = mbar_wait(BAR_SFREE, ph, a.status, abort_flag))) break;
+        if (!(ok = mbar_wait(BAR_KF(s1), ph1, a.status, abort_flag))) break;
+        tc_fence_after();
+        mma_kmajor_tile(tmem + L::kTmS, dQ, dKk + s1 * kStep, T::kChunks, idesc_s, false);
+        mma_commit(BAR_SF);
+      }
+      // dQ += dS K_j once dS is in TMEM
+      if (!(ok = mbar_wait(BAR_DSF, ph, a.status, abort_flag))) break;
+      tc_fence_after();
+      mma_tmem_a(tmem + L::kTmDQ, tmem + L::kTmDP, dKm + s * kStep, idesc_acc, j > 0);
+      if (j + 2 < n) mma_commit(BAR_KE(s));
+      if (j + 1 < n) {
+        if (!(ok = mbar_wait(BAR_VF(s1), ph1, a.status, abort_flag))) break;
+        tc_fence_after();
+        mma_kmajor_tile(tmem + L::kTmDP, dDO, dVk + s1 * kStep, T::kChunks, idesc_s, false);
+        mma_commit(BAR_DPF);
+        if (j + 3 < n) mma_commit(BAR_VE(s1));
+      }
+    }
+    if (ok) mma_commit(BAR_ACC);
+  } else if (warp >= kWorkWarp0) {
+    // ======================= per-query-row work + epilogue =======================
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int qrow = q0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float c2 = a.scale_log2;
+    const size_t vrow = static_cast<size_t>(bh) * (a.n_qt * kT) + qrow;   // padded rows exist for every r
+    const float l2 = a.lse2[vrow], dl = a.delta[vrow];
+    const int vis_end = a.causal ? min(a.Nkv, qrow + (a.Nkv - a.Nq) + 1) : a.Nkv;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const uint32_t ph = j & 1u;
+      ok = mbar_wait(BAR_SF, ph, a.status, abort_flag);
+      ok = ok && mbar_wait(BAR_DPF, ph, a.status, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int lim = vis_end - j * kT;   // visible key columns: [0, lim)
+      const bool need_mask = (j * kT + kT > a.Nkv) || (a.causal && j * kT + kT - 1 > q0 + (a.Nkv - a.Nq));
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sr[2][32], dr[2][32];
+        tmem_ld32(tmem + L::kTmS + lane_off + h * 64, sr[0]);
+        tmem_ld32(tmem + L::kTmS + lane_off + h * 64 + 32, sr[1]);
+        tmem_ld32(tmem + L::kTmDP + lane_off + h * 64, dr[0]);
+        tmem_ld32(tmem + L::kTmDP + lane_off + h * 64 + 32, dr[1]);
+        tmem_wait_ld();
+        if (h == 1) {
+          // all of S is in registers: the next Q K^T may overwrite it
+          tc_fence_before();
+          mbar_arrive(BAR_SFREE);
+        }
+        const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+        const float* dpv = reinterpret_cast<const float*>(&dr[0][0]);
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = h * 64 + 2 * e;
+          float p0 = ex2(fmaf(sv[2 * e], c2, -l2));
+          float p1 = ex2(fmaf(sv[2 * e + 1], c2, -l2));
+          if (need_mask) {
+            p0 = c < lim ? p0 : 0.f;
+            p1 = c + 1 < lim ? p1 : 0.f;
+          }
+          // dS rounds P to bf16 first, as the dK/dV kernel does
+          const uint32_t pb = pack_bf16x2(p0, p1);
+          pk[e] = pack_bf16x2(bf16lo(pb) * (dpv[2 * e] - dl), bf16hi(pb) * (dpv[2 * e + 1] - dl));
+        }
+        // dS over the dP buffer: columns [32h, 32h + 32) hold keys already read
+        tmem_st32(tmem + L::kTmDP + lane_off + h * 32, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR_DSF);
+    }
+    // ---- epilogue: dQ (times scale)
+    const bool have = ok && n > 0;
+    if (have) {
+      ok = __all_sync(0xffffffffu, mbar_wait(BAR_ACC, 0, a.status, abort_flag));
+      tc_fence_after();
+    }
+    // TMEM loads are warp-collective: every lane loads, only rows < Nq store
+    const bool store = qrow < a.Nq;
+    __nv_bfloat16* dst_row = a.dq + (static_cast<size_t>(bh) * a.Nq + (store ? qrow : 0)) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t v[32];
+      if (have && ok) {
+        tmem_ld32(tmem + L::kTmDQ + lane_off + c * 32, v);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
+      }
+      if (store) {
+        uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * a.scale, __uint_as_float(v[8 * e + 1]) * a.scale);
+          w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * a.scale, __uint_as_float(v[8 * e + 3]) * a.scale);
+          w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * a.scale, __uint_as_float(v[8 * e + 5]) * a.scale);
+          w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * a.scale, __uint_as_float(v[8 * e + 7]) * a.scale);
+          dst[e] = w;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+template <int D>
+ta_status launch_bwd_d(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                       const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv,
+                       int Nq, int Nkv, float scale, int causal, cudaStream_t stream) {
+  BwdArgs a;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nq = Nq;
+  a.Nkv = Nkv;
+  a.n_qt = (Nq + kT - 1) / kT;
+  a.n_kt = (Nkv + kT - 1) / kT;
+  a.causal = causal;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  const size_t padded = static_cast<size_t>(B) * Hq * a.n_qt * kT;
+  float* ws = static_cast<float*>(workspace);
+  a.delta = ws;
+  a.lse2 = ws + padded;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.status = device_status_ptr();
+  if (!a.status) return fail(TA_ERR_CUDA, "attn_bwd: device status word");
+
+  // delta and lse2 for every padded query row
+  {
+    const long long threads = static_cast<long long>(padded) * 8;
+    bwd_prep_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, ws, ws + padded, Nq,
+        a.n_qt * kT, static_cast<long long>(padded));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(TA_ERR_CUDA, "attn_bwd: prep launch", e);
+  }
+  CUtensorMap tq, tk, tv, tdo;
+  ta_status st;
+  if ((st = encode_rows_3d(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
+  if ((st = encode_rows_3d(&tdo, dout, D, Nq, B * Hq)) != TA_OK) return st;
+  if ((st = encode_rows_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_rows_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
+  static int done_kv[64] = {0}, done_q[64] = {0};
+  cudaError_t e = ensure_smem_limit(bwd_dkdv_kernel<D>, DkdvLayout<D>::kAlloc, done_kv);
+  if (e != cudaSuccess) return fail(TA_ERR_CUDA, "attn_bwd: shared-memory limit (dK/dV)", e);
+  e = ensure_smem_limit(bwd_dq_kernel<D>, DqLayout<D>::kAlloc, done_q);
+  if (e != cudaSuccess) return fail(TA_ERR_CUDA, "attn_bwd: shared-memory limit (dQ)", e);
+  const unsigned grid_kv = static_cast<unsigned>(a.n_kt) * static_cast<unsigned>(B * Hkv);
+  bwd_dkdv_kernel<D><<<grid_kv, kBwdThreads, DkdvLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return fail(TA_ERR_CUDA, "attn_bwd: dK/dV launch", e);
+  const unsigned grid_q = static_cast<unsigned>(a.n_qt) * static_cast<unsigned>(B * Hq);
+  bwd_dq_kernel<D><<<grid_q, kBwdThreads, DqLayout<D>::kAlloc, stream>>>(tq, tk, tv, tdo, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return fail(TA_ERR_CUDA, "attn_bwd: dQ launch", e);
+  return TA_OK;
+}
+
+}  // namespace
+
+size_t bwd_workspace_bytes(int B, int Hq, int Nq) {
+  const size_t padded = static_cast<size_t>(B) * Hq * ((Nq + kT - 1) / kT) * kT;
+  return ((2 * padded * sizeof(float)) + 255) & ~size_t(255);
+}
+
+ta_status launch_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                          const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv,
+                          int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream) {
+  if (d == 128)
+    return launch_bwd_d<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nkv, scale, causal,
+                             stream);
+  return launch_bwd_d<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, Hq, Hkv, Nq, Nkv, scale, causal, stream);
+}
+
+}  // namespace ta

@@ -484,28 +484,15 @@ __global__ void empty_keys_kernel(__nv_bfloat16* o, float* lse, size_t rows, int
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-static ta_status encode_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
-  PFN_encodeTiled enc = get_encode_tiled();
-  if (!enc) return fail(TA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slices)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? TA_OK : fail_cu(TA_ERR_CUDA, "cuTensorMapEncodeTiled", static_cast<int>(r));
-}
-
 template <int D>
 static ta_status launch_prefill_d(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                                   int Hkv, int Nq, int Nkv, float scale, int causal, cudaStream_t stream) {
   using L = PrefillLayout<D>;
   CUtensorMap tq, tk, tv;
   ta_status st;
-  if ((st = encode_3d(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
-  if ((st = encode_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
-  if ((st = encode_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_rows_3d(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
+  if ((st = encode_rows_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_rows_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
   static int attr_done[64] = {0};
   cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D>, L::kAlloc, attr_done);
   if (e != cudaSuccess) return fail(TA_ERR_CUDA, "prefill: shared-memory limit", e);

@@ -14,6 +14,11 @@ using PFN_encodeTiled = PFN_cuTensorMapEncodeTiled_v12000;
 // cuTensorMapEncodeTiled fetched through the runtime (no libcuda link).
 PFN_encodeTiled get_encode_tiled();
 
+// Tensor map over a bf16 array [slices, rows, d] (d contiguous) that loads
+// 128-row x 64-column boxes with the 128-byte swizzle; rows past `rows` read
+// as zero.
+ta_status encode_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices);
+
 // Records a description of the last host-side failure of this thread
 // (returned by ta_last_error) and returns `code`.
 ta_status fail(ta_status code, const char* where, cudaError_t err = cudaSuccess);
@@ -57,5 +62,10 @@ ta_status launch_gather_debug(const void* k_cache, const void* v_cache, const in
                               int max_pages, int num_pages_total, void* k_out, void* v_out, cudaStream_t stream);
 
 ta_status launch_selftest_wait(unsigned limit_us, cudaStream_t stream);
+
+size_t bwd_workspace_bytes(int B, int Hq, int Nq);
+ta_status launch_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                          const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv,
+                          int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);
 
 }  // namespace ta

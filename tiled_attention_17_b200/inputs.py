@@ -130,6 +130,12 @@ def _chunked_f32(seed_words, n: int, chunk: int = 1 << 22) -> np.ndarray:
     return out
 
 
+def grad_output(shape, seed: int) -> np.ndarray:
+    """Seeded loss gradient dO ~ N(0, 1) as bf16 bits (backward-pass inputs)."""
+    n = int(np.prod(shape))
+    return f32_to_bf16_bits(_chunked_f32([seed, 0xD0], n).reshape(shape))
+
+
 def random_prefill(B, Hq, Hkv, Nq, Nkv, d, seed, scale_k_rows_every=0, factor=1.0):
     """Small ad-hoc prefill inputs (tests): (q, k, v) uint16 bf16 bits."""
     cfg = PrefillConfig("adhoc", B, Hq, Hkv, Nq, Nkv, d, False, scale_k_rows_every, factor)
