@@ -7,7 +7,9 @@ One step = one pass of the whole hot path over one batch of synthetic input:
     16-token pages, lengths uniform on [512, 32768] (attn_paged_decode + combine).
 The headline metric is the prefill's TFLOP/s (visible (q, k) pairs, both
 contractions, 2 flop per multiply-add); the decode's KV GB/s is reported in
-the same line under "decode".  Inputs are resident in HBM when timing starts;
+the same line under "decode", and the backward pass (attn_bwd on the prefill
+workload, timed on its own after the step) under "backward".  Inputs are
+resident in HBM when timing starts;
 L2 (126 MB) is flushed by writing a 256 MB buffer before every step, outside
 the kernels' event brackets.  Kernel times are CUDA events on the launching
 stream; multi-GPU runs take the max over ranks.
@@ -332,6 +334,11 @@ def run_ours(args):
     if not args.no_e2e:
         e2e, dec_e2e = run_e2e(args, torch, binding, dev, stream, q_h, k_h, v_h, dinp, dist)
 
+    # ---- backward pass on the prefill workload (timed on its own, after the step)
+    bwd = None
+    if not args.no_backward:
+        bwd = run_backward(args, torch, binding, dev, stream, q, k, v, o, lse, flush, dist, rank, world, peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(q_h, k_h, v_h, args.cpu_stride)
@@ -355,6 +362,7 @@ def run_ours(args):
                                             recorded_traffic("decode_split_g4_kernel", "decode_paged.cu",
                                                              float(dinp.seq_lens.sum()))),
                        "e2e": dec_e2e},
+            "backward": bwd,
             "roofline": roofline("tensor", pre_per_gpu, peaks["bf16_tflops"], "TFLOP/s",
                                  recorded_traffic("prefill_fwd_kernel", "prefill_sm100.cu", float(c.B * c.Hq))),
             "peaks": {"source": peak_kind, "bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"],
@@ -369,6 +377,46 @@ def run_ours(args):
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def run_backward(args, torch, binding, dev, stream, q, k, v, o, lse, flush, dist, rank, world, peaks):
+    """attn_bwd on the causal prefill workload (o and lse from the step's
+    forward call, seeded dO): CUDA events around each call, L2 flushed before
+    every call, max over ranks.  FLOPs are the method's five products
+    (2.5x the forward count); the kernels compute seven."""
+    c = PREFILL
+    do_h = inputs.grad_output((c.B, c.Hq, c.Nq, c.d), seed=rank_seed(inputs.CONFIG_SEEDS["causal"] + 100, rank))
+    dout = torch.from_numpy(np.ascontiguousarray(do_h).view(np.int16)).view(torch.bfloat16).to(dev)
+    ws_bytes = binding.attn_bwd_workspace_size(c.B, c.Hq, c.Nq)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    gq, gk, gv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def call():
+        binding.attn_bwd(q, k, v, o, dout, lse, gq, gk, gv, ws, ws_bytes, c.B, c.Hq, c.Hkv, c.Nq, c.Nkv, c.d,
+                         c.scale, 1, stream)
+
+    for _ in range(3):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(dist, dev.index)
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+    (t,) = max_over_ranks([t], dist, device=dev)
+    flops = 2.5 * accounting.prefill_flops(c.B, c.Hq, c.Nq, c.Nkv, c.d, True)
+    per_gpu = flops / (t * 1e-3) / 1e12
+    return {"value": per_gpu * world, "unit": "TFLOP/s", "ms": t, "steps": steps,
+            "flops_per_call_per_gpu": flops, "flops_note": "5 products of the method (2.5x forward); 7 computed",
+            "gpu_launches_per_call": 3,
+            "roofline": roofline("tensor", per_gpu, peaks["bf16_tflops"], "TFLOP/s",
+                                 recorded_traffic("bwd_dkdv_kernel", "backward_sm100.cu", float(c.B * c.Hkv)))}
 
 
 def roofline(bound, achieved, peak, unit, traffic):
@@ -473,7 +521,15 @@ def run_ncu_case(args):
     def dev_bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    if args.ncu_case == "prefill":
+    if args.ncu_case == "backward":
+        c = PREFILL
+        q_h, k_h, v_h = inputs.prefill_inputs(c)
+        q, k, v = dev_bf16(q_h), dev_bf16(k_h), dev_bf16(v_h)
+        dout = dev_bf16(inputs.grad_output(q_h.shape, seed=inputs.CONFIG_SEEDS["causal"] + 100))
+        o, lse = binding.attention(q, k, v, True, c.scale)
+        for _ in range(args.reps):
+            binding.attention_backward(q, k, v, o, lse, dout, True, c.scale)
+    elif args.ncu_case == "prefill":
         c = PREFILL
         q_h, k_h, v_h = inputs.prefill_inputs(c)
         q, k, v = dev_bf16(q_h), dev_bf16(k_h), dev_bf16(v_h)
@@ -507,7 +563,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-stride", type=int, default=1, help="oracle baseline: every n-th query row")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--ncu-case", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--ncu-case", choices=["prefill", "decode", "backward"], default=None,
                     help="run a small single-kernel case for a profiler capture and exit")
     ap.add_argument("--reps", type=int, default=4)
     args = ap.parse_args(argv)

@@ -426,13 +426,14 @@ struct DqLayout {
   static constexpr int kK = kDO + T::kTileBytes;     // 2 stages
   static constexpr int kV = kK + 2 * T::kTileBytes;  // 2 stages
   static constexpr int kBar = kV + 2 * T::kTileBytes;
-  // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full, s_free, dp_full, ds_full, acc_done
-  static constexpr int kNumBars = 14;
+  // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full, loaded, dp_full, ds_full, ds_empty,
+  // acc_done
+  static constexpr int kNumBars = 15;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16 + 1024;
   static_assert(kAlloc <= 232448, "dynamic shared memory per block");
-  // TMEM: S | dP | dQ
-  static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDQ = 256;
+  // TMEM: S | dP | dQ | dS (bf16, 64 columns)
+  static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDQ = 256, kTmDS = 256 + D;
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -460,8 +461,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto BAR_KE = [&](int s) { return bar0 + 8u * (3 + s); };
   auto BAR_VF = [&](int s) { return bar0 + 8u * (5 + s); };
   auto BAR_VE = [&](int s) { return bar0 + 8u * (7 + s); };
-  const uint32_t BAR_SF = bar0 + 8u * 9, BAR_SFREE = bar0 + 8u * 10, BAR_DPF = bar0 + 8u * 11,
-                 BAR_DSF = bar0 + 8u * 12, BAR_ACC = bar0 + 8u * 13;
+  // loaded: S and dP of the current tile are in registers (both buffers may be
+  // overwritten); ds_empty: the dQ product has read the dS buffer
+  const uint32_t BAR_SF = bar0 + 8u * 9, BAR_LOADED = bar0 + 8u * 10, BAR_DPF = bar0 + 8u * 11,
+                 BAR_DSF = bar0 + 8u * 12, BAR_DSE = bar0 + 8u * 13, BAR_ACC = bar0 + 8u * 14;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -484,9 +487,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(BAR_VE(s), 1);
     }
     mbar_init(BAR_SF, 1);
-    mbar_init(BAR_SFREE, 128);
+    mbar_init(BAR_LOADED, 128);
     mbar_init(BAR_DPF, 1);
     mbar_init(BAR_DSF, 128);
+    mbar_init(BAR_DSE, 1);
     mbar_init(BAR_ACC, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -548,26 +552,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int j = 0; j < n && ok; ++j) {
       const int s = j & 1, s1 = s ^ 1;
       const uint32_t ph = j & 1u, ph1 = ((j + 1) >> 1) & 1u;
-      // next S once the work warps hold this one in registers
+      // next S and dP as soon as the work warps hold this tile's in registers
       if (j + 1 < n) {
-        if (!(ok = mbar_wait(BAR_SFREE, ph, a.status, abort_flag))) break;
+        if (!(ok = mbar_wait(BAR_LOADED, ph, a.status, abort_flag))) break;
         if (!(ok = mbar_wait(BAR_KF(s1), ph1, a.status, abort_flag))) break;
         tc_fence_after();
         mma_kmajor_tile(tmem + L::kTmS, dQ, dKk + s1 * kStep, T::kChunks, idesc_s, false);
         mma_commit(BAR_SF);
-      }
-      // dQ += dS K_j once dS is in TMEM
-      if (!(ok = mbar_wait(BAR_DSF, ph, a.status, abort_flag))) break;
-      tc_fence_after();
-      mma_tmem_a(tmem + L::kTmDQ, tmem + L::kTmDP, dKm + s * kStep, idesc_acc, j > 0);
-      if (j + 2 < n) mma_commit(BAR_KE(s));
-      if (j + 1 < n) {
         if (!(ok = mbar_wait(BAR_VF(s1), ph1, a.status, abort_flag))) break;
         tc_fence_after();
         mma_kmajor_tile(tmem + L::kTmDP, dDO, dVk + s1 * kStep, T::kChunks, idesc_s, false);
         mma_commit(BAR_DPF);
         if (j + 3 < n) mma_commit(BAR_VE(s1));
       }
+      // dQ += dS K_j once dS is in its buffer
+      if (!(ok = mbar_wait(BAR_DSF, ph, a.status, abort_flag))) break;
+      tc_fence_after();
+      mma_tmem_a(tmem + L::kTmDQ, tmem + L::kTmDS, dKm + s * kStep, idesc_acc, j > 0);
+      mma_commit(BAR_DSE);
+      if (j + 2 < n) mma_commit(BAR_KE(s));
     }
     if (ok) mma_commit(BAR_ACC);
   } else if (warp >= kWorkWarp0) {
@@ -590,6 +593,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const int lim = vis_end - j * kT;   // visible key columns: [0, lim)
       const bool need_mask = (j * kT + kT > a.Nkv) || (a.causal && j * kT + kT - 1 > q0 + (a.Nkv - a.Nq));
+      uint32_t pk[2][32];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t sr[2][32], dr[2][32];
@@ -599,13 +603,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(tmem + L::kTmDP + lane_off + h * 64 + 32, dr[1]);
         tmem_wait_ld();
         if (h == 1) {
-          // all of S is in registers: the next Q K^T may overwrite it
+          // S and dP are in registers: the next tile's products may overwrite them
           tc_fence_before();
-          mbar_arrive(BAR_SFREE);
+          mbar_arrive(BAR_LOADED);
         }
         const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
         const float* dpv = reinterpret_cast<const float*>(&dr[0][0]);
-        uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int c = h * 64 + 2 * e;
@@ -617,11 +620,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           // dS rounds P to bf16 first, as the dK/dV kernel does
           const uint32_t pb = pack_bf16x2(p0, p1);
-          pk[e] = pack_bf16x2(bf16lo(pb) * (dpv[2 * e] - dl), bf16hi(pb) * (dpv[2 * e + 1] - dl));
+          pk[h][e] = pack_bf16x2(bf16lo(pb) * (dpv[2 * e] - dl), bf16hi(pb) * (dpv[2 * e + 1] - dl));
         }
-        // dS over the dP buffer: columns [32h, 32h + 32) hold keys already read
-        tmem_st32(tmem + L::kTmDP + lane_off + h * 32, pk);
       }
+      // the previous dQ product must have read the dS buffer
+      if (j > 0) {
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_DSE, (j - 1) & 1u, a.status, abort_flag)))) break;
+        tc_fence_after();
+      }
+      tmem_st32(tmem + L::kTmDS + lane_off, pk[0]);
+      tmem_st32(tmem + L::kTmDS + lane_off + 32, pk[1]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR_DSF);
