@@ -416,7 +416,7 @@ def run_backward(args, torch, binding, dev, stream, q, k, v, o, lse, flush, dist
             "flops_per_call_per_gpu": flops, "flops_note": "5 products of the method (2.5x forward); 7 computed",
             "gpu_launches_per_call": 3,
             "roofline": roofline("tensor", per_gpu, peaks["bf16_tflops"], "TFLOP/s",
-                                 recorded_traffic("bwd_dkdv_kernel", "backward_sm100.cu", float(c.B * c.Hkv)))}
+                                 recorded_traffic("attn_bwd", "backward_sm100.cu", float(c.B * c.Hkv)))}
 
 
 def roofline(bound, achieved, peak, unit, traffic):
