@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for exact attention, its paged-decode form and its gradients.
+"""fp64 CPU oracle for exact attention, its paged forms (decode and varlen
+prefill) and its gradients.
 
 TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
 benchmark's CPU-baseline leg import this package; the library under
@@ -33,6 +34,10 @@ def _bind(path):
     L.oracle_paged_decode.argtypes = [c_u16p, c_u16p, c_u16p, c_i32p, c_i32p] + [ctypes.c_int] * 6 + [
         ctypes.c_int64, ctypes.c_double, c_i32p, ctypes.c_int, c_dp, c_dp]
     L.oracle_paged_decode.restype = ctypes.c_int
+    L.oracle_paged_prefill.argtypes = [c_u16p, c_u16p, c_u16p, c_i32p, c_i32p, c_i32p, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int64, ctypes.c_double, ctypes.c_int, c_i32p, ctypes.c_int, c_dp, c_dp]
+    L.oracle_paged_prefill.restype = ctypes.c_int
     L.oracle_attn_bwd.argtypes = [c_u16p, c_u16p, c_u16p, c_u16p] + [ctypes.c_int] * 6 + [
         ctypes.c_double, ctypes.c_int, c_i64p, ctypes.c_int64, c_dp, c_dp, c_dp]
     L.oracle_attn_bwd.restype = ctypes.c_int
@@ -154,6 +159,43 @@ def paged_decode(q, k_cache, v_cache, block_table, seq_lens, scale: float | None
     return o[:n], lse[:n]
 
 
+def paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens, seq_lens, causal: bool, scale: float | None = None,
+                  seqs=None, _L=None):
+    """Varlen prefill against the paged cache in fp64.
+
+    q [total_q, Hq, d] (bf16 bits, sequences packed by cu_seqlens [S+1]);
+    caches [P, Hkv, page, d]; block_table [S, max_pages]; seq_lens [S] keys per
+    sequence.  Returns o [total_q, Hq, d] and lse [total_q, Hq] (rows of
+    sequences outside `seqs` are zero).
+    """
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k_cache = np.ascontiguousarray(k_cache, dtype=np.uint16)
+    v_cache = np.ascontiguousarray(v_cache, dtype=np.uint16)
+    block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+    cu_seqlens = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    T, Hq, d = q.shape
+    P, Hkv, ps, _ = k_cache.shape
+    S = seq_lens.size
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if seqs is None:
+        n, sp = S, None
+    else:
+        seqs = np.ascontiguousarray(seqs, dtype=np.int32)
+        n, sp = seqs.size, _p(seqs, ctypes.c_int32)
+    o = np.zeros((max(T, 1), Hq, d), dtype=np.float64)
+    lse = np.zeros((max(T, 1), Hq), dtype=np.float64)
+    err = (_L or lib()).oracle_paged_prefill(_p(q, ctypes.c_uint16), _p(k_cache, ctypes.c_uint16),
+                                             _p(v_cache, ctypes.c_uint16), _p(block_table, ctypes.c_int32),
+                                             _p(cu_seqlens, ctypes.c_int32), _p(seq_lens, ctypes.c_int32), ps, S, T,
+                                             Hq, Hkv, d, block_table.shape[1], P, float(scale), int(bool(causal)), sp,
+                                             n, _p(o, ctypes.c_double), _p(lse, ctypes.c_double))
+    if err:
+        raise OracleError(f"oracle_paged_prefill failed with code {err}")
+    return o[:T], lse[:T]
+
+
 def attn_bwd(q, k, v, dout, causal: bool, scale: float | None = None, groups=None, _L=None):
     """Gradients (dq, dk, dv) of attention in fp64 for the loss gradient dout.
 
@@ -207,3 +249,6 @@ class Variant:
 
     def attn_bwd(self, *a, **kw):
         return attn_bwd(*a, _L=self._L, **kw)
+
+    def paged_prefill(self, *a, **kw):
+        return paged_prefill(*a, _L=self._L, **kw)

@@ -276,6 +276,81 @@ int oracle_paged_decode(const uint16_t *q, const uint16_t *k_cache, const uint16
 }
 
 /*
+ * Varlen (chunked) prefill against the paged cache: several sequences' new
+ * query rows, packed, each attending over its sequence's keys in the pool
+ * (the new tokens' K/V already appended).  The page structure is the paged
+ * decode's (paged-gather article, sections 2.1-2.4; GPU-optimisation tag
+ * page, PagedAttention); chunked prefill joins it to the prefill
+ * (LLM-inference article, section 3.2).
+ *
+ * Sequence s owns query rows [cu_seqlens[s], cu_seqlens[s+1]) of q
+ * [total_q, Hq, d] and seq_lens[s] keys.  Its logical K/V rows are gathered
+ * explicitly (oracle_paged_gather), then every query row follows the
+ * definition of oracle_attn with Nq = q_len and Nkv = seq_len: under the
+ * bottom-right causal alignment query i sits at position seq_len - q_len + i.
+ * seqs: optional subset of sequences (NULL = all).  o [total_q, Hq, d] and
+ * lse [total_q, Hq] (fp64) are written for the listed sequences' rows only.
+ */
+int oracle_paged_prefill(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                         const int32_t *block_table, const int32_t *cu_seqlens, const int32_t *seq_lens,
+                         int page_size, int num_seqs, int64_t total_q, int Hq, int Hkv, int d,
+                         int max_pages, int64_t num_pages_total, double scale, int causal,
+                         const int32_t *seqs, int nseqs, double *o, double *lse)
+{
+    if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv || page_size <= 0 || total_q < 0)
+        return ORACLE_ERR_ARG;
+    if (!seqs)
+        nseqs = num_seqs;
+    const int G = Hq / Hkv;
+    int err = ORACLE_OK;
+    const int64_t items = (int64_t)nseqs * Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t it = 0; it < items; ++it) {
+        int si = (int)(it / Hkv), hkv = (int)(it % Hkv);
+        int s = seqs ? seqs[si] : si;
+        if (s < 0 || s >= num_seqs || cu_seqlens[s] < 0 || cu_seqlens[s + 1] < cu_seqlens[s] ||
+            cu_seqlens[s + 1] > total_q) {
+#pragma omp atomic write
+            err = ORACLE_ERR_ARG;
+            continue;
+        }
+        int q0 = cu_seqlens[s], q_len = cu_seqlens[s + 1] - cu_seqlens[s];
+        int len = seq_lens[s] > 0 ? seq_lens[s] : 0;
+        size_t n = (size_t)(len > 0 ? len : 1);
+        uint16_t *kg = (uint16_t *)malloc(sizeof(uint16_t) * n * d);
+        uint16_t *vg = (uint16_t *)malloc(sizeof(uint16_t) * n * d);
+        double *sc = (double *)malloc(sizeof(double) * n);
+        if (!kg || !vg || !sc) {
+#pragma omp atomic write
+            err = ORACLE_ERR_NOMEM;
+        } else {
+            int e = oracle_paged_gather(k_cache, v_cache, block_table, seq_lens, s, hkv,
+                                        page_size, Hkv, d, max_pages, num_pages_total, kg, vg);
+            if (e) {
+#pragma omp atomic write
+                err = e;
+            } else {
+                for (int g = 0; g < G; ++g) {
+                    int hq = hkv * G + g;
+                    for (int i = 0; i < q_len; ++i) {
+                        size_t row = (size_t)(q0 + i) * Hq + hq;
+                        double l;
+                        attend_row(q + row * d, kg, vg, len, d, scale, visible_keys(i, q_len, len, causal),
+                                   sc, o + row * d, &l);
+                        if (lse)
+                            lse[row] = l;
+                    }
+                }
+            }
+        }
+        free(kg);
+        free(vg);
+        free(sc);
+    }
+    return err;
+}
+
+/*
  * Gradients of attention (the backward pass), plain chain rule in fp64.
  *
  * The kernel-fusion post (section 4, recomputation) fixes the strategy of the

@@ -301,6 +301,62 @@ def pin_paged_decode(orc):
             _close(lse[s, h], lb, what=f"decode lse seq {s} head {h}")
 
 
+def _varlen_batch(rng, q_lens, kv_lens, Hq, Hkv, d, page_size):
+    """Packed queries, per-sequence contiguous K/V and their paged copy."""
+    S = len(q_lens)
+    cu = np.zeros(S + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(q_lens)
+    q = _bf16(rng, (int(cu[-1]), Hq, d))
+    K = [_bf16(rng, (Hkv, L, d)) for L in kv_lens]
+    V = [_bf16(rng, (Hkv, L, d)) for L in kv_lens]
+    kc, vc, table, lens = _page(K, V, page_size, Hkv, rng)
+    return q, K, V, kc, vc, table, cu, lens
+
+
+def pin_paged_prefill_brute_force(orc):
+    # every packed query row against its own sequence's keys, by brute force on
+    # the contiguous rows (extended precision, explicit visibility count)
+    rng = np.random.Generator(np.random.PCG64(31))
+    for (q_lens, kv_lens, Hq, Hkv, d, ps) in [([3, 1, 4], [5, 2, 4], 2, 1, 3, 2),
+                                               ([2, 5], [7, 5], 4, 2, 2, 3),
+                                               ([4, 0, 3], [4, 3, 9], 1, 1, 4, 4)]:
+        for causal in (False, True):
+            q, K, V, kc, vc, table, cu, lens = _varlen_batch(rng, q_lens, kv_lens, Hq, Hkv, d, ps)
+            o, lse = orc.paged_prefill(q, kc, vc, table, cu, lens, causal, scale=0.9)
+            G = Hq // Hkv
+            for s, (ql, L) in enumerate(zip(q_lens, kv_lens)):
+                for h in range(Hq):
+                    for i in range(ql):
+                        row = cu[s] + i
+                        ob, lb = brute_row(widen(q[row, h]), widen(K[s][h // G]), widen(V[s][h // G]), 0.9,
+                                           _visible(i, ql, L, causal))
+                        _close(o[row, h], ob, what=f"paged prefill o seq {s} row {i} c={causal}")
+                        _close(lse[row, h], lb, what=f"paged prefill lse seq {s} row {i} c={causal}")
+
+
+def pin_paged_prefill_one_query_is_decode(orc):
+    # one new token per sequence is the paged decode
+    rng = np.random.Generator(np.random.PCG64(32))
+    kv_lens = [9, 1, 17, 6]
+    q, K, V, kc, vc, table, cu, lens = _varlen_batch(rng, [1] * 4, kv_lens, 4, 2, 3, 4)
+    o, lse = orc.paged_prefill(q, kc, vc, table, cu, lens, True, scale=0.7)
+    od, ld = orc.paged_decode(q, kc, vc, table, lens, scale=0.7)
+    _close(o, od, what="one query vs decode o")
+    _close(lse, ld, what="one query vs decode lse")
+
+
+def pin_paged_prefill_matches_dense(orc):
+    # one sequence through the pool equals the contiguous attention of its rows
+    rng = np.random.Generator(np.random.PCG64(33))
+    for causal in (False, True):
+        q, K, V, kc, vc, table, cu, lens = _varlen_batch(rng, [2, 6], [3, 11], 2, 2, 4, 4)
+        o, lse = orc.paged_prefill(q, kc, vc, table, cu, lens, causal, scale=0.5)
+        qs = np.ascontiguousarray(q[cu[1]:cu[2]].transpose(1, 0, 2))[None]
+        od, ld = orc.attn(qs, K[1][None], V[1][None], causal, scale=0.5)
+        _close(o[cu[1]:cu[2]], od[0].transpose(1, 0, 2), what="paged prefill vs dense o")
+        _close(lse[cu[1]:cu[2]], ld[0].T, what="paged prefill vs dense lse")
+
+
 # ---------------------------------------------------------------------------
 # Backward pass (gradients of attention)
 # ---------------------------------------------------------------------------
@@ -446,4 +502,5 @@ BWD_PINS = [pin_bwd_finite_differences, pin_bwd_single_key, pin_bwd_scale_zero,
 ALL_PINS = [pin_brute_force, pin_large_scores, pin_handpicked, pin_rows_of_p_sum_to_one,
             pin_constant_v, pin_permutation_invariance, pin_single_key, pin_scale_zero,
             pin_causal_row0, pin_identical_keys, pin_online_recurrence, pin_paged_gather,
-            pin_paged_decode] + BWD_PINS
+            pin_paged_decode, pin_paged_prefill_brute_force, pin_paged_prefill_one_query_is_decode,
+            pin_paged_prefill_matches_dense] + BWD_PINS

@@ -24,6 +24,9 @@ MUTANTS = {
     "page_row_index": ("(size_t)(t % page_size)) * d;", "(size_t)(t / page_size)) * d;"),
     "sum_without_max": ("l += exp(s[j] - m);", "l += exp(s[j]);"),
     "decode_head_mapping": ("int hq = hkv * G + g;", "int hq = g * Hkv + hkv;"),
+    # varlen prefill over the paged cache
+    "pp_alignment_swapped": ("visible_keys(i, q_len, len, causal)", "visible_keys(i, len, q_len, causal)"),
+    "pp_row_offset_ignored": ("size_t row = (size_t)(q0 + i) * Hq + hq;", "size_t row = (size_t)i * Hq + hq;"),
     # backward pass
     "bwd_dq_without_scale": ("dqi[t] += scale * ds *", "dqi[t] += ds *"),
     "bwd_no_jacobian_row_term": ("double ds = p[j] * (dp[j] - rowterm);", "double ds = p[j] * dp[j];"),
