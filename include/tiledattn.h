@@ -92,6 +92,38 @@ ta_status attn_fwd(const void *q, const void *k, const void *v, void *o, float *
                    float scale, int causal, ta_stream_t stream);
 
 /*
+ * attn_paged_prefill - varlen (chunked) prefill against the paged KV cache:
+ * the new query tokens of several sequences, packed, attend over their
+ * sequences' keys in the page pool (chunked prefill, LLM-inference article
+ * section 3.2; PagedAttention, GPU-optimisation tag page; block gather,
+ * paged-gather article section 2).  The new tokens' K/V must already be in
+ * the pool.
+ *
+ *   q, o         [total_q, Hq, d] bf16, sequences packed: sequence s owns rows
+ *                [cu_seqlens[s], cu_seqlens[s+1])
+ *   lse          [total_q, Hq] fp32 (may be NULL)
+ *   cu_seqlens   [num_seqs + 1] int32, nondecreasing, cu_seqlens[num_seqs] <=
+ *                total_q; every q_len = cu_seqlens[s+1] - cu_seqlens[s] <=
+ *                max_q_len (max_q_len sizes the grid)
+ *   seq_lens     [num_seqs] int32: keys of sequence s (0 <= len <=
+ *                max_pages * page_size)
+ *   k_cache, v_cache, block_table: as attn_paged_decode.
+ *
+ * Query i of sequence s sits at position seq_lens[s] - q_len + i: with causal
+ * = 1 it sees keys j <= that position (the bottom-right alignment of
+ * attn_fwd), with causal = 0 all keys.  A row with no visible key gets O = 0,
+ * lse = -inf.  Supported: d in {64, 128}, page_size in {8, 16, 32, 64},
+ * Hq % Hkv == 0.  Out-of-range lengths, offsets and table entries are clamped
+ * on the device (never dereferenced) and flagged in the library status word
+ * (ta_device_status).  Allocates nothing.
+ */
+ta_status attn_paged_prefill(const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *block_table, const int32_t *cu_seqlens, const int32_t *seq_lens,
+                             int page_size, int num_seqs, int total_q, int max_q_len, int Hq, int Hkv, int d,
+                             int max_pages, int num_pages_total, float scale, int causal, void *o,
+                             float *lse, ta_stream_t stream);
+
+/*
  * Bytes of device workspace attn_bwd needs (256-byte multiple): two fp32
  * values per query row, rows padded to a multiple of 128 per head.  Pure
  * host arithmetic; returns 0 for invalid sizes.

@@ -33,6 +33,39 @@ def test_header_functions_exported(lib):
         assert isinstance(getattr(L, n), ctypes._CFuncPtr)
 
 
+def declared_signatures():
+    """{name: [parameter types]} parsed from the header's prototypes."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b([a-z_][a-z0-9_ ]*?[ *]+)([a-z_][a-z0-9_]*)\s*\(([^;{]*?)\)\s*;", text):
+        name, params = m.group(2), " ".join(m.group(3).split())
+        if name == "defined":
+            continue
+        out[name] = [] if params in ("", "void") else [p.strip() for p in params.split(",")]
+    return out
+
+
+def test_binding_argtypes_match_header(lib):
+    # every ctypes prototype has the header's parameter count, and pointer /
+    # integer / float / size_t kinds in the same places
+    import ctypes
+    L = lib.load()
+    sigs = declared_signatures()
+    assert set(sigs) == set(lib.EXPORTS)
+    for name, params in sigs.items():
+        argtypes = getattr(L, name).argtypes or []
+        assert len(argtypes) == len(params), (name, len(argtypes), params)
+        for p, t in zip(params, argtypes):
+            if "*" in p or p.startswith("ta_stream_t"):
+                assert t is ctypes.c_void_p or issubclass(t, ctypes._Pointer) or t is ctypes.c_char_p, (name, p, t)
+            elif p.startswith("float"):
+                assert t is ctypes.c_float, (name, p, t)
+            elif p.startswith("size_t"):
+                assert t is ctypes.c_size_t, (name, p, t)
+            else:
+                assert t in (ctypes.c_int, ctypes.c_uint), (name, p, t)
+
+
 def test_status_strings(lib):
     assert lib.ta_status_string(0) == "TA_OK"
     assert lib.ta_status_string(4) == "TA_ERR_BAD_BLOCK_TABLE"

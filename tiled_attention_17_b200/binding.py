@@ -25,6 +25,7 @@ TA_DEV_BAD_BLOCK_TABLE = 2
 TA_DEV_BAD_SEQ_LEN = 4
 
 EXPORTS = ["ta_status_string", "ta_version", "ta_last_error", "attn_fwd", "attn_bwd_workspace_size", "attn_bwd",
+           "attn_paged_prefill",
            "attn_paged_decode_workspace_size",
            "attn_paged_decode", "attn_paged_decode_noalloc", "attn_paged_decode_check", "attn_paged_gather_debug",
            "ta_device_status", "ta_selftest_bounded_wait"]
@@ -57,6 +58,8 @@ def load(path: str | None = None):
     L.ta_last_error.restype = ctypes.c_char_p
     L.attn_fwd.argtypes = [vp, vp, vp, vp, vp] + [i32] * 6 + [f32, i32, vp]
     L.attn_fwd.restype = i32
+    L.attn_paged_prefill.argtypes = [vp] * 6 + [i32] * 9 + [f32, i32, vp, vp, vp]
+    L.attn_paged_prefill.restype = i32
     L.attn_bwd_workspace_size.argtypes = [i32] * 3
     L.attn_bwd_workspace_size.restype = sz
     L.attn_bwd.argtypes = [vp] * 10 + [sz] + [i32] * 6 + [f32, i32, vp]
@@ -123,6 +126,18 @@ def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream=None
                            float(scale), int(causal), _stream(stream))
     if check:
         _check("attn_fwd", code)
+    return code
+
+
+def attn_paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens, seq_lens, page_size, num_seqs, total_q,
+                       max_q_len, Hq, Hkv, d, max_pages, num_pages_total, scale, causal, o, lse, stream=None,
+                       check=True) -> int:
+    code = load().attn_paged_prefill(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cu_seqlens),
+                                     _ptr(seq_lens), page_size, num_seqs, total_q, max_q_len, Hq, Hkv, d, max_pages,
+                                     num_pages_total, float(scale), int(causal), _ptr(o), _ptr(lse),
+                                     _stream(stream))
+    if check:
+        _check("attn_paged_prefill", code)
     return code
 
 
@@ -234,6 +249,24 @@ def attention_backward(q, k, v, o, lse, dout, causal: bool, scale: float | None 
     attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace.numel(), B, Hq, Hkv, Nq, Nkv, d, scale,
              causal, stream)
     return dq, dk, dv
+
+
+def paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens, seq_lens, max_q_len: int, causal: bool,
+                  scale: float | None = None, out=None, lse=None, stream=None):
+    """q [total_q, Hq, d] packed by cu_seqlens [S+1] (int32, device); caches
+    [P, Hkv, page, d]; block_table [S, max_pages]; seq_lens [S] -> (o, lse)."""
+    import torch
+    T, Hq, d = q.shape
+    P, Hkv, ps, _ = k_cache.shape
+    S = seq_lens.shape[0]
+    if scale is None:
+        scale = d ** -0.5
+    o = out if out is not None else torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    attn_paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens, seq_lens, ps, S, T, max_q_len, Hq, Hkv, d,
+                       block_table.shape[1], P, scale, causal, o, lse, stream)
+    return o, lse
 
 
 def paged_decode(q, k_cache, v_cache, block_table, seq_lens, scale: float | None = None, workspace=None,

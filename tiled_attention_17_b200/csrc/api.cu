@@ -50,17 +50,29 @@ PFN_encodeTiled get_encode_tiled() {
   return fn;
 }
 
-ta_status encode_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
+ta_status encode_bf16_tiled(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                            const uint64_t* strides_bytes, const uint32_t* box) {
   PFN_encodeTiled enc = get_encode_tiled();
   if (!enc) return fail(TA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slices)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  cuuint64_t d[5], st[4];
+  cuuint32_t bx[5], estr[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    estr[i] = 1;
+    if (i + 1 < rank) st[i] = strides_bytes[i];
+  }
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d,
+                   st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? TA_OK : fail_cu(TA_ERR_CUDA, "cuTensorMapEncodeTiled", static_cast<int>(r));
+}
+
+ta_status encode_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows), static_cast<uint64_t>(slices)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(rows) * d * 2};
+  const uint32_t box[3] = {64, 128, 1};
+  return encode_bf16_tiled(map, base, 3, dims, strides, box);
 }
 
 static thread_local char g_last_error[256] = "";
@@ -119,6 +131,32 @@ ta_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* 
   const long long pairs = (static_cast<long long>(Nq) + 255) / 256;
   if (pairs * B * Hq > INT32_MAX) return TA_ERR_UNSUPPORTED;
   return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ta_status attn_paged_prefill(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                             const int32_t* cu_seqlens, const int32_t* seq_lens, int page_size, int num_seqs,
+                             int total_q, int max_q_len, int Hq, int Hkv, int d, int max_pages, int num_pages_total,
+                             float scale, int causal, void* o, float* lse, ta_stream_t stream) {
+  if (num_seqs < 0 || total_q < 0 || max_q_len < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || page_size <= 0 ||
+      max_pages <= 0 || num_pages_total <= 0)
+    return TA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return TA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return TA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return TA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return TA_ERR_UNSUPPORTED;
+  if (page_size != 8 && page_size != 16 && page_size != 32 && page_size != 64) return TA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_pages) * page_size > (1 << 30) || Hq > 65535) return TA_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || total_q == 0 || max_q_len == 0) return TA_OK;
+  const long long pairs = (static_cast<long long>(max_q_len) + 255) / 256;
+  if (pairs * num_seqs * Hq > INT32_MAX) return TA_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !block_table || !cu_seqlens || !seq_lens || !o) return TA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) || (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return TA_ERR_INVALID_ARG;
+  return launch_paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens, seq_lens, page_size, num_seqs, total_q,
+                              max_q_len, Hq, Hkv, d, max_pages, num_pages_total, scale, causal, o, lse,
+                              reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Nq) {

@@ -88,21 +88,28 @@ struct PrefillArgs {
   float scale;       // natural-log scale (for lse)
   float scale_log2;  // scale * log2(e)
   unsigned* status;
+  // varlen prefill over the paged cache (kPaged): the queries of num_seqs
+  // sequences are packed as [total_q, Hq, d] (o and lse the same way), and
+  // sequence s owns rows [cu_seqlens[s], cu_seqlens[s+1]) and seq_lens[s] keys
+  const int32_t* block_table;
+  const int32_t* cu_seqlens;
+  const int32_t* seq_lens;
+  int num_seqs, total_q, max_q_len, page_size, max_pages, num_pages_total;
 };
 
 // Number of K/V tiles query tile [q0, q0+128) must visit (0 if it has no rows
 // or every row is fully masked).
-__device__ __forceinline__ int kv_tiles_for(int q0, const PrefillArgs& a) {
-  if (q0 >= a.Nq) return 0;
-  int kv_end = a.Nkv;
-  if (a.causal) {
-    int last = min(q0 + kBM, a.Nq) - 1;
-    kv_end = min(a.Nkv, last + (a.Nkv - a.Nq) + 1);
+__device__ __forceinline__ int kv_tiles_for(int q0, int Nq, int Nkv, int causal) {
+  if (q0 >= Nq) return 0;
+  int kv_end = Nkv;
+  if (causal) {
+    int last = min(q0 + kBM, Nq) - 1;
+    kv_end = min(Nkv, last + (Nkv - Nq) + 1);
   }
   return kv_end <= 0 ? 0 : (kv_end + kBN - 1) / kBN;
 }
 
-template <int D>
+template <int D, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
@@ -127,14 +134,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: heavy (late) query pairs first so causal tails are short
-  const int bh_count = a.B * a.Hq;
+  // ---- work item: heavy (late) query pairs first so causal tails are short.
+  // Dense: (pair, batch, head).  Paged: (pair, sequence, head), with the
+  // sequence's query and key counts read (and range-checked) here.
+  const int bh_count = (kPaged ? a.num_seqs : a.B) * a.Hq;
   const int pair = a.n_pairs - 1 - static_cast<int>(blockIdx.x) / bh_count;
   const int bh = static_cast<int>(blockIdx.x) % bh_count;
-  const int b = bh / a.Hq, hq = bh % a.Hq;
+  const int b = bh / a.Hq, hq = bh % a.Hq;   // b = sequence when paged
   const int hkv = hq / (a.Hq / a.Hkv);
+  int Nq = a.Nq, Nkv = a.Nkv;
+  int q_base = 0;                  // packed row of the sequence's first query (paged)
+  if constexpr (kPaged) {
+    int lo = a.cu_seqlens[b], hi = a.cu_seqlens[b + 1];
+    int len = a.seq_lens[b];
+    unsigned bad = 0;
+    if (lo < 0 || lo > a.total_q || hi < lo || hi > a.total_q || hi - lo > a.max_q_len) bad |= kDevBadSeqLen;
+    if (len < 0 || len > a.max_pages * a.page_size) bad |= kDevBadSeqLen;
+    lo = min(max(lo, 0), a.total_q);
+    hi = min(max(hi, lo), min(a.total_q, lo + a.max_q_len));
+    len = min(max(len, 0), a.max_pages * a.page_size);
+    if (bad && threadIdx.x == 0 && pair == 0 && hq == 0) atomicOr(a.status, bad);
+    q_base = lo;
+    Nq = hi - lo;
+    Nkv = len;
+  }
   const int q0_0 = pair * 2 * kBM, q0_1 = q0_0 + kBM;
-  const int nt_0 = kv_tiles_for(q0_0, a), nt_1 = kv_tiles_for(q0_1, a);
+  if (kPaged && q0_0 >= Nq) return;   // this sequence has fewer query pairs (uniform per CTA)
+  const int nt_0 = kv_tiles_for(q0_0, Nq, Nkv, a.causal), nt_1 = kv_tiles_for(q0_1, Nq, Nkv, a.causal);
   const int n_max = max(nt_0, nt_1);
 
   // ---- setup
@@ -174,14 +200,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
     // ======================= TMA producer =======================
       const int zq = b * a.Hq + hq, zk = b * a.Hkv + hkv;
-      const uint32_t qbytes = static_cast<uint32_t>((q0_0 < a.Nq) + (q0_1 < a.Nq)) * L::kTileBytes;
+      const uint32_t qbytes = static_cast<uint32_t>((q0_0 < Nq) + (q0_1 < Nq)) * L::kTileBytes;
       mbar_arrive_expect_tx(BAR_Q(), qbytes);
       for (int t = 0; t < 2; ++t) {
         const int q0 = t ? q0_1 : q0_0;
-        if (q0 >= a.Nq) continue;
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * 64, q0, zq);
+        if (q0 >= Nq) continue;
+        for (int c = 0; c < L::kChunks; ++c) {
+          if constexpr (kPaged)   // packed [total_q, Hq, d]: box of 128 rows of one head
+            tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * 64, hq, q_base + q0);
+          else
+            tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * 64, q0, zq);
+        }
       }
+      // K or V tile j into ring slot `dst`: one tile box (dense), or one box per
+      // page through the block table (paged).  Pages past the sequence, and
+      // entries outside the pool (flagged), read page 0: the pool's contents
+      // are finite and those keys are masked.
+      auto load_kv = [&](const CUtensorMap* tm, uint32_t dst, uint32_t bar, int j) {
+        if constexpr (kPaged) {
+          const int per_tile = kBN / a.page_size;
+          for (int p = 0; p < per_tile; ++p) {
+            const int logical = j * per_tile + p;
+            int phys = 0;
+            if (logical * a.page_size < Nkv) {
+              phys = a.block_table[static_cast<size_t>(b) * a.max_pages + logical];
+              if (phys < 0 || phys >= a.num_pages_total) {
+                atomicOr(a.status, kDevBadBlockTable);
+                phys = 0;
+              }
+            }
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_load_4d(dst + c * L::kChunkBytes + p * a.page_size * 128, tm, bar, c * 64, 0, hkv, phys);
+          }
+        } else {
+          for (int c = 0; c < L::kChunks; ++c) tma_load_3d(dst + c * L::kChunkBytes, tm, bar, c * 64, j * kBN, zk);
+        }
+      };
       bool ok = true;
       for (int j = 0; j < n_max && ok; ++j) {
         const int s = j % L::kStages;
@@ -189,13 +243,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(BAR_KE(s), ph ^ 1u, a.status, abort_flag);
         if (!ok) break;
         mbar_arrive_expect_tx(BAR_KF(s), L::kTileBytes);
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(sK + s * L::kTileBytes + c * L::kChunkBytes, &tmK, BAR_KF(s), c * 64, j * kBN, zk);
+        load_kv(&tmK, sK + s * L::kTileBytes, BAR_KF(s), j);
         ok = mbar_wait(BAR_VE(s), ph ^ 1u, a.status, abort_flag);
         if (!ok) break;
         mbar_arrive_expect_tx(BAR_VF(s), L::kTileBytes);
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(sV + s * L::kTileBytes + c * L::kChunkBytes, &tmV, BAR_VF(s), c * 64, j * kBN, zk);
+        load_kv(&tmV, sV + s * L::kTileBytes, BAR_VF(s), j);
       }
       // drain: make sure no copy into this CTA's smem is still in flight at exit
       mbar_wait(BAR_Q(), 0, a.status, abort_flag);
@@ -302,9 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + (t == 0 ? L::kTmS0 : L::kTmS1) + lane_off;
     const uint32_t tO = tmem + (t == 0 ? L::kTmO0 : L::kTmO1) + lane_off;
     const int n = t ? nt_1 : nt_0;
-    const int off = a.Nkv - a.Nq;
+    const int off = Nkv - Nq;
     // visible keys of this row: [0, vis_end)
-    const int vis_end = a.causal ? min(a.Nkv, qrow + off + 1) : a.Nkv;
+    const int vis_end = a.causal ? min(Nkv, qrow + off + 1) : Nkv;
     const float c2 = a.scale_log2;
 
     float m = -INFINITY;  // running max of the raw scores q.k
@@ -325,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // tile-uniform: does any row of this tile have masked keys in tile j?
       const int kv0 = j * kBN;
       const bool need_mask =
-          (kv0 + kBN > a.Nkv) || (a.causal && kv0 + kBN - 1 > q0 + off);
+          (kv0 + kBN > Nkv) || (a.causal && kv0 + kBN - 1 > q0 + off);
       const int lim = vis_end - kv0;  // visible columns of this tile for this row: [0, lim)
       if (need_mask) {
 #pragma unroll
@@ -432,8 +484,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
     }
-    const bool store = qrow < a.Nq;
-    const size_t orow = (static_cast<size_t>(b) * a.Hq + hq) * a.Nq + qrow;
+    const bool store = qrow < Nq;
+    // output row: [B, Hq, Nq] (dense) or packed [total_q, Hq] (paged)
+    const size_t orow = kPaged ? static_cast<size_t>(q_base + (store ? qrow : 0)) * a.Hq + hq
+                               : (static_cast<size_t>(b) * a.Hq + hq) * Nq + qrow;
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
     __nv_bfloat16* optr = a.o + orow * D;
 #pragma unroll 1
@@ -494,9 +548,9 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   if ((st = encode_rows_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
   if ((st = encode_rows_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
   static int attr_done[64] = {0};
-  cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D>, L::kAlloc, attr_done);
+  cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, false>, L::kAlloc, attr_done);
   if (e != cudaSuccess) return fail(TA_ERR_CUDA, "prefill: shared-memory limit", e);
-  PrefillArgs a;
+  PrefillArgs a = {};
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.B = B;
@@ -511,9 +565,77 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   a.status = device_status_ptr();
   if (!a.status) return fail(TA_ERR_CUDA, "prefill: device status word");
   const unsigned grid = static_cast<unsigned>(a.n_pairs) * static_cast<unsigned>(B * Hq);
-  prefill_fwd_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
+  prefill_fwd_kernel<D, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "prefill: launch", e);
+}
+
+template <int D>
+static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, const void* v_cache,
+                                        const int32_t* block_table, const int32_t* cu_seqlens,
+                                        const int32_t* seq_lens, int page_size, int num_seqs, int total_q,
+                                        int max_q_len, int Hq, int Hkv, int max_pages, int num_pages_total,
+                                        float scale, int causal, void* o, float* lse, cudaStream_t stream) {
+  using L = PrefillLayout<D>;
+  CUtensorMap tq, tk, tv;
+  ta_status st;
+  {  // packed queries [total_q, Hq, d]: boxes of 128 rows of one head
+    const uint64_t dims[3] = {D, static_cast<uint64_t>(Hq), static_cast<uint64_t>(total_q)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(Hq) * D * 2};
+    const uint32_t box[3] = {64, 1, 128};
+    if ((st = encode_bf16_tiled(&tq, q, 3, dims, strides, box)) != TA_OK) return st;
+  }
+  {  // pool [P, Hkv, page, d]: boxes of one page of one KV head
+    const uint64_t dims[4] = {D, static_cast<uint64_t>(page_size), static_cast<uint64_t>(Hkv),
+                              static_cast<uint64_t>(num_pages_total)};
+    const uint64_t strides[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(page_size) * D * 2,
+                                 static_cast<uint64_t>(Hkv) * page_size * D * 2};
+    const uint32_t box[4] = {64, static_cast<uint32_t>(page_size), 1, 1};
+    if ((st = encode_bf16_tiled(&tk, k_cache, 4, dims, strides, box)) != TA_OK) return st;
+    if ((st = encode_bf16_tiled(&tv, v_cache, 4, dims, strides, box)) != TA_OK) return st;
+  }
+  static int attr_done[64] = {0};
+  cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, true>, L::kAlloc, attr_done);
+  if (e != cudaSuccess) return fail(TA_ERR_CUDA, "paged prefill: shared-memory limit", e);
+  PrefillArgs a = {};
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.B = 1;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.n_pairs = (max_q_len + 2 * kBM - 1) / (2 * kBM);
+  a.causal = causal;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.status = device_status_ptr();
+  if (!a.status) return fail(TA_ERR_CUDA, "paged prefill: device status word");
+  a.block_table = block_table;
+  a.cu_seqlens = cu_seqlens;
+  a.seq_lens = seq_lens;
+  a.num_seqs = num_seqs;
+  a.total_q = total_q;
+  a.max_q_len = max_q_len;
+  a.page_size = page_size;
+  a.max_pages = max_pages;
+  a.num_pages_total = num_pages_total;
+  const unsigned grid = static_cast<unsigned>(a.n_pairs) * static_cast<unsigned>(num_seqs * Hq);
+  prefill_fwd_kernel<D, true><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "paged prefill: launch", e);
+}
+
+ta_status launch_paged_prefill(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                               const int32_t* cu_seqlens, const int32_t* seq_lens, int page_size, int num_seqs,
+                               int total_q, int max_q_len, int Hq, int Hkv, int d, int max_pages,
+                               int num_pages_total, float scale, int causal, void* o, float* lse,
+                               cudaStream_t stream) {
+  if (d == 128)
+    return launch_paged_prefill_d<128>(q, k_cache, v_cache, block_table, cu_seqlens, seq_lens, page_size, num_seqs,
+                                       total_q, max_q_len, Hq, Hkv, max_pages, num_pages_total, scale, causal, o,
+                                       lse, stream);
+  return launch_paged_prefill_d<64>(q, k_cache, v_cache, block_table, cu_seqlens, seq_lens, page_size, num_seqs,
+                                    total_q, max_q_len, Hq, Hkv, max_pages, num_pages_total, scale, causal, o, lse,
+                                    stream);
 }
 
 ta_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,

@@ -19,6 +19,11 @@ PFN_encodeTiled get_encode_tiled();
 // as zero.
 ta_status encode_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices);
 
+// General bf16 tensor map (rank 2-5, 128-byte swizzle, zero fill out of
+// bounds); strides_bytes has rank - 1 entries.
+ta_status encode_bf16_tiled(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                            const uint64_t* strides_bytes, const uint32_t* box);
+
 // Records a description of the last host-side failure of this thread
 // (returned by ta_last_error) and returns `code`.
 ta_status fail(ta_status code, const char* where, cudaError_t err = cudaSuccess);
@@ -62,6 +67,12 @@ ta_status launch_gather_debug(const void* k_cache, const void* v_cache, const in
                               int max_pages, int num_pages_total, void* k_out, void* v_out, cudaStream_t stream);
 
 ta_status launch_selftest_wait(unsigned limit_us, cudaStream_t stream);
+
+ta_status launch_paged_prefill(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+                               const int32_t* cu_seqlens, const int32_t* seq_lens, int page_size, int num_seqs,
+                               int total_q, int max_q_len, int Hq, int Hkv, int d, int max_pages,
+                               int num_pages_total, float scale, int causal, void* o, float* lse,
+                               cudaStream_t stream);
 
 size_t bwd_workspace_bytes(int B, int Hq, int Nq);
 ta_status launch_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,

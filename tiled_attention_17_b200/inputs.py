@@ -267,3 +267,45 @@ def gather_pages_for(inp: PagedInputs, seqs) -> dict:
                 v = pool_pages(inp.cfg, inp.seed, 2, slot, 1)[0]
                 out[slot] = (k, v)
     return out
+
+
+# --------------------------------------------------------------------------
+# Varlen prefill over the paged cache
+# --------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class PagedPrefillInputs:
+    q: np.ndarray            # [total_q, Hq, d] bf16 bits, packed by cu_seqlens
+    cu_seqlens: np.ndarray   # [S + 1] int32
+    seq_lens: np.ndarray     # [S] int32 keys per sequence (prefix + new tokens)
+    block_table: np.ndarray  # [S, max_pages] int32, -1 beyond each sequence
+    k_cache: np.ndarray      # [P, Hkv, page, d] bf16 bits
+    v_cache: np.ndarray
+    max_q_len: int
+
+
+def paged_prefill_inputs(q_lens, kv_lens, Hq: int, Hkv: int, d: int, page_size: int, seed: int,
+                         extra_pages: int = 2) -> PagedPrefillInputs:
+    """Seeded varlen batch: sequence s has q_lens[s] new queries and kv_lens[s]
+    keys in total; its pages sit at a seeded permutation of the pool's slots."""
+    q_lens = np.asarray(q_lens, dtype=np.int32)
+    kv_lens = np.asarray(kv_lens, dtype=np.int32)
+    S = q_lens.size
+    cu = np.zeros(S + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(q_lens)
+    npages = (kv_lens.astype(np.int64) + page_size - 1) // page_size
+    total = int(npages.sum()) + extra_pages
+    max_pages = max(int(npages.max()) if S else 1, 1)
+    perm = np.random.Generator(np.random.PCG64([seed, 1])).permutation(total).astype(np.int32)
+    table = np.full((S, max_pages), -1, dtype=np.int32)
+    off = 0
+    for s in range(S):
+        n = int(npages[s])
+        table[s, :n] = perm[off:off + n]
+        off += n
+    T = int(cu[-1])
+    q = _normal_bf16([seed, 2], max(T, 1) * Hq * d)[:T * Hq * d].reshape(T, Hq, d)
+    per = total * Hkv * page_size * d
+    k = _normal_bf16_chunked([seed, 3], per).reshape(total, Hkv, page_size, d)
+    v = _normal_bf16_chunked([seed, 4], per).reshape(total, Hkv, page_size, d)
+    return PagedPrefillInputs(q, cu, kv_lens, table, k, v, int(q_lens.max()) if S else 0)
