@@ -7,8 +7,10 @@ One step = one pass of the whole hot path over one batch of synthetic input:
     16-token pages, lengths uniform on [512, 32768] (attn_paged_decode + combine).
 The headline metric is the prefill's TFLOP/s (visible (q, k) pairs, both
 contractions, 2 flop per multiply-add); the decode's KV GB/s is reported in
-the same line under "decode", and the backward pass (attn_bwd on the prefill
-workload, timed on its own after the step) under "backward".  Inputs are
+the same line under "decode"; the backward pass (attn_bwd on the prefill
+workload) and a varlen chunked prefill over the paged cache
+(attn_paged_prefill) are timed on their own after the step and reported under
+"backward" and "paged_prefill".  Inputs are
 resident in HBM when timing starts;
 L2 (126 MB) is flushed by writing a 256 MB buffer before every step, outside
 the kernels' event brackets.  Kernel times are CUDA events on the launching
@@ -334,6 +336,11 @@ def run_ours(args):
     if not args.no_e2e:
         e2e, dec_e2e = run_e2e(args, torch, binding, dev, stream, q_h, k_h, v_h, dinp, dist)
 
+    # ---- varlen prefill over the paged cache (timed on its own, after the step)
+    paged = None
+    if not args.no_paged_prefill:
+        paged = run_paged_prefill(args, torch, binding, dev, stream, flush, dist, rank, world, peaks)
+
     # ---- backward pass on the prefill workload (timed on its own, after the step)
     bwd = None
     if not args.no_backward:
@@ -363,6 +370,7 @@ def run_ours(args):
                                                              float(dinp.seq_lens.sum()))),
                        "e2e": dec_e2e},
             "backward": bwd,
+            "paged_prefill": paged,
             "roofline": roofline("tensor", pre_per_gpu, peaks["bf16_tflops"], "TFLOP/s",
                                  recorded_traffic("prefill_fwd_kernel", "prefill_sm100.cu", float(c.B * c.Hq))),
             "peaks": {"source": peak_kind, "bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"],
@@ -377,6 +385,63 @@ def run_ours(args):
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+PAGED_MIX = dict(num_seqs=32, q_lo=1, q_hi=2048, prefix_lo=0, prefix_hi=8192, Hq=32, Hkv=8, d=128, page_size=16)
+
+
+def run_paged_prefill(args, torch, binding, dev, stream, flush, dist, rank, world, peaks):
+    """attn_paged_prefill on a serving-like chunked-prefill batch: 32 sequences,
+    1-2048 new tokens each after a 0-8192-token prefix already in the pool
+    (Hq=32, Hkv=8, d=128, 16-token pages at a seeded permutation), causal.
+    CUDA events around each call, L2 flushed before every call."""
+    m = PAGED_MIX
+    rng = np.random.Generator(np.random.PCG64(rank_seed(4321, rank)))
+    q_lens = rng.integers(m["q_lo"], m["q_hi"], size=m["num_seqs"], endpoint=True)
+    kv_lens = q_lens + rng.integers(m["prefix_lo"], m["prefix_hi"], size=m["num_seqs"], endpoint=True)
+    inp = inputs.paged_prefill_inputs(q_lens, kv_lens, m["Hq"], m["Hkv"], m["d"], m["page_size"],
+                                      seed=rank_seed(4322, rank))
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    def i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+
+    q, kc, vc = bf(inp.q), bf(inp.k_cache), bf(inp.v_cache)
+    bt, cu, sl = i32(inp.block_table), i32(inp.cu_seqlens), i32(inp.seq_lens)
+    o = torch.empty_like(q)
+    lse = torch.empty((q.shape[0], m["Hq"]), dtype=torch.float32, device=dev)
+
+    def call():
+        binding.attn_paged_prefill(q, kc, vc, bt, cu, sl, m["page_size"], m["num_seqs"], q.shape[0], inp.max_q_len,
+                                   m["Hq"], m["Hkv"], m["d"], bt.shape[1], kc.shape[0], m["d"] ** -0.5, 1, o, lse,
+                                   stream)
+
+    for _ in range(3):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(dist, dev.index)
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+    (t,) = max_over_ranks([t], dist, device=dev)
+    flops = accounting.varlen_prefill_flops(q_lens, kv_lens, m["Hq"], m["d"], True)
+    per_gpu = flops / (t * 1e-3) / 1e12
+    return {"value": per_gpu * world, "unit": "TFLOP/s", "ms": t, "steps": steps,
+            "workload": (f"{m['num_seqs']} seqs, new tokens U[{m['q_lo']},{m['q_hi']}] after prefix "
+                         f"U[{m['prefix_lo']},{m['prefix_hi']}], Hq={m['Hq']} Hkv={m['Hkv']} d={m['d']}, "
+                         f"{m['page_size']}-token pages, causal; total_q {int(q_lens.sum())}, "
+                         f"keys {int(kv_lens.sum())}"),
+            "flops_per_call_per_gpu": flops, "gpu_launches_per_call": 1,
+            "roofline": roofline("tensor", per_gpu, peaks["bf16_tflops"], "TFLOP/s", None)}
 
 
 def run_backward(args, torch, binding, dev, stream, q, k, v, o, lse, flush, dist, rank, world, peaks):
@@ -564,6 +629,7 @@ def main(argv=None):
     ap.add_argument("--cpu-stride", type=int, default=1, help="oracle baseline: every n-th query row")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-paged-prefill", action="store_true")
     ap.add_argument("--ncu-case", choices=["prefill", "decode", "backward"], default=None,
                     help="run a small single-kernel case for a profiler capture and exit")
     ap.add_argument("--reps", type=int, default=4)

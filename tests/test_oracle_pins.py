@@ -49,6 +49,12 @@ def test_page_size_examples():
         assert accounting.kv_cache_bytes(32, 32, 128, int(L)) == gib * 2**30
 
 
+def test_varlen_flops_sum_of_sequences():
+    assert accounting.varlen_prefill_flops([3, 0, 4], [5, 2, 4], 2, 8, True) == \
+        4.0 * 2 * 8 * (accounting.visible_pairs(3, 5, True) + 0 + 4 * 5 // 2)
+    assert accounting.varlen_prefill_flops([3, 4], [5, 4], 1, 1, False) == 4.0 * (15 + 16)
+
+
 def test_visible_pairs_closed_form():
     for N in (1, 7, 256, 4096):
         assert accounting.visible_pairs(N, N, True) == N * (N + 1) // 2

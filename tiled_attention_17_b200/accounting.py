@@ -39,6 +39,12 @@ def prefill_flops(B: int, Hq: int, Nq: int, Nkv: int, d: int, causal: bool) -> f
     return 4.0 * B * Hq * d * visible_pairs(Nq, Nkv, causal)
 
 
+def varlen_prefill_flops(q_lens, kv_lens, Hq: int, d: int, causal: bool) -> float:
+    """Both contractions over the visible pairs of every sequence (sequence s
+    has q_lens[s] queries against kv_lens[s] keys, bottom-right aligned)."""
+    return 4.0 * Hq * d * sum(visible_pairs(int(a), int(b), causal) for a, b in zip(q_lens, kv_lens))
+
+
 def prefill_min_bytes(B: int, Hq: int, Hkv: int, Nq: int, Nkv: int, d: int, lse: bool = True) -> int:
     """Q, K, V read once, O (and lse) written once, bf16 tensors."""
     b = 2 * (B * Hq * Nq * d) * 2 + 2 * (B * Hkv * Nkv * d) * 2

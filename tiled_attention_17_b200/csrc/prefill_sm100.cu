@@ -212,25 +212,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * 64, q0, zq);
         }
       }
+      // Physical pages of K/V tile j (paged): the table entries are read
+      // together, once per tile, for both the K and the V copies.  Pages past
+      // the sequence, and entries outside the pool (flagged), read page 0: the
+      // pool's contents are finite and those keys are masked.
+      constexpr int kMaxPagesPerTile = kBN / 8;
+      int phys[kMaxPagesPerTile];
+      auto lookup_pages = [&](int j) {
+        if constexpr (kPaged) {
+          const int per_tile = kBN / a.page_size;
+          const int32_t* row = a.block_table + static_cast<size_t>(b) * a.max_pages + j * per_tile;
+#pragma unroll
+          for (int p = 0; p < kMaxPagesPerTile; ++p)
+            phys[p] = (p < per_tile && (j * per_tile + p) * a.page_size < Nkv) ? __ldg(row + p) : 0;
+#pragma unroll
+          for (int p = 0; p < kMaxPagesPerTile; ++p)
+            if (phys[p] < 0 || phys[p] >= a.num_pages_total) {
+              atomicOr(a.status, kDevBadBlockTable);
+              phys[p] = 0;
+            }
+        }
+      };
       // K or V tile j into ring slot `dst`: one tile box (dense), or one box per
-      // page through the block table (paged).  Pages past the sequence, and
-      // entries outside the pool (flagged), read page 0: the pool's contents
-      // are finite and those keys are masked.
+      // page (paged, pages from lookup_pages)
       auto load_kv = [&](const CUtensorMap* tm, uint32_t dst, uint32_t bar, int j) {
         if constexpr (kPaged) {
           const int per_tile = kBN / a.page_size;
-          for (int p = 0; p < per_tile; ++p) {
-            const int logical = j * per_tile + p;
-            int phys = 0;
-            if (logical * a.page_size < Nkv) {
-              phys = a.block_table[static_cast<size_t>(b) * a.max_pages + logical];
-              if (phys < 0 || phys >= a.num_pages_total) {
-                atomicOr(a.status, kDevBadBlockTable);
-                phys = 0;
-              }
-            }
+#pragma unroll
+          for (int p = 0; p < kMaxPagesPerTile; ++p) {
+            if (p >= per_tile) break;
             for (int c = 0; c < L::kChunks; ++c)
-              tma_load_4d(dst + c * L::kChunkBytes + p * a.page_size * 128, tm, bar, c * 64, 0, hkv, phys);
+              tma_load_4d(dst + c * L::kChunkBytes + p * a.page_size * 128, tm, bar, c * 64, 0, hkv, phys[p]);
           }
         } else {
           for (int c = 0; c < L::kChunks; ++c) tma_load_3d(dst + c * L::kChunkBytes, tm, bar, c * 64, j * kBN, zk);
@@ -240,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n_max && ok; ++j) {
         const int s = j % L::kStages;
         const uint32_t ph = (j / L::kStages) & 1u;
+        lookup_pages(j);   // before the wait, so the table reads overlap it
         ok = mbar_wait(BAR_KE(s), ph ^ 1u, a.status, abort_flag);
         if (!ok) break;
         mbar_arrive_expect_tx(BAR_KF(s), L::kTileBytes);
