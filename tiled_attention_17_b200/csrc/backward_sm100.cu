@@ -21,9 +21,13 @@
 // Splitting dQ from dK/dV recomputes S and dP once more (7 tile GEMMs instead
 // of 5) but needs no atomics, so the gradients are deterministic.
 //
-// Warp roles (256 threads): warp 0 TMA producer, warp 1 TMEM allocator and
-// single-thread tcgen05.mma issuer, warps 4-7 one thread per tile row for the
-// elementwise work and the epilogue.  All operand forms are the forward
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator and
+// single-thread tcgen05.mma issuer, warps 4-11 two warpgroups for the
+// elementwise work and the epilogue: thread (h, row) owns one tile row's
+// columns [64h, 64h + 64).  The elementwise steps need no row reduction (the
+// row statistics come precomputed), so the two halves never exchange data;
+// each writes its bf16 result over the TMEM columns it read, and the
+// accumulating products take the two halves as separate A addresses.  All operand forms are the forward
 // kernel's: K-major A and B from shared memory for the score-like products,
 // bf16 probabilities from TMEM as A with an MN-major B for the accumulating
 // ones.
@@ -40,8 +44,14 @@ namespace ta {
 namespace {
 
 constexpr int kT = 128;          // rows per tile (queries or keys)
-constexpr int kBwdThreads = 256;
-constexpr int kWorkWarp0 = 4;    // warps 4-7: one thread per tile row
+constexpr int kBwdThreads = 384;
+constexpr int kWorkWarp0 = 4;    // warps 4-11: thread (h, row) owns columns [64h, 64h + 64) of a tile row
+// Launch at 168 registers per thread (one warp of each of the three
+// warpgroups per sub-partition: 3 x 168 = 504 of 512), then re-split.
+constexpr int kBwdLaunchRegs = 168;
+constexpr int kBwdRegsControl = 120;
+constexpr int kBwdRegsWork = 192;
+static_assert(kBwdRegsControl + 2 * kBwdRegsWork <= 3 * kBwdLaunchRegs, "register split");
 
 template <int D>
 struct BwdTiles {
@@ -78,12 +88,14 @@ __device__ __forceinline__ void mma_kmajor_tile(uint32_t d_tmem, uint64_t a0, ui
   }
 }
 
-// D += A B with A = 128 x 128 bf16 in TMEM (64 columns of packed pairs) and
-// B = an MN-major 128-row x D tile in shared memory (K = its rows).
-__device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc, bool acc) {
+// D += A B with A = 128 x 128 bf16 in TMEM (packed pairs: K = 0..63 in the 32
+// columns at a_lo, K = 64..127 in the 32 columns at a_hi) and B = an MN-major
+// 128-row x D tile in shared memory (K = its rows).
+__device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint64_t b0,
+                                           uint32_t idesc, bool acc) {
 #pragma unroll
   for (int kk = 0; kk < kT / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc,
+    mma_ts(d_tmem, (kk < 4 ? a_lo : a_hi - 32) + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc,
            (acc || kk > 0) ? 1u : 0u);
 }
 
@@ -203,9 +215,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(BAR_QE(s), 1);
     }
     mbar_init(BAR_SF, 1);
-    mbar_init(BAR_PF, 128);
+    mbar_init(BAR_PF, 256);
     mbar_init(BAR_DPF, 1);
-    mbar_init(BAR_DSF, 128);
+    mbar_init(BAR_DSF, 256);
     mbar_init(BAR_ACC, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -224,7 +236,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp < kWorkWarp0) {
+  setmaxnreg_dec<kBwdRegsControl>();
   if (n_items > 0 && warp == 0 && lane == 0) {
     // ======================= TMA producer =======================
     const int zk = b * a.Hkv + hkv;
@@ -271,7 +284,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // dV += P^T dO once P^T is in TMEM
       if (!(ok = mbar_wait(BAR_PF, ph, a.status, abort_flag))) break;
       tc_fence_after();
-      mma_tmem_a(tmem + L::kTmDV, tmem + L::kTmS, dDOm + s * kStep, idesc_acc, it > 0);
+      mma_tmem_a(tmem + L::kTmDV, tmem + L::kTmS, tmem + L::kTmS + 64, dDOm + s * kStep, idesc_acc, it > 0);
       // next item's S^T: the S buffer is free once the dV product above has read P^T
       if (it + 1 < n_items) {
         if (!(ok = mbar_wait(BAR_QF(s1), ((it + 1) >> 1) & 1u, a.status, abort_flag))) break;
@@ -282,7 +295,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // dK += dS^T Q once dS^T is in TMEM
       if (!(ok = mbar_wait(BAR_DSF, ph, a.status, abort_flag))) break;
       tc_fence_after();
-      mma_tmem_a(tmem + L::kTmDK, tmem + L::kTmDP, dQm + s * kStep, idesc_acc, it > 0);
+      mma_tmem_a(tmem + L::kTmDK, tmem + L::kTmDP, tmem + L::kTmDP + 64, dQm + s * kStep, idesc_acc, it > 0);
       mma_commit(BAR_QE(s));   // this stage's Q, dO, lse and delta are read once these land
       if (it + 1 < n_items) {
         mma_kmajor_tile(tmem + L::kTmDP, dV, dDOk + s1 * kStep, T::kChunks, idesc_s, false);
@@ -290,8 +303,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     if (ok) mma_commit(BAR_ACC);
-  } else if (warp >= kWorkWarp0) {
+  }
+  } else {
+    setmaxnreg_inc<kBwdRegsWork>();
     // ======================= per-key-row work + epilogue =======================
+    const int h = (warp - kWorkWarp0) / 4;         // query columns [64h, 64h + 64) of each tile
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;             // key row within the tile
     const int key = kt * kT + r;
@@ -305,7 +321,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int qt = i0 + it % per_head;
       const int q0 = qt * kT;
       // query columns c with key > q0 + c + off are masked: c < lim
-      const int lim = (a.causal ? key - off - q0 : 0);
+      const int lim = (a.causal ? key - off - q0 : 0) - h * 64;
       const bool row_ok = key < a.Nkv;
       const bool need_mask = !row_ok || lim > 0;
       ok = mbar_wait(BAR_QF(s), (it >> 1) & 1u, a.status, abort_flag);
@@ -313,40 +329,41 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float* l2v = vec + (s * 2 + 0) * kT;
-      const float* dlv = vec + (s * 2 + 1) * kT;
-      // P^T = exp2(S^T c2 - lse2[query]) for this key row, in two 64-column halves
-      uint32_t pk[2][32];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      const float* l2v = vec + (s * 2 + 0) * kT + h * 64;
+      const float* dlv = vec + (s * 2 + 1) * kT + h * 64;
+      // P^T = exp2(S^T c2 - lse2[query]) over this half's 64 query columns,
+      // written as bf16 over the first 32 of the columns it was read from
+      uint32_t pk[32];
+      {
         uint32_t sr[2][32];
         tmem_ld32(tmem + L::kTmS + lane_off + h * 64, sr[0]);
         tmem_ld32(tmem + L::kTmS + lane_off + h * 64 + 32, sr[1]);
         tmem_wait_ld();
         const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = h * 64 + 2 * e;
-          const float4 l4 = *reinterpret_cast<const float4*>(l2v + (c & ~3));
-          const float la = (c & 2) ? l4.z : l4.x, lb = (c & 2) ? l4.w : l4.y;
-          float p0 = ex2(fmaf(sv[2 * e], c2, -la));
-          float p1 = ex2(fmaf(sv[2 * e + 1], c2, -lb));
+        for (int e4 = 0; e4 < 16; ++e4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(l2v + 4 * e4);
+          const int c = 4 * e4;
+          float p0 = ex2(fmaf(sv[c + 0], c2, -l4.x)), p1 = ex2(fmaf(sv[c + 1], c2, -l4.y));
+          float p2 = ex2(fmaf(sv[c + 2], c2, -l4.z)), p3 = ex2(fmaf(sv[c + 3], c2, -l4.w));
           if (need_mask) {
-            p0 = (row_ok && c >= lim) ? p0 : 0.f;
+            p0 = (row_ok && c + 0 >= lim) ? p0 : 0.f;
             p1 = (row_ok && c + 1 >= lim) ? p1 : 0.f;
+            p2 = (row_ok && c + 2 >= lim) ? p2 : 0.f;
+            p3 = (row_ok && c + 3 >= lim) ? p3 : 0.f;
           }
-          pk[h][e] = pack_bf16x2(p0, p1);
+          pk[2 * e4] = pack_bf16x2(p0, p1);
+          pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
         }
-        tmem_st32(tmem + L::kTmS + lane_off + h * 32, pk[h]);
+        tmem_st32(tmem + L::kTmS + lane_off + h * 64, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR_PF);
-      // dS^T = P^T o (dP^T - delta[query])
+      // dS^T = P^T o (dP^T - delta[query]) over this half, written over dP^T
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_DPF, ph, a.status, abort_flag)))) break;
       tc_fence_after();
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      {
         uint32_t dr[2][32];
         tmem_ld32(tmem + L::kTmDP + lane_off + h * 64, dr[0]);
         tmem_ld32(tmem + L::kTmDP + lane_off + h * 64 + 32, dr[1]);
@@ -354,13 +371,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float* dpv = reinterpret_cast<const float*>(&dr[0][0]);
         uint32_t dk[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = h * 64 + 2 * e;
-          const float4 d4 = *reinterpret_cast<const float4*>(dlv + (c & ~3));
-          const float da = (c & 2) ? d4.z : d4.x, db = (c & 2) ? d4.w : d4.y;
-          dk[e] = pack_bf16x2(bf16lo(pk[h][e]) * (dpv[2 * e] - da), bf16hi(pk[h][e]) * (dpv[2 * e + 1] - db));
+        for (int e2 = 0; e2 < 16; ++e2) {
+          const float4 d4 = *reinterpret_cast<const float4*>(dlv + 4 * e2);
+          const uint32_t w0 = pk[2 * e2], w1 = pk[2 * e2 + 1];
+          dk[2 * e2] = pack_bf16x2(bf16lo(w0) * (dpv[4 * e2 + 0] - d4.x), bf16hi(w0) * (dpv[4 * e2 + 1] - d4.y));
+          dk[2 * e2 + 1] = pack_bf16x2(bf16lo(w1) * (dpv[4 * e2 + 2] - d4.z), bf16hi(w1) * (dpv[4 * e2 + 3] - d4.w));
         }
-        tmem_st32(tmem + L::kTmDP + lane_off + h * 32, dk);
+        tmem_st32(tmem + L::kTmDP + lane_off + h * 64, dk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -377,11 +394,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const size_t orow = (static_cast<size_t>(b) * a.Hkv + hkv) * a.Nkv + (store ? key : 0);
 #pragma unroll 1
     for (int which = 0; which < 2; ++which) {
-      __nv_bfloat16* dst_row = (which ? a.dv : a.dk) + orow * D;
+      // this warpgroup's half of the row: columns [h D/2, (h+1) D/2)
+      __nv_bfloat16* dst_row = (which ? a.dv : a.dk) + orow * D + h * (D / 2);
       const float mul = which ? 1.f : a.scale;
-      const uint32_t src = tmem + (which ? L::kTmDV : L::kTmDK) + lane_off;
+      const uint32_t src = tmem + (which ? L::kTmDV : L::kTmDK) + lane_off + h * (D / 2);
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t v[32];
         if (have && ok) {
           tmem_ld32(src + c * 32, v);
@@ -487,9 +505,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(BAR_VE(s), 1);
     }
     mbar_init(BAR_SF, 1);
-    mbar_init(BAR_LOADED, 128);
+    mbar_init(BAR_LOADED, 256);
     mbar_init(BAR_DPF, 1);
-    mbar_init(BAR_DSF, 128);
+    mbar_init(BAR_DSF, 256);
     mbar_init(BAR_DSE, 1);
     mbar_init(BAR_ACC, 1);
     *abort_flag = 0;
@@ -509,7 +527,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp < kWorkWarp0) {
+  setmaxnreg_dec<kBwdRegsControl>();
   if (n > 0 && warp == 0 && lane == 0) {
     // ======================= TMA producer =======================
     const int zq = b * a.Hq + hq, zk = b * a.Hkv + hkv;
@@ -568,13 +587,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // dQ += dS K_j once dS is in its buffer
       if (!(ok = mbar_wait(BAR_DSF, ph, a.status, abort_flag))) break;
       tc_fence_after();
-      mma_tmem_a(tmem + L::kTmDQ, tmem + L::kTmDS, dKm + s * kStep, idesc_acc, j > 0);
+      mma_tmem_a(tmem + L::kTmDQ, tmem + L::kTmDS, tmem + L::kTmDS + 32, dKm + s * kStep, idesc_acc, j > 0);
       mma_commit(BAR_DSE);
       if (j + 2 < n) mma_commit(BAR_KE(s));
     }
     if (ok) mma_commit(BAR_ACC);
-  } else if (warp >= kWorkWarp0) {
+  }
+  } else {
+    setmaxnreg_inc<kBwdRegsWork>();
     // ======================= per-query-row work + epilogue =======================
+    const int h = (warp - kWorkWarp0) / 4;         // key columns [64h, 64h + 64) of each tile
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int qrow = q0 + r;
@@ -591,27 +613,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int lim = vis_end - j * kT;   // visible key columns: [0, lim)
+      const int lim = vis_end - j * kT - h * 64;   // visible key columns of this half: [0, lim)
       const bool need_mask = (j * kT + kT > a.Nkv) || (a.causal && j * kT + kT - 1 > q0 + (a.Nkv - a.Nq));
-      uint32_t pk[2][32];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      uint32_t pk[32];
+      {
         uint32_t sr[2][32], dr[2][32];
         tmem_ld32(tmem + L::kTmS + lane_off + h * 64, sr[0]);
         tmem_ld32(tmem + L::kTmS + lane_off + h * 64 + 32, sr[1]);
         tmem_ld32(tmem + L::kTmDP + lane_off + h * 64, dr[0]);
         tmem_ld32(tmem + L::kTmDP + lane_off + h * 64 + 32, dr[1]);
         tmem_wait_ld();
-        if (h == 1) {
-          // S and dP are in registers: the next tile's products may overwrite them
-          tc_fence_before();
-          mbar_arrive(BAR_LOADED);
-        }
+        // this half of S and dP is in registers: the next tile's products may
+        // overwrite both buffers once the other half has read its part too
+        tc_fence_before();
+        mbar_arrive(BAR_LOADED);
         const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
         const float* dpv = reinterpret_cast<const float*>(&dr[0][0]);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int c = h * 64 + 2 * e;
+          const int c = 2 * e;
           float p0 = ex2(fmaf(sv[2 * e], c2, -l2));
           float p1 = ex2(fmaf(sv[2 * e + 1], c2, -l2));
           if (need_mask) {
@@ -620,7 +640,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           // dS rounds P to bf16 first, as the dK/dV kernel does
           const uint32_t pb = pack_bf16x2(p0, p1);
-          pk[h][e] = pack_bf16x2(bf16lo(pb) * (dpv[2 * e] - dl), bf16hi(pb) * (dpv[2 * e + 1] - dl));
+          pk[e] = pack_bf16x2(bf16lo(pb) * (dpv[2 * e] - dl), bf16hi(pb) * (dpv[2 * e + 1] - dl));
         }
       }
       // the previous dQ product must have read the dS buffer
@@ -628,8 +648,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_DSE, (j - 1) & 1u, a.status, abort_flag)))) break;
         tc_fence_after();
       }
-      tmem_st32(tmem + L::kTmDS + lane_off, pk[0]);
-      tmem_st32(tmem + L::kTmDS + lane_off + 32, pk[1]);
+      tmem_st32(tmem + L::kTmDS + lane_off + h * 32, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR_DSF);
@@ -642,12 +661,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     // TMEM loads are warp-collective: every lane loads, only rows < Nq store
     const bool store = qrow < a.Nq;
-    __nv_bfloat16* dst_row = a.dq + (static_cast<size_t>(bh) * a.Nq + (store ? qrow : 0)) * D;
+    // this warpgroup's half of the row: columns [h D/2, (h+1) D/2)
+    __nv_bfloat16* dst_row = a.dq + (static_cast<size_t>(bh) * a.Nq + (store ? qrow : 0)) * D + h * (D / 2);
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < D / 64; ++c) {
       uint32_t v[32];
       if (have && ok) {
-        tmem_ld32(tmem + L::kTmDQ + lane_off + c * 32, v);
+        tmem_ld32(tmem + L::kTmDQ + lane_off + h * (D / 2) + c * 32, v);
         tmem_wait_ld();
       } else {
 #pragma unroll
