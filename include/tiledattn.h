@@ -124,6 +124,33 @@ ta_status attn_paged_prefill(const void *q, const void *k_cache, const void *v_c
                              float *lse, ta_stream_t stream);
 
 /*
+ * attn_lse_merge - merge one partial attention result into an accumulator.
+ * A partial is the attention of a set of rows over one block of keys: its
+ * output normalised over that block and the block's lse.  Blocks combine
+ * exactly by their lse (FlashAttention optimisation article, section 3.2.2:
+ * the result does not depend on how keys are blocked), which is how the ring
+ * schedule of the LLM-inference article (section 4.1) assembles each device's
+ * output from one block per hop.
+ *
+ *   acc_o     [rows, d] fp32, 16-byte aligned (read unless first, written)
+ *   acc_lse   [rows] fp32 (read unless first, written)
+ *   part_o    [rows, d] bf16, 8-byte aligned (e.g. attn_fwd's o)
+ *   part_lse  [rows] fp32 (attn_fwd's lse; -inf = no visible key)
+ *   first     1: acc = part; 0: acc = merge(acc, part):
+ *             lse = log(e^lse_acc + e^lse_part),
+ *             o = e^(lse_acc - lse) o_acc + e^(lse_part - lse) o_part
+ * Rows where both sides are -inf stay O = 0, lse = -inf.  d in {64, 128}.
+ */
+ta_status attn_lse_merge(float *acc_o, float *acc_lse, const void *part_o, const float *part_lse,
+                         int64_t rows, int d, int first, ta_stream_t stream);
+
+/*
+ * attn_lse_merge_finish - the accumulator's output as bf16: out [rows, d]
+ * (8-byte aligned) = round(acc_o).
+ */
+ta_status attn_lse_merge_finish(const float *acc_o, void *out, int64_t rows, int d, ta_stream_t stream);
+
+/*
  * Bytes of device workspace attn_bwd needs (256-byte multiple): two fp32
  * values per query row, rows padded to a multiple of 128 per head.  Pure
  * host arithmetic; returns 0 for invalid sizes.

@@ -62,6 +62,8 @@ def test_binding_argtypes_match_header(lib):
                 assert t is ctypes.c_float, (name, p, t)
             elif p.startswith("size_t"):
                 assert t is ctypes.c_size_t, (name, p, t)
+            elif p.startswith("int64_t"):
+                assert t is ctypes.c_int64, (name, p, t)
             else:
                 assert t in (ctypes.c_int, ctypes.c_uint), (name, p, t)
 

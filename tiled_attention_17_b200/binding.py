@@ -25,7 +25,7 @@ TA_DEV_BAD_BLOCK_TABLE = 2
 TA_DEV_BAD_SEQ_LEN = 4
 
 EXPORTS = ["ta_status_string", "ta_version", "ta_last_error", "attn_fwd", "attn_bwd_workspace_size", "attn_bwd",
-           "attn_paged_prefill",
+           "attn_paged_prefill", "attn_lse_merge", "attn_lse_merge_finish",
            "attn_paged_decode_workspace_size",
            "attn_paged_decode", "attn_paged_decode_noalloc", "attn_paged_decode_check", "attn_paged_gather_debug",
            "ta_device_status", "ta_selftest_bounded_wait"]
@@ -60,6 +60,11 @@ def load(path: str | None = None):
     L.attn_fwd.restype = i32
     L.attn_paged_prefill.argtypes = [vp] * 6 + [i32] * 9 + [f32, i32, vp, vp, vp]
     L.attn_paged_prefill.restype = i32
+    i64 = ctypes.c_int64
+    L.attn_lse_merge.argtypes = [vp, vp, vp, vp, i64, i32, i32, vp]
+    L.attn_lse_merge.restype = i32
+    L.attn_lse_merge_finish.argtypes = [vp, vp, i64, i32, vp]
+    L.attn_lse_merge_finish.restype = i32
     L.attn_bwd_workspace_size.argtypes = [i32] * 3
     L.attn_bwd_workspace_size.restype = sz
     L.attn_bwd.argtypes = [vp] * 10 + [sz] + [i32] * 6 + [f32, i32, vp]
@@ -138,6 +143,21 @@ def attn_paged_prefill(q, k_cache, v_cache, block_table, cu_seqlens, seq_lens, p
                                      _stream(stream))
     if check:
         _check("attn_paged_prefill", code)
+    return code
+
+
+def attn_lse_merge(acc_o, acc_lse, part_o, part_lse, rows, d, first, stream=None, check=True) -> int:
+    code = load().attn_lse_merge(_ptr(acc_o), _ptr(acc_lse), _ptr(part_o), _ptr(part_lse), int(rows), d, int(first),
+                                 _stream(stream))
+    if check:
+        _check("attn_lse_merge", code)
+    return code
+
+
+def attn_lse_merge_finish(acc_o, out, rows, d, stream=None, check=True) -> int:
+    code = load().attn_lse_merge_finish(_ptr(acc_o), _ptr(out), int(rows), d, _stream(stream))
+    if check:
+        _check("attn_lse_merge_finish", code)
     return code
 
 

@@ -159,6 +159,28 @@ ta_status attn_paged_prefill(const void* q, const void* k_cache, const void* v_c
                               reinterpret_cast<cudaStream_t>(stream));
 }
 
+ta_status attn_lse_merge(float* acc_o, float* acc_lse, const void* part_o, const float* part_lse, int64_t rows, int d,
+                         int first, ta_stream_t stream) {
+  if (rows < 0 || d <= 0 || (first != 0 && first != 1)) return TA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return TA_ERR_UNSUPPORTED;
+  if (rows > (int64_t(1) << 33)) return TA_ERR_UNSUPPORTED;   // grid of rows / 8 blocks
+  if (rows == 0) return TA_OK;
+  if (!acc_o || !acc_lse || !part_o || !part_lse) return TA_ERR_INVALID_ARG;
+  if (!aligned16(acc_o) || (reinterpret_cast<uintptr_t>(part_o) & 7u) || (reinterpret_cast<uintptr_t>(acc_lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(part_lse) & 3u))
+    return TA_ERR_INVALID_ARG;
+  return launch_lse_merge(acc_o, acc_lse, part_o, part_lse, rows, d, first, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ta_status attn_lse_merge_finish(const float* acc_o, void* out, int64_t rows, int d, ta_stream_t stream) {
+  if (rows < 0 || d <= 0) return TA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return TA_ERR_UNSUPPORTED;
+  if (rows > (int64_t(1) << 33)) return TA_ERR_UNSUPPORTED;   // grid of rows / 8 blocks
+  if (rows == 0) return TA_OK;
+  if (!acc_o || !out || !aligned16(acc_o) || (reinterpret_cast<uintptr_t>(out) & 7u)) return TA_ERR_INVALID_ARG;
+  return launch_lse_merge_finish(acc_o, out, rows, d, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t attn_bwd_workspace_size(int B, int Hq, int Nq) {
   if (B < 0 || Hq <= 0 || Nq < 0) return 0;
   if (static_cast<long long>(B) * Hq > INT32_MAX / 2 || Nq > (1 << 30)) return 0;

@@ -74,6 +74,10 @@ ta_status launch_paged_prefill(const void* q, const void* k_cache, const void* v
                                int num_pages_total, float scale, int causal, void* o, float* lse,
                                cudaStream_t stream);
 
+ta_status launch_lse_merge(float* acc_o, float* acc_lse, const void* part_o, const float* part_lse, int64_t rows,
+                           int d, int first, cudaStream_t stream);
+ta_status launch_lse_merge_finish(const float* acc_o, void* out, int64_t rows, int d, cudaStream_t stream);
+
 size_t bwd_workspace_bytes(int B, int Hq, int Nq);
 ta_status launch_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                           const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int Hq, int Hkv,
