@@ -189,11 +189,13 @@ def test_bounded_wait_selftest(torch_cuda):
     assert binding.ta_device_status(reset=True) == (0, 0)
 
 
-def test_decode_full_size_sampled(torch_cuda):
+@pytest.mark.parametrize("seed_offset", [0, 1, 2])
+def test_decode_full_size_sampled(torch_cuda, seed_offset):
     """The full decode workload (64 sequences, lengths 512..32768) in the
-    benchmark's launch configuration; sampled sequences vs the oracle."""
+    benchmark's launch configuration, three seeds (the config's own and two
+    more); sampled sequences vs the oracle."""
     torch = torch_cuda
-    inp = inputs.paged_inputs(inputs.DECODE_CONFIG)
+    inp = inputs.paged_inputs(inputs.DECODE_CONFIG, seed=inputs.CONFIG_SEEDS["decode"] + 1000 * seed_offset)
     o, lse, ws = run_decode(torch, inp)
     lens = inp.seq_lens
     pick = sorted({int(np.argmin(lens)), int(np.argmax(lens)), 0, 31, 63, 17})

@@ -140,11 +140,13 @@ def test_prefill_bad_args_do_not_launch(torch_cuda):
     assert binding.STATUS_NAMES[code] == "TA_ERR_UNSUPPORTED"
 
 
+@pytest.mark.parametrize("seed_offset", [0, 1, 2])
 @pytest.mark.parametrize("name", ["causal", "long", "gqa"])
-def test_prefill_full_size_sampled(torch_cuda, name):
-    """Full-size workloads in the benchmark's launch configuration; sampled rows vs the oracle."""
+def test_prefill_full_size_sampled(torch_cuda, name, seed_offset):
+    """Full-size workloads in the benchmark's launch configuration, three seeds
+    each (the config's own and two more); sampled rows vs the oracle."""
     cfg = inputs.PREFILL_CONFIGS[name]
-    q, k, v = inputs.prefill_inputs(cfg)
+    q, k, v = inputs.prefill_inputs(cfg, seed=inputs.CONFIG_SEEDS[name] + 1000 * seed_offset)
     o, lse = run_fwd(torch_cuda, q, k, v, cfg.causal, cfg.scale)
     rng = np.random.Generator(np.random.PCG64(77))
     rows = sample_rows(cfg.B, cfg.Hq, cfg.Nq, 384, rng)

@@ -7,7 +7,11 @@
 // optimisation article, sections 3.1-3.2 and 7.1).
 //
 // CTA = two 128-row query tiles of one (batch, query head) sharing one K/V
-// stream.  Warp roles (384 threads, three warpgroups):
+// stream.  The kernel has two instantiations: dense [B, H, N, d] tensors, and
+// (kPaged) varlen query rows of several sequences packed as [total_q, Hq, d]
+// against K/V gathered page by page from a paged cache through a block table
+// (chunked prefill, LLM-inference article section 3.2; PagedAttention,
+// GPU-optimisation tag page).  Warp roles (384 threads, three warpgroups):
 //   warp 0      TMA producer: Q tiles once, then K_j / V_j into a smem ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2-3   idle after setup
@@ -53,10 +57,9 @@ static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
 static_assert(kRegsControl + 2 * kRegsSoftmax <= 512, "per sub-partition: one warp of each warpgroup");
 constexpr float kRescaleLog2 = 8.0f;   // skip O rescale while max grew by <= 2^8
 // Column pairs whose index i has bit (i % 8) set in kPolyMask compute 2^x on
-// the FMA pipe instead of the MUFU unit (3 of every 8 pairs): the two softmax
-// warpgroups of an SM would otherwise need as many MUFU cycles as the tensor
-// pipe needs for the four MMAs of a K/V tile.
-constexpr unsigned kPolyMask = 0x00u;   // measured fastest on B200: all on MUFU
+// the FMA pipe (exp2_poly2) instead of the MUFU unit.  Moving 1/8 to 4/8 of
+// them there was measured: none was faster on B200, so all stay on MUFU.
+constexpr unsigned kPolyMask = 0x00u;
 
 template <int D>
 struct PrefillLayout {
