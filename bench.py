@@ -586,7 +586,18 @@ def run_ncu_case(args):
     def dev_bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    if args.ncu_case == "backward":
+    if args.ncu_case == "paged":
+        m = PAGED_MIX
+        rng = np.random.Generator(np.random.PCG64(4321))
+        q_lens = rng.integers(m["q_lo"], m["q_hi"], size=m["num_seqs"], endpoint=True)
+        kv_lens = q_lens + rng.integers(m["prefix_lo"], m["prefix_hi"], size=m["num_seqs"], endpoint=True)
+        inp = inputs.paged_prefill_inputs(q_lens, kv_lens, m["Hq"], m["Hkv"], m["d"], m["page_size"], seed=4322)
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+        q, kc, vc = dev_bf16(inp.q), dev_bf16(inp.k_cache), dev_bf16(inp.v_cache)
+        bt, cu, sl = i32(inp.block_table), i32(inp.cu_seqlens), i32(inp.seq_lens)
+        for _ in range(args.reps):
+            binding.paged_prefill(q, kc, vc, bt, cu, sl, inp.max_q_len, True)
+    elif args.ncu_case == "backward":
         c = PREFILL
         q_h, k_h, v_h = inputs.prefill_inputs(c)
         q, k, v = dev_bf16(q_h), dev_bf16(k_h), dev_bf16(v_h)
@@ -630,7 +641,7 @@ def main(argv=None):
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-paged-prefill", action="store_true")
-    ap.add_argument("--ncu-case", choices=["prefill", "decode", "backward"], default=None,
+    ap.add_argument("--ncu-case", choices=["prefill", "decode", "backward", "paged"], default=None,
                     help="run a small single-kernel case for a profiler capture and exit")
     ap.add_argument("--reps", type=int, default=4)
     args = ap.parse_args(argv)
