@@ -441,7 +441,8 @@ def run_paged_prefill(args, torch, binding, dev, stream, flush, dist, rank, worl
                          f"{m['page_size']}-token pages, causal; total_q {int(q_lens.sum())}, "
                          f"keys {int(kv_lens.sum())}"),
             "flops_per_call_per_gpu": flops, "gpu_launches_per_call": 1,
-            "roofline": roofline("tensor", per_gpu, peaks["bf16_tflops"], "TFLOP/s", None)}
+            "roofline": roofline("tensor", per_gpu, peaks["bf16_tflops"], "TFLOP/s",
+                                 recorded_traffic("paged_prefill", "prefill_sm100.cu", 1.0))}
 
 
 def run_backward(args, torch, binding, dev, stream, q, k, v, o, lse, flush, dist, rank, world, peaks):
