@@ -39,9 +39,11 @@ inline cudaError_t ensure_smem_limit(Kernel kernel, int bytes, int (&done)[64]) 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  // The flags may be read and set by several host threads: atomic accesses
+  // (setting the attribute twice is harmless).
+  if (dev >= 0 && dev < 64 && __atomic_load_n(&done[dev], __ATOMIC_ACQUIRE)) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
+  if (e == cudaSuccess && dev >= 0 && dev < 64) __atomic_store_n(&done[dev], 1, __ATOMIC_RELEASE);
   return e;
 }
 
