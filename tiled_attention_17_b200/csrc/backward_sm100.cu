@@ -441,12 +441,15 @@ struct DqLayout {
   using T = BwdTiles<D>;
   static constexpr int kQ = 0;
   static constexpr int kDO = kQ + T::kTileBytes;
-  static constexpr int kK = kDO + T::kTileBytes;     // 2 stages
-  static constexpr int kV = kK + 2 * T::kTileBytes;  // 2 stages
-  static constexpr int kBar = kV + 2 * T::kTileBytes;
-  // q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full, loaded, dp_full, ds_full, ds_empty,
+  // K_j is read by S_j and again by dQ_j, so its slot frees late: three K
+  // slots let K_{j+1} load while dQ_{j-1} still runs.  V_j is read by dP_j only.
+  static constexpr int kSK = 3, kSV = 2;
+  static constexpr int kK = kDO + T::kTileBytes;
+  static constexpr int kV = kK + kSK * T::kTileBytes;
+  static constexpr int kBar = kV + kSV * T::kTileBytes;
+  // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, loaded, dp_full, ds_full, ds_empty,
   // acc_done
-  static constexpr int kNumBars = 15;
+  static constexpr int kNumBars = 17;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16 + 1024;
   static_assert(kAlloc <= 232448, "dynamic shared memory per block");
@@ -475,14 +478,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sQ = sb + L::kQ, sDO = sb + L::kDO, sK = sb + L::kK, sV = sb + L::kV;
   const uint32_t bar0 = sb + L::kBar;
   const uint32_t BAR_Q = bar0;
+  constexpr int kSK = L::kSK, kSV = L::kSV;
   auto BAR_KF = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto BAR_KE = [&](int s) { return bar0 + 8u * (3 + s); };
-  auto BAR_VF = [&](int s) { return bar0 + 8u * (5 + s); };
-  auto BAR_VE = [&](int s) { return bar0 + 8u * (7 + s); };
+  auto BAR_KE = [&](int s) { return bar0 + 8u * (1 + kSK + s); };
+  auto BAR_VF = [&](int s) { return bar0 + 8u * (1 + 2 * kSK + s); };
+  auto BAR_VE = [&](int s) { return bar0 + 8u * (1 + 2 * kSK + kSV + s); };
   // loaded: S and dP of the current tile are in registers (both buffers may be
   // overwritten); ds_empty: the dQ product has read the dS buffer
-  const uint32_t BAR_SF = bar0 + 8u * 9, BAR_LOADED = bar0 + 8u * 10, BAR_DPF = bar0 + 8u * 11,
-                 BAR_DSF = bar0 + 8u * 12, BAR_DSE = bar0 + 8u * 13, BAR_ACC = bar0 + 8u * 14;
+  const uint32_t bar1 = bar0 + 8u * (1 + 2 * kSK + 2 * kSV);
+  const uint32_t BAR_SF = bar1, BAR_LOADED = bar1 + 8u, BAR_DPF = bar1 + 16u, BAR_DSF = bar1 + 24u,
+                 BAR_DSE = bar1 + 32u, BAR_ACC = bar1 + 40u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -498,9 +503,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(BAR_Q, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSK; ++s) {
       mbar_init(BAR_KF(s), 1);
       mbar_init(BAR_KE(s), 1);
+    }
+    for (int s = 0; s < kSV; ++s) {
       mbar_init(BAR_VF(s), 1);
       mbar_init(BAR_VE(s), 1);
     }
@@ -538,16 +545,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_load_3d(sDO + c * T::kChunkBytes, &tmDO, BAR_Q, c * 64, q0, zq);
     }
     for (int j = 0; j < n; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = ((j >> 1) & 1u) ^ 1u;
-      if (!mbar_wait(BAR_KE(s), ph, a.status, abort_flag)) break;
-      mbar_arrive_expect_tx(BAR_KF(s), T::kTileBytes);
+      const int sk = j % kSK, sv = j % kSV;
+      if (!mbar_wait(BAR_KE(sk), ((j / kSK) & 1u) ^ 1u, a.status, abort_flag)) break;
+      mbar_arrive_expect_tx(BAR_KF(sk), T::kTileBytes);
       for (int c = 0; c < T::kChunks; ++c)
-        tma_load_3d(sK + s * T::kTileBytes + c * T::kChunkBytes, &tmK, BAR_KF(s), c * 64, j * kT, zk);
-      if (!mbar_wait(BAR_VE(s), ph, a.status, abort_flag)) break;
-      mbar_arrive_expect_tx(BAR_VF(s), T::kTileBytes);
+        tma_load_3d(sK + sk * T::kTileBytes + c * T::kChunkBytes, &tmK, BAR_KF(sk), c * 64, j * kT, zk);
+      if (!mbar_wait(BAR_VE(sv), ((j / kSV) & 1u) ^ 1u, a.status, abort_flag)) break;
+      mbar_arrive_expect_tx(BAR_VF(sv), T::kTileBytes);
       for (int c = 0; c < T::kChunks; ++c)
-        tma_load_3d(sV + s * T::kTileBytes + c * T::kChunkBytes, &tmV, BAR_VF(s), c * 64, j * kT, zk);
+        tma_load_3d(sV + sv * T::kTileBytes + c * T::kChunkBytes, &tmV, BAR_VF(sv), c * 64, j * kT, zk);
     }
   } else if (n > 0 && warp == 1 && lane == 0) {
     // ======================= MMA issuer =======================
@@ -566,30 +572,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit(BAR_SF);
       mma_kmajor_tile(tmem + L::kTmDP, dDO, dVk, T::kChunks, idesc_s, false);   // dP = dO V_0^T
       mma_commit(BAR_DPF);
-      if (n > 2) mma_commit(BAR_VE(0));   // release a stage only when a later load reuses it
+      if (kSV < n) mma_commit(BAR_VE(0));   // release a slot only when a later load reuses it
     }
     for (int j = 0; j < n && ok; ++j) {
-      const int s = j & 1, s1 = s ^ 1;
-      const uint32_t ph = j & 1u, ph1 = ((j + 1) >> 1) & 1u;
+      const int sk = j % kSK, sk1 = (j + 1) % kSK, sv1 = (j + 1) % kSV;
+      const uint32_t ph = j & 1u;
+      const uint32_t phk1 = ((j + 1) / kSK) & 1u, phv1 = ((j + 1) / kSV) & 1u;
       // next S and dP as soon as the work warps hold this tile's in registers
       if (j + 1 < n) {
         if (!(ok = mbar_wait(BAR_LOADED, ph, a.status, abort_flag))) break;
-        if (!(ok = mbar_wait(BAR_KF(s1), ph1, a.status, abort_flag))) break;
+        if (!(ok = mbar_wait(BAR_KF(sk1), phk1, a.status, abort_flag))) break;
         tc_fence_after();
-        mma_kmajor_tile(tmem + L::kTmS, dQ, dKk + s1 * kStep, T::kChunks, idesc_s, false);
+        mma_kmajor_tile(tmem + L::kTmS, dQ, dKk + sk1 * kStep, T::kChunks, idesc_s, false);
         mma_commit(BAR_SF);
-        if (!(ok = mbar_wait(BAR_VF(s1), ph1, a.status, abort_flag))) break;
+        if (!(ok = mbar_wait(BAR_VF(sv1), phv1, a.status, abort_flag))) break;
         tc_fence_after();
-        mma_kmajor_tile(tmem + L::kTmDP, dDO, dVk + s1 * kStep, T::kChunks, idesc_s, false);
+        mma_kmajor_tile(tmem + L::kTmDP, dDO, dVk + sv1 * kStep, T::kChunks, idesc_s, false);
         mma_commit(BAR_DPF);
-        if (j + 3 < n) mma_commit(BAR_VE(s1));
+        if (j + 1 + kSV < n) mma_commit(BAR_VE(sv1));
       }
       // dQ += dS K_j once dS is in its buffer
       if (!(ok = mbar_wait(BAR_DSF, ph, a.status, abort_flag))) break;
       tc_fence_after();
-      mma_tmem_a(tmem + L::kTmDQ, tmem + L::kTmDS, tmem + L::kTmDS + 32, dKm + s * kStep, idesc_acc, j > 0);
+      mma_tmem_a(tmem + L::kTmDQ, tmem + L::kTmDS, tmem + L::kTmDS + 32, dKm + sk * kStep, idesc_acc, j > 0);
       mma_commit(BAR_DSE);
-      if (j + 2 < n) mma_commit(BAR_KE(s));
+      if (j + kSK < n) mma_commit(BAR_KE(sk));
     }
     if (ok) mma_commit(BAR_ACC);
   }
