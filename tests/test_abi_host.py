@@ -142,3 +142,67 @@ def test_gather_debug_validation(lib):
 def test_selftest_validation(lib):
     assert code(lib, lib.ta_selftest_bounded_wait(0, stream=0)) == "TA_ERR_INVALID_ARG"
     assert code(lib, lib.ta_selftest_bounded_wait(2_000_000, stream=0)) == "TA_ERR_INVALID_ARG"
+
+
+def test_bwd_validation(lib):
+    a = 256
+    ws = lib.attn_bwd_workspace_size(4, 16, 4096)
+    assert ws == 2 * 4 * 16 * 4096 * 4 and ws % 256 == 0
+    assert lib.attn_bwd_workspace_size(1, 2, 130) == 2 * 2 * 256 * 4   # rows padded to 128 per head
+    assert lib.attn_bwd_workspace_size(1, 0, 128) == 0
+    f = lambda *x, **kw: code(lib, lib.attn_bwd(*x, check=False, stream=0, **kw))
+
+    def call(**kw):
+        g = dict(q=a, k=a, v=a, o=a, do=a, lse=a, dq=a, dk=a, dv=a, ws=a, wsb=1 << 20,
+                 B=1, Hq=2, Hkv=1, Nq=128, Nkv=128, d=128, scale=0.1, causal=1)
+        g.update(kw)
+        return f(g["q"], g["k"], g["v"], g["o"], g["do"], g["lse"], g["dq"], g["dk"], g["dv"], g["ws"], g["wsb"],
+                 g["B"], g["Hq"], g["Hkv"], g["Nq"], g["Nkv"], g["d"], g["scale"], g["causal"])
+
+    assert call(Hq=3, Hkv=2) == "TA_ERR_INVALID_ARG"
+    assert call(d=96) == "TA_ERR_UNSUPPORTED"
+    assert call(causal=2) == "TA_ERR_INVALID_ARG"
+    assert call(scale=-1.0) == "TA_ERR_UNSUPPORTED"
+    assert call(dq=a + 8) == "TA_ERR_INVALID_ARG"          # 16-byte alignment
+    assert call(lse=None) == "TA_ERR_INVALID_ARG"
+    assert call(wsb=16) == "TA_ERR_INVALID_ARG"            # workspace too small
+    assert call(ws=a + 16) == "TA_ERR_INVALID_ARG"         # workspace not 256-byte aligned
+    assert call(B=0) == "TA_OK"                            # nothing to do, no CUDA call
+
+
+def test_paged_prefill_validation(lib):
+    a = 256
+    f = lambda *x, **kw: code(lib, lib.attn_paged_prefill(*x, check=False, stream=0, **kw))
+
+    def call(**kw):
+        g = dict(q=a, kc=a, vc=a, bt=a, cu=a, sl=a, ps=16, S=2, T=100, mq=64, Hq=4, Hkv=2, d=128, mp=8, P=20,
+                 scale=0.1, causal=1, o=a, lse=None)
+        g.update(kw)
+        return f(g["q"], g["kc"], g["vc"], g["bt"], g["cu"], g["sl"], g["ps"], g["S"], g["T"], g["mq"], g["Hq"],
+                 g["Hkv"], g["d"], g["mp"], g["P"], g["scale"], g["causal"], g["o"], g["lse"])
+
+    assert call(ps=12) == "TA_ERR_UNSUPPORTED"
+    assert call(d=80) == "TA_ERR_UNSUPPORTED"
+    assert call(Hq=6, Hkv=4) == "TA_ERR_INVALID_ARG"
+    assert call(causal=3) == "TA_ERR_INVALID_ARG"
+    assert call(q=a + 4) == "TA_ERR_INVALID_ARG"
+    assert call(cu=None) == "TA_ERR_INVALID_ARG"
+    assert call(lse=a + 2) == "TA_ERR_INVALID_ARG"
+    assert call(P=0) == "TA_ERR_INVALID_ARG"
+    assert call(S=0) == "TA_OK"
+    assert call(T=0) == "TA_OK"
+
+
+def test_merge_validation(lib):
+    a = 256
+    m = lambda *x: code(lib, lib.attn_lse_merge(*x, stream=0, check=False))
+    assert m(a, a, a, a, 16, 80, 0) == "TA_ERR_UNSUPPORTED"
+    assert m(a, a, a, a, 16, 128, 2) == "TA_ERR_INVALID_ARG"
+    assert m(a + 8, a, a, a, 16, 128, 0) == "TA_ERR_INVALID_ARG"    # fp32 accumulator 16-byte aligned
+    assert m(a, a, a + 4, a, 16, 128, 0) == "TA_ERR_INVALID_ARG"    # bf16 partial 8-byte aligned
+    assert m(a, a, a, a, -1, 128, 0) == "TA_ERR_INVALID_ARG"
+    assert m(a, a, a, a, 0, 128, 0) == "TA_OK"
+    fin = lambda *x: code(lib, lib.attn_lse_merge_finish(*x, stream=0, check=False))
+    assert fin(a, a, 16, 96) == "TA_ERR_UNSUPPORTED"
+    assert fin(a, a + 4, 16, 128) == "TA_ERR_INVALID_ARG"
+    assert fin(a, a, 0, 128) == "TA_OK"
