@@ -1,5 +1,5 @@
 """fp64 CPU oracle for exact attention, its paged forms (decode and varlen
-prefill) and its gradients.
+prefill), its FP8-input form and its gradients.
 
 TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
 benchmark's CPU-baseline leg import this package; the library under
@@ -41,6 +41,12 @@ def _bind(path):
     L.oracle_attn_bwd.argtypes = [c_u16p, c_u16p, c_u16p, c_u16p] + [ctypes.c_int] * 6 + [
         ctypes.c_double, ctypes.c_int, c_i64p, ctypes.c_int64, c_dp, c_dp, c_dp]
     L.oracle_attn_bwd.restype = ctypes.c_int
+    c_u8p = ctypes.POINTER(ctypes.c_uint8)
+    L.oracle_e4m3_decode.argtypes = [c_u8p, ctypes.c_int64, c_dp]
+    L.oracle_e4m3_decode.restype = None
+    L.oracle_attn_fp8.argtypes = [c_u8p, c_u8p, c_u8p] + [ctypes.c_double] * 3 + [ctypes.c_int] * 6 + [
+        ctypes.c_double, ctypes.c_int, c_i64p, ctypes.c_int64, c_dp, c_dp]
+    L.oracle_attn_fp8.restype = ctypes.c_int
     L.oracle_num_threads.restype = ctypes.c_int
     L.oracle_set_num_threads.argtypes = [ctypes.c_int]
     return L
@@ -101,6 +107,49 @@ def attn(q, k, v, causal: bool, scale: float | None = None, rows=None, _L=None):
                             _p(o, ctypes.c_double), _p(lse, ctypes.c_double))
     if err:
         raise OracleError(f"oracle_attn failed with code {err}")
+    o, lse = o[:n], lse[:n]
+    if rows is None:
+        return o.reshape(B, Hq, Nq, d), lse.reshape(B, Hq, Nq)
+    return o, lse
+
+
+def e4m3_decode(codes, _L=None):
+    """Values (float64) of OCP E4M3 ("e4m3fn") codes; NaN for S.1111.111."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(codes.shape, dtype=np.float64)
+    (_L or lib()).oracle_e4m3_decode(_p(codes, ctypes.c_uint8), codes.size, _p(out, ctypes.c_double))
+    return out
+
+
+def attn_fp8(q, k, v, descale, causal: bool, scale: float | None = None, rows=None, _L=None):
+    """Exact attention in fp64 of FP8 inputs.
+
+    q [B,Hq,Nq,d], k/v [B,Hkv,Nkv,d] as uint8 E4M3 codes; descale =
+    (q_descale, k_descale, v_descale), the real inputs being q_descale * e4m3(q)
+    and so on.  rows and the returned shapes as attn().
+    """
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    k = np.ascontiguousarray(k, dtype=np.uint8)
+    v = np.ascontiguousarray(v, dtype=np.uint8)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nkv, _ = k.shape
+    dq, dk, dv = (float(x) for x in descale)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if rows is None:
+        n = B * Hq * Nq
+        rp = None
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        n = rows.size
+        rp = _p(rows, ctypes.c_int64)
+    o = np.zeros((max(n, 1), d), dtype=np.float64)
+    lse = np.zeros(max(n, 1), dtype=np.float64)
+    err = (_L or lib()).oracle_attn_fp8(_p(q, ctypes.c_uint8), _p(k, ctypes.c_uint8), _p(v, ctypes.c_uint8),
+                                        dq, dk, dv, B, Hq, Hkv, Nq, Nkv, d, float(scale), int(bool(causal)), rp, n,
+                                        _p(o, ctypes.c_double), _p(lse, ctypes.c_double))
+    if err:
+        raise OracleError(f"oracle_attn_fp8 failed with code {err}")
     o, lse = o[:n], lse[:n]
     if rows is None:
         return o.reshape(B, Hq, Nq, d), lse.reshape(B, Hq, Nq)
@@ -252,3 +301,9 @@ class Variant:
 
     def paged_prefill(self, *a, **kw):
         return paged_prefill(*a, _L=self._L, **kw)
+
+    def e4m3_decode(self, *a, **kw):
+        return e4m3_decode(*a, _L=self._L, **kw)
+
+    def attn_fp8(self, *a, **kw):
+        return attn_fp8(*a, _L=self._L, **kw)

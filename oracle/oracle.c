@@ -24,7 +24,12 @@
  *  - the paged cache is [num_pages_total, Hkv, page_size, d]; logical token t
  *    of sequence s lives at page block_table[s][t / page_size], row
  *    t % page_size (paged-gather article, section 2.1/2.3: a per-sequence list
- *    of physical blocks); table entries beyond the sequence are never read.
+ *    of physical blocks); table entries beyond the sequence are never read;
+ *  - FP8 attention (the FP8 tensor-core variant named in the LLM-inference
+ *    page's Flash Attention V3 section) takes E4M3 codes with one descale
+ *    factor per tensor; its result here is the exact attention of the
+ *    dequantised values.  Rounding P to FP8 for a tensor-core P.V product is
+ *    part of a kernel's error, not of the definition.
  *
  * All bf16 inputs are passed as uint16 bit patterns and widened exactly.
  */
@@ -177,6 +182,130 @@ int oracle_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             double l;
             attend_row(qi, kb, vb, Nkv, d, scale, visible_keys(i, Nq, Nkv, causal),
                        s, o + (size_t)r * d, &l);
+            if (lse)
+                lse[r] = l;
+        }
+        free(s);
+    }
+    return err;
+}
+
+/*
+ * FP8 inputs.  A code is an OCP 8-bit float in the E4M3 form ("e4m3fn"):
+ * sign bit, 4 exponent bits with bias 7, 3 mantissa bits.  Exponent field 0
+ * holds the subnormals m/8 * 2^-6; there is no infinity, and S.1111.111 is NaN,
+ * so the largest finite magnitude is 1.75 * 2^8 = 448.
+ */
+static double e4m3_to_f64(uint8_t b)
+{
+    int e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);          /* (m / 8) * 2^(1 - 7) */
+    else
+        v = ldexp(8.0 + m, e - 10);        /* (1 + m / 8) * 2^(e - 7) */
+    return (b & 0x80) ? -v : v;
+}
+
+void oracle_e4m3_decode(const uint8_t *codes, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = e4m3_to_f64(codes[i]);
+}
+
+/*
+ * One query row of FP8 attention: the same three sweeps as attend_row, on the
+ * dequantised values dq * e4m3(q), dk * e4m3(k), dv * e4m3(v).
+ */
+static void attend_row_fp8(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                           double dq, double dk, double dv, int n, int d, double scale,
+                           int visible, double *s, double *o, double *lse)
+{
+    for (int j = 0; j < n; ++j) {
+        if (j >= visible) {
+            s[j] = -INFINITY;
+            continue;
+        }
+        double acc = 0.0;
+        const uint8_t *kj = k + (size_t)j * d;
+        for (int t = 0; t < d; ++t)
+            acc += (dq * e4m3_to_f64(q[t])) * (dk * e4m3_to_f64(kj[t]));
+        s[j] = scale * acc;
+    }
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j)
+        if (s[j] > m)
+            m = s[j];
+    for (int t = 0; t < d; ++t)
+        o[t] = 0.0;
+    if (m == -INFINITY) {
+        *lse = -INFINITY;
+        return;
+    }
+    double l = 0.0;
+    for (int j = 0; j < n; ++j)
+        if (s[j] != -INFINITY)
+            l += exp(s[j] - m);
+    for (int j = 0; j < n; ++j) {
+        if (s[j] == -INFINITY)
+            continue;
+        double p = exp(s[j] - m) / l;
+        const uint8_t *vj = v + (size_t)j * d;
+        for (int t = 0; t < d; ++t)
+            o[t] += p * (dv * e4m3_to_f64(vj[t]));
+    }
+    *lse = m + log(l);
+}
+
+/*
+ * Contiguous FP8 attention: q [B,Hq,Nq,d], k/v [B,Hkv,Nkv,d] as E4M3 codes,
+ * one descale factor per tensor (the real inputs are q_descale * e4m3(q) and
+ * so on).  The exact attention of the dequantised inputs; rows, masking, head
+ * mapping and outputs as oracle_attn.
+ */
+int oracle_attn_fp8(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                    double q_descale, double k_descale, double v_descale,
+                    int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                    double scale, int causal, const int64_t *rows, int64_t nrows,
+                    double *o, double *lse)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nkv < 0 || d <= 0 || Hq % Hkv)
+        return ORACLE_ERR_ARG;
+    const int64_t total = (int64_t)B * Hq * Nq;
+    if (!rows)
+        nrows = total;
+    const int G = Hq / Hkv;
+    int err = ORACLE_OK;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Nkv > 0 ? Nkv : 1));
+        if (!s) {
+#pragma omp atomic write
+            err = ORACLE_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < nrows; ++r) {
+            if (!s)
+                continue;
+            int64_t id = rows ? rows[r] : r;
+            if (id < 0 || id >= total) {
+#pragma omp atomic write
+                err = ORACLE_ERR_ARG;
+                continue;
+            }
+            int i = (int)(id % Nq);
+            int64_t bh = id / Nq;
+            int hq = (int)(bh % Hq);
+            int b = (int)(bh / Hq);
+            int hkv = hq / G;
+            const uint8_t *qi = q + (size_t)id * d;
+            const uint8_t *kb = k + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
+            const uint8_t *vb = v + ((size_t)b * Hkv + hkv) * (size_t)Nkv * d;
+            double l;
+            attend_row_fp8(qi, kb, vb, q_descale, k_descale, v_descale, Nkv, d, scale,
+                           visible_keys(i, Nq, Nkv, causal), s, o + (size_t)r * d, &l);
             if (lse)
                 lse[r] = l;
         }

@@ -10,7 +10,10 @@ of oracle.c) and raises AssertionError when the oracle disagrees with:
   permutation of key/value pairs);
 * the online-softmax recurrence for arbitrary tilings and key orders, and the
   split + log-sum-exp merge (FlashAttention optimisation article, 3.2.1-3.2.2);
-* an explicit page gather checked against the contiguous rows it was paged from.
+* an explicit page gather checked against the contiguous rows it was paged from;
+* for FP8 inputs: every E4M3 code against torch's float8_e4m3fn conversion and
+  the format's closed forms, brute force on the library-decoded values, and the
+  bf16 oracle where the descaled values are exactly bfloat16.
 """
 from __future__ import annotations
 
@@ -496,6 +499,82 @@ def pin_bwd_grouped_heads(orc):
         _close(dv1.reshape(B, Hkv, G, Nkv, d).sum(axis=2), dv, tol=1e-11, what="gqa dv")
 
 
+# --------------------------------------------------------------------------
+# FP8 (E4M3) inputs
+# --------------------------------------------------------------------------
+
+def _torch_e4m3(codes):
+    """E4M3 codes -> float64 through torch's float8_e4m3fn type (a library
+    conversion, independent of the oracle's decoder)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def _fp8(rng, shape):
+    from tiled_attention_17_b200.inputs import quantize_e4m3
+    codes, _ = quantize_e4m3(rng.standard_normal(int(np.prod(shape))).astype(np.float32))
+    return codes.reshape(shape)
+
+
+def pin_e4m3_codes(orc):
+    codes = np.arange(256, dtype=np.uint8)
+    got = orc.e4m3_decode(codes)
+    ref = _torch_e4m3(codes)
+    nan = np.isnan(ref)
+    if not np.array_equal(np.isnan(got), nan):
+        raise AssertionError("e4m3: NaN codes differ from the library's")
+    if not np.array_equal(got[~nan], ref[~nan]):
+        bad = np.nonzero(got[~nan] != ref[~nan])[0][:4]
+        raise AssertionError(f"e4m3: codes {codes[~nan][bad]} decode to {got[~nan][bad]}, library {ref[~nan][bad]}")
+    # closed forms of the format: smallest subnormal, smallest normal, one, largest finite, signs
+    for code, val in ((0x01, 2.0 ** -9), (0x08, 2.0 ** -6), (0x38, 1.0), (0x7E, 448.0), (0xB8, -1.0),
+                      (0xFE, -448.0)):
+        if got[code] != val:
+            raise AssertionError(f"e4m3 code {code:#x}: {got[code]} != {val}")
+    if not (np.isnan(got[0x7F]) and np.isnan(got[0xFF])):
+        raise AssertionError("e4m3: S.1111.111 must be NaN")
+
+
+def pin_fp8_brute_force(orc):
+    """FP8 attention on tiny inputs against the textbook definition evaluated
+    on the library-decoded, descaled values."""
+    rng = np.random.Generator(np.random.PCG64(19))
+    for (B, Hq, Hkv, Nq, Nkv, d) in ((1, 2, 1, 5, 7, 4), (2, 2, 2, 6, 6, 3), (1, 1, 1, 3, 9, 8)):
+        for causal in (False, True):
+            q8, k8, v8 = _fp8(rng, (B, Hq, Nq, d)), _fp8(rng, (B, Hkv, Nkv, d)), _fp8(rng, (B, Hkv, Nkv, d))
+            desc = (0.037, 0.0081, 0.0059)
+            scale = 0.9
+            o, lse = orc.attn_fp8(q8, k8, v8, desc, causal, scale=scale)
+            Q, K, V = (_torch_e4m3(x) * s for x, s in zip((q8, k8, v8), desc))
+            G = Hq // Hkv
+            for b in range(B):
+                for h in range(Hq):
+                    for i in range(Nq):
+                        ob, lb = brute_row(Q[b, h, i], K[b, h // G], V[b, h // G], scale,
+                                           _visible(i, Nq, Nkv, causal))
+                        _close(o[b, h, i], ob, what=f"fp8 brute o row {b, h, i}")
+                        _close(lse[b, h, i], lb, what=f"fp8 brute lse row {b, h, i}")
+
+
+def pin_fp8_is_bf16_attention(orc):
+    """Every E4M3 value times a power of two (within range) is a bfloat16 value,
+    so FP8 attention with power-of-two descales must equal the bf16 oracle on
+    those values, to rounding."""
+    rng = np.random.Generator(np.random.PCG64(23))
+    B, Hq, Hkv, Nq, Nkv, d = 1, 4, 2, 40, 56, 16
+    q8, k8, v8 = _fp8(rng, (B, Hq, Nq, d)), _fp8(rng, (B, Hkv, Nkv, d)), _fp8(rng, (B, Hkv, Nkv, d))
+    for desc in ((1.0, 1.0, 1.0), (2.0 ** -6, 2.0 ** -7, 4.0)):
+        bits = [f32_to_bf16_bits((_torch_e4m3(x) * s).astype(np.float32)) for x, s in zip((q8, k8, v8), desc)]
+        for causal in (False, True):
+            o8, l8 = orc.attn_fp8(q8, k8, v8, desc, causal, scale=0.25)
+            ob, lb = orc.attn(*bits, causal, scale=0.25)
+            _close(o8, ob, tol=1e-12, what=f"fp8 vs bf16 o desc={desc} causal={causal}")
+            _close(l8, lb, tol=1e-12, what=f"fp8 vs bf16 lse desc={desc} causal={causal}")
+
+
+FP8_PINS = [pin_e4m3_codes, pin_fp8_brute_force, pin_fp8_is_bf16_attention]
+
 BWD_PINS = [pin_bwd_finite_differences, pin_bwd_single_key, pin_bwd_scale_zero,
             pin_bwd_key_gradients_sum_to_zero, pin_bwd_permutation, pin_bwd_grouped_heads]
 
@@ -503,4 +582,4 @@ ALL_PINS = [pin_brute_force, pin_large_scores, pin_handpicked, pin_rows_of_p_sum
             pin_constant_v, pin_permutation_invariance, pin_single_key, pin_scale_zero,
             pin_causal_row0, pin_identical_keys, pin_online_recurrence, pin_paged_gather,
             pin_paged_decode, pin_paged_prefill_brute_force, pin_paged_prefill_one_query_is_decode,
-            pin_paged_prefill_matches_dense] + BWD_PINS
+            pin_paged_prefill_matches_dense] + BWD_PINS + FP8_PINS

@@ -38,6 +38,14 @@ MUTANTS = {
     "bwd_dp_from_k": ("dp[j] = dot_bf16(doi, vb + (size_t)j * d, d);", "dp[j] = dot_bf16(doi, kb + (size_t)j * d, d);"),
     "bwd_key_sweep_dp_from_k": ("double ds = p * (dot_bf16(doi, vj, d) - rr[x]);", "double ds = p * (dot_bf16(doi, kj, d) - rr[x]);"),
     "bwd_key_sweep_unnormalised": ("- rm[x]) / rl[x];", "- rm[x]);"),
+    # FP8 inputs
+    "e4m3_exponent_bias": ("v = ldexp(8.0 + m, e - 10);", "v = ldexp(8.0 + m, e - 11);"),
+    "e4m3_subnormal_scale": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "e4m3_sign_ignored": ("return (b & 0x80) ? -v : v;", "return v;"),
+    "e4m3_no_nan": ("if (e == 15 && m == 7)\n        return NAN;", "if (0)\n        return NAN;"),
+    "fp8_v_descale_dropped": ("o[t] += p * (dv * e4m3_to_f64(vj[t]));", "o[t] += p * e4m3_to_f64(vj[t]);"),
+    "fp8_k_descale_dropped": ("(dk * e4m3_to_f64(kj[t]))", "e4m3_to_f64(kj[t])"),
+    "fp8_q_descale_squared": ("(dq * e4m3_to_f64(q[t]))", "(dq * dq * e4m3_to_f64(q[t]))"),
     "bwd_key_sweep_mask_ignored": ("if (j >= visible_keys(i, Nq, Nkv, causal))\n                    continue;", "if (0)\n                    continue;"),
 }
 

@@ -2,8 +2,8 @@
 
 This module is shared by the CUDA path's tests/benchmark and by the CPU oracle's
 tests.  It holds no attention arithmetic: it only draws N(0, 1) numbers, rounds
-them to bfloat16 bit patterns, and lays out the paged KV pool and its block
-table.  Everything is a deterministic function of the seed.
+them to bfloat16 bit patterns (or quantises them to FP8 E4M3 codes with a
+per-tensor scale), and lays out the paged KV pool and its block table.  Everything is a deterministic function of the seed.
 
 Workloads (shapes and value recipes of the fused-attention pages: FlashAttention
 optimisation article, sections 2.1 and 3.1 for N=4096/d=128; the Gemini 3 Flash
@@ -140,6 +140,64 @@ def random_prefill(B, Hq, Hkv, Nq, Nkv, d, seed, scale_k_rows_every=0, factor=1.
     """Small ad-hoc prefill inputs (tests): (q, k, v) uint16 bf16 bits."""
     cfg = PrefillConfig("adhoc", B, Hq, Hkv, Nq, Nkv, d, False, scale_k_rows_every, factor)
     return prefill_inputs(cfg, seed)
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) prefill inputs
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0   # largest finite OCP E4M3 ("e4m3fn") magnitude
+
+
+def f32_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values (|x| <= 448) to OCP E4M3 codes (nearest, ties to
+    even) with torch's float8_e4m3fn conversion; return uint8 codes."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def quantize_e4m3(x: np.ndarray):
+    """Per-tensor quantisation: descale = amax / 448 (float32) and codes =
+    e4m3(x / descale), so descale * e4m3(code) approximates x."""
+    amax = float(np.max(np.abs(x))) if x.size else 1.0
+    descale = np.float32(amax / E4M3_MAX if amax > 0 else 1.0)
+    codes = f32_to_e4m3_bits(np.clip(x / descale, -E4M3_MAX, E4M3_MAX).astype(np.float32))
+    return codes, float(descale)
+
+
+def random_prefill_fp8(B, Hq, Hkv, Nq, Nkv, d, seed):
+    """FP8 prefill inputs: the float32 N(0, 1) draws of prefill_inputs (same
+    seed streams), each tensor quantised to E4M3 with its own descale.
+    Returns (q8, k8, v8, (q_descale, k_descale, v_descale)), codes as uint8."""
+    out, ds = [], []
+    for word, shape in ((0, (B, Hq, Nq, d)), (1, (B, Hkv, Nkv, d)), (2, (B, Hkv, Nkv, d))):
+        x = _chunked_f32([seed, word], int(np.prod(shape)))
+        codes, descale = quantize_e4m3(x)
+        out.append(codes.reshape(shape))
+        ds.append(descale)
+    return out[0], out[1], out[2], tuple(ds)
+
+
+def fp8_integer_score_inputs(B, Hq, Hkv, Nq, Nkv, d, seed, nnz=3):
+    """FP8 inputs whose scores q.k are small integers: every Q and K row has
+    `nnz` entries of +-1 at seeded positions (zeros elsewhere), so |q.k| <= nnz;
+    V is N(0, 1) quantised per tensor.  With scale = ln 2 every softmax weight
+    relative to any score of the row is an exact power of two, which FP8
+    represents exactly.  Returns (q8, k8, v8, v_descale)."""
+    rng = np.random.Generator(np.random.PCG64([seed, 0xF8]))
+
+    def sparse_rows(rows):
+        x = np.zeros((rows, d), dtype=np.float32)
+        for r in range(rows):
+            cols = rng.choice(d, size=nnz, replace=False)
+            x[r, cols] = rng.choice(np.array([-1.0, 1.0], dtype=np.float32), size=nnz)
+        return f32_to_e4m3_bits(x)
+
+    q8 = sparse_rows(B * Hq * Nq).reshape(B, Hq, Nq, d)
+    k8 = sparse_rows(B * Hkv * Nkv).reshape(B, Hkv, Nkv, d)
+    v8, dv = quantize_e4m3(_chunked_f32([seed, 2], B * Hkv * Nkv * d))
+    return q8, k8, v8.reshape(B, Hkv, Nkv, d), dv
 
 
 # --------------------------------------------------------------------------
