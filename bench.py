@@ -346,6 +346,11 @@ def run_ours(args):
     if not args.no_backward:
         bwd = run_backward(args, torch, binding, dev, stream, q, k, v, o, lse, flush, dist, rank, world, peaks)
 
+    # ---- FP8 (E4M3) prefill on the same shape (timed on its own, after the step)
+    fp8 = None
+    if not args.no_fp8:
+        fp8 = run_fp8_prefill(args, torch, binding, dev, stream, flush, dist, rank, world, peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(q_h, k_h, v_h, args.cpu_stride)
@@ -371,6 +376,7 @@ def run_ours(args):
                        "e2e": dec_e2e},
             "backward": bwd,
             "paged_prefill": paged,
+            "fp8_prefill": fp8,
             "roofline": roofline("tensor", pre_per_gpu, peaks["bf16_tflops"], "TFLOP/s",
                                  recorded_traffic("prefill_fwd_kernel", "prefill_sm100.cu", float(c.B * c.Hq))),
             "peaks": {"source": peak_kind, "bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"],
@@ -485,6 +491,46 @@ def run_backward(args, torch, binding, dev, stream, q, k, v, o, lse, flush, dist
                                  recorded_traffic("attn_bwd", "backward_sm100.cu", float(c.B * c.Hkv)))}
 
 
+def run_fp8_prefill(args, torch, binding, dev, stream, flush, dist, rank, world, peaks):
+    """attn_fwd_fp8 on the causal prefill workload's shape (the same N(0, 1)
+    draws quantised per tensor to E4M3): CUDA events around each call, L2
+    flushed before every call, max over ranks.  The roofline peak is the
+    measured bf16 GEMM peak times the nominal fp8/bf16 ratio (4.5 / 2.25)."""
+    c = PREFILL
+    q8, k8, v8, desc = inputs.random_prefill_fp8(c.B, c.Hq, c.Hkv, c.Nq, c.Nkv, c.d,
+                                                 seed=rank_seed(inputs.CONFIG_SEEDS["causal"], rank))
+    q, k, v = (torch.from_numpy(x).to(dev) for x in (q8, k8, v8))
+    o = torch.empty((c.B, c.Hq, c.Nq, c.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+
+    def call():
+        binding.attn_fwd_fp8(q, k, v, *desc, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nkv, c.d, c.scale, 1, stream)
+
+    for _ in range(3):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(dist, dev.index)
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+    (t,) = max_over_ranks([t], dist, device=dev)
+    flops = accounting.prefill_flops(c.B, c.Hq, c.Nq, c.Nkv, c.d, True)
+    per_gpu = flops / (t * 1e-3) / 1e12
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    return {"value": per_gpu * world, "unit": "TFLOP/s", "ms": t, "steps": steps, "dtype": "e4m3 in, f32 accumulate",
+            "flops_per_call_per_gpu": flops, "gpu_launches_per_call": 1,
+            "vs_bf16_peak": per_gpu / peaks["bf16_tflops"],
+            "roofline": roofline("tensor", per_gpu, fp8_peak, "TFLOP/s",
+                                 recorded_traffic("prefill_fwd_kernel_fp8", "prefill_sm100.cu", float(c.B * c.Hq)))}
+
+
 def roofline(bound, achieved, peak, unit, traffic):
     return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
             "traffic": traffic}
@@ -587,7 +633,16 @@ def run_ncu_case(args):
     def dev_bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    if args.ncu_case == "paged":
+    if args.ncu_case == "fp8":
+        c = PREFILL
+        q8, k8, v8, desc = inputs.random_prefill_fp8(c.B, c.Hq, c.Hkv, c.Nq, c.Nkv, c.d,
+                                                     seed=inputs.CONFIG_SEEDS["causal"])
+        q, k, v = (torch.from_numpy(x).to(dev) for x in (q8, k8, v8))
+        o = torch.empty((c.B, c.Hq, c.Nq, c.d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+        for _ in range(args.reps):
+            binding.attn_fwd_fp8(q, k, v, *desc, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nkv, c.d, c.scale, 1)
+    elif args.ncu_case == "paged":
         m = PAGED_MIX
         rng = np.random.Generator(np.random.PCG64(4321))
         q_lens = rng.integers(m["q_lo"], m["q_hi"], size=m["num_seqs"], endpoint=True)
@@ -642,7 +697,8 @@ def main(argv=None):
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-paged-prefill", action="store_true")
-    ap.add_argument("--ncu-case", choices=["prefill", "decode", "backward", "paged"], default=None,
+    ap.add_argument("--no-fp8", action="store_true")
+    ap.add_argument("--ncu-case", choices=["prefill", "decode", "backward", "paged", "fp8"], default=None,
                     help="run a small single-kernel case for a profiler capture and exit")
     ap.add_argument("--reps", type=int, default=4)
     args = ap.parse_args(argv)

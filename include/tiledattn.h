@@ -92,6 +92,28 @@ ta_status attn_fwd(const void *q, const void *k, const void *v, void *o, float *
                    float scale, int causal, ta_stream_t stream);
 
 /*
+ * attn_fwd_fp8 - fused attention forward with FP8 inputs (the FP8 tensor-core
+ * variant of the LLM-inference page's Flash Attention V3 section).
+ *
+ *   q   [B, Hq,  Nq,  d]  E4M3 codes  o   [B, Hq, Nq, d] bf16 (written)
+ *   k   [B, Hkv, Nkv, d]  E4M3 codes  lse [B, Hq, Nq]    fp32 (written; may be NULL)
+ *   v   [B, Hkv, Nkv, d]  E4M3 codes
+ *
+ * One byte per element in the OCP E4M3 form ("e4m3fn": bias 7, no infinity,
+ * largest finite 448).  The real inputs are q_descale * e4m3(q), k_descale *
+ * e4m3(k), v_descale * e4m3(v) (one factor per tensor, finite and > 0), and
+ * the result approximates the attention of those values: the scores are
+ * exact products accumulated in fp32, but the softmax weights are rounded to
+ * E4M3 for the FP8 P.V product (relative error up to 2^-4 per weight, about
+ * 2.6% RMS), so O carries an error of a few percent of its magnitude; lse is
+ * as accurate as attn_fwd's.  Scale, causal alignment, GQA mapping, empty
+ * cases and alignment rules as attn_fwd.  Supported: d = 128.
+ */
+ta_status attn_fwd_fp8(const void *q, const void *k, const void *v, float q_descale, float k_descale,
+                       float v_descale, void *o, float *lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                       float scale, int causal, ta_stream_t stream);
+
+/*
  * attn_paged_prefill - varlen (chunked) prefill against the paged KV cache:
  * the new query tokens of several sequences, packed, attend over their
  * sequences' keys in the page pool (chunked prefill, LLM-inference article

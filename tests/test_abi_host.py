@@ -95,6 +95,27 @@ def test_attn_fwd_validation(lib):
     assert f(None, None, None, None, None, 1, 1, 1, 0, 128, 128, 0.1, 0) == "TA_OK"
 
 
+def test_attn_fwd_fp8_validation(lib):
+    a = 256
+    f = lambda *x: code(lib, lib.attn_fwd_fp8(*x, check=False, stream=0))
+
+    def call(q=a, lse=None, dq=0.01, dk=0.02, dv=0.03, B=1, Hq=2, Hkv=1, d=128, scale=0.1, causal=1):
+        return f(q, a, a, dq, dk, dv, a, lse, B, Hq, Hkv, 256, 256, d, scale, causal)
+
+    assert call(d=64) == "TA_ERR_UNSUPPORTED"                 # fp8 path: d = 128 only
+    assert call(Hq=3, Hkv=2) == "TA_ERR_INVALID_ARG"
+    assert call(dq=0.0) == "TA_ERR_INVALID_ARG"               # descales finite and > 0
+    assert call(dk=-1.0) == "TA_ERR_INVALID_ARG"
+    assert call(dv=float("inf")) == "TA_ERR_INVALID_ARG"
+    assert call(dq=1e30, dk=1e30) == "TA_ERR_UNSUPPORTED"     # folded score scale overflows fp32
+    assert call(scale=-1.0) == "TA_ERR_UNSUPPORTED"
+    assert call(causal=3) == "TA_ERR_INVALID_ARG"
+    assert call(q=a + 1) == "TA_ERR_INVALID_ARG"              # 16-byte alignment
+    assert call(lse=a + 2) == "TA_ERR_INVALID_ARG"
+    assert call(q=None) == "TA_ERR_INVALID_ARG"
+    assert call(B=0) == "TA_OK"
+
+
 def test_decode_validation(lib):
     a = 256
     f = lambda *x: code(lib, lib.attn_paged_decode(*x, check=False, stream=0))

@@ -24,7 +24,8 @@ TA_DEV_TIMEOUT = 1
 TA_DEV_BAD_BLOCK_TABLE = 2
 TA_DEV_BAD_SEQ_LEN = 4
 
-EXPORTS = ["ta_status_string", "ta_version", "ta_last_error", "attn_fwd", "attn_bwd_workspace_size", "attn_bwd",
+EXPORTS = ["ta_status_string", "ta_version", "ta_last_error", "attn_fwd", "attn_fwd_fp8", "attn_bwd_workspace_size",
+           "attn_bwd",
            "attn_paged_prefill", "attn_lse_merge", "attn_lse_merge_finish",
            "attn_paged_decode_workspace_size",
            "attn_paged_decode", "attn_paged_decode_noalloc", "attn_paged_decode_check", "attn_paged_gather_debug",
@@ -58,6 +59,8 @@ def load(path: str | None = None):
     L.ta_last_error.restype = ctypes.c_char_p
     L.attn_fwd.argtypes = [vp, vp, vp, vp, vp] + [i32] * 6 + [f32, i32, vp]
     L.attn_fwd.restype = i32
+    L.attn_fwd_fp8.argtypes = [vp, vp, vp, f32, f32, f32, vp, vp] + [i32] * 6 + [f32, i32, vp]
+    L.attn_fwd_fp8.restype = i32
     L.attn_paged_prefill.argtypes = [vp] * 6 + [i32] * 9 + [f32, i32, vp, vp, vp]
     L.attn_paged_prefill.restype = i32
     i64 = ctypes.c_int64
@@ -131,6 +134,15 @@ def attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream=None
                            float(scale), int(causal), _stream(stream))
     if check:
         _check("attn_fwd", code)
+    return code
+
+
+def attn_fwd_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal,
+                 stream=None, check=True) -> int:
+    code = load().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), float(q_descale), float(k_descale), float(v_descale),
+                               _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nkv, d, float(scale), int(causal), _stream(stream))
+    if check:
+        _check("attn_fwd_fp8", code)
     return code
 
 
@@ -247,6 +259,26 @@ def attention(q, k, v, causal: bool, scale: float | None = None, out=None, lse=N
     if lse is None:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream)
+    return o, lse
+
+
+def attention_fp8(q, k, v, descale, causal: bool, scale: float | None = None, out=None, lse=None, stream=None):
+    """q [B,Hq,Nq,128], k/v [B,Hkv,Nkv,128] contiguous CUDA tensors of E4M3
+    codes (torch.float8_e4m3fn or uint8); descale = (q_descale, k_descale,
+    v_descale) -> (o bf16, lse fp32)."""
+    import torch
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nkv, _ = k.shape
+    for t in (q, k, v):
+        if t.dtype not in (torch.float8_e4m3fn, torch.uint8) or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous float8_e4m3fn (or uint8) CUDA tensors")
+    if scale is None:
+        scale = d ** -0.5
+    o = out if out is not None else torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    dq, dk, dv = descale
+    attn_fwd_fp8(q, k, v, dq, dk, dv, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream)
     return o, lse
 
 

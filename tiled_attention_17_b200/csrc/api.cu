@@ -50,8 +50,8 @@ PFN_encodeTiled get_encode_tiled() {
   return fn;
 }
 
-ta_status encode_bf16_tiled(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                            const uint64_t* strides_bytes, const uint32_t* box) {
+static ta_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int rank,
+                              const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
   PFN_encodeTiled enc = get_encode_tiled();
   if (!enc) return fail(TA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t d[5], st[4];
@@ -62,10 +62,22 @@ ta_status encode_bf16_tiled(CUtensorMap* map, const void* base, int rank, const 
     estr[i] = 1;
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d,
+  CUresult r = enc(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d,
                    st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? TA_OK : fail_cu(TA_ERR_CUDA, "cuTensorMapEncodeTiled", static_cast<int>(r));
+}
+
+ta_status encode_bf16_tiled(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                            const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box);
+}
+
+ta_status encode_u8_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows), static_cast<uint64_t>(slices)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows) * d};
+  const uint32_t box[3] = {128, 128, 1};
+  return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 3, dims, strides, box);
 }
 
 ta_status encode_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
@@ -131,6 +143,29 @@ ta_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* 
   const long long pairs = (static_cast<long long>(Nq) + 255) / 256;
   if (pairs * B * Hq > INT32_MAX) return TA_ERR_UNSUPPORTED;
   return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ta_status attn_fwd_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+                       float v_descale, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                       float scale, int causal, ta_stream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nkv < 0 || d <= 0) return TA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return TA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return TA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return TA_ERR_UNSUPPORTED;
+  for (float ds : {q_descale, k_descale, v_descale})
+    if (!std::isfinite(ds) || ds <= 0.f) return TA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale * q_descale * k_descale)) return TA_ERR_UNSUPPORTED;
+  if (d != 128) return TA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq > INT32_MAX / 2 || Nq > (1 << 30) || Nkv > (1 << 30)) return TA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hq * Nq == 0) return TA_OK;
+  if (!q || !o || (Nkv > 0 && (!k || !v))) return TA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return TA_ERR_INVALID_ARG;
+  const long long pairs = (static_cast<long long>(Nq) + 255) / 256;
+  if (pairs * B * Hq > INT32_MAX) return TA_ERR_UNSUPPORTED;
+  return launch_prefill_fp8(q, k, v, q_descale, k_descale, v_descale, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 ta_status attn_paged_prefill(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,

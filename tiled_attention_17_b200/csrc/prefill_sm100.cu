@@ -61,13 +61,18 @@ constexpr float kRescaleLog2 = 8.0f;   // skip O rescale while max grew by <= 2^
 // them there was measured: none was faster on B200, so all stay on MUFU.
 constexpr unsigned kPolyMask = 0x00u;
 
-template <int D>
+template <int D, bool kFp8 = false>
 struct PrefillLayout {
   static_assert(D == 64 || D == 128, "head dim");
-  static constexpr int kChunks = D / 64;              // 64-column (128-byte) swizzle atoms along d
-  static constexpr int kTileBytes = 128 * D * 2;      // one 128-row bf16 tile
-  static constexpr int kChunkBytes = 128 * 128;       // 128 rows x 128 bytes
-  static constexpr int kStages = (D == 128) ? 2 : 3;  // K ring and V ring depth
+  static_assert(!kFp8 || D == 128, "fp8 inputs: d = 128 (one 128-byte swizzle row)");
+  static constexpr int kElemBytes = kFp8 ? 1 : 2;
+  static constexpr int kChunkElems = 128 / kElemBytes;           // elements of one 128-byte swizzle row
+  static constexpr int kChunks = D / kChunkElems;                // swizzle atoms along d
+  static constexpr int kTileBytes = 128 * D * kElemBytes;        // one 128-row tile
+  static constexpr int kChunkBytes = 128 * 128;                  // 128 rows x 128 bytes
+  static constexpr int kStages = (kTileBytes > kChunkBytes) ? 2 : 3;  // K ring and V ring depth
+  static constexpr int kKeysPerMma = 32 / kElemBytes;            // one MMA reads 32 bytes of each row
+  static constexpr int kPWords = 64 * kElemBytes / 4;            // TMEM columns of one half (64 keys) of P
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
@@ -98,6 +103,9 @@ struct PrefillArgs {
   const int32_t* cu_seqlens;
   const int32_t* seq_lens;
   int num_seqs, total_q, max_q_len, page_size, max_pages, num_pages_total;
+  // fp8 inputs: the values are descale * e4m3(code); q and k descales are
+  // folded into scale / scale_log2, v's is applied to O in the epilogue
+  float v_descale;
 };
 
 // Number of K/V tiles query tile [q0, q0+128) must visit (0 if it has no rows
@@ -112,11 +120,12 @@ __device__ __forceinline__ int kv_tiles_for(int q0, int Nq, int Nkv, int causal)
   return kv_end <= 0 ? 0 : (kv_end + kBN - 1) / kBN;
 }
 
-template <int D, bool kPaged>
+template <int D, bool kPaged, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
-  using L = PrefillLayout<D>;
+  static_assert(!(kPaged && kFp8), "fp8 inputs: dense layout only");
+  using L = PrefillLayout<D, kFp8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -210,9 +219,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (q0 >= Nq) continue;
         for (int c = 0; c < L::kChunks; ++c) {
           if constexpr (kPaged)   // packed [total_q, Hq, d]: box of 128 rows of one head
-            tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * 64, hq, q_base + q0);
+            tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, hq,
+                        q_base + q0);
           else
-            tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * 64, q0, zq);
+            tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, q0, zq);
         }
       }
       // Physical pages of K/V tile j (paged): the table entries are read
@@ -245,10 +255,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int p = 0; p < kMaxPagesPerTile; ++p) {
             if (p >= per_tile) break;
             for (int c = 0; c < L::kChunks; ++c)
-              tma_load_4d(dst + c * L::kChunkBytes + p * a.page_size * 128, tm, bar, c * 64, 0, hkv, phys[p]);
+              tma_load_4d(dst + c * L::kChunkBytes + p * a.page_size * 128, tm, bar, c * L::kChunkElems, 0, hkv,
+                          phys[p]);
           }
         } else {
-          for (int c = 0; c < L::kChunks; ++c) tma_load_3d(dst + c * L::kChunkBytes, tm, bar, c * 64, j * kBN, zk);
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_3d(dst + c * L::kChunkBytes, tm, bar, c * L::kChunkElems, j * kBN, zk);
         }
       };
       bool ok = true;
@@ -275,8 +287,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 1 && lane == 0) {
     // ======================= MMA issuer =======================
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+      constexpr uint32_t idesc_qk = kFp8 ? idesc_e4m3_f32(kBM, kBN, false) : idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_pv = kFp8 ? idesc_e4m3_f32(kBM, D, true) : idesc_bf16_f32(kBM, D, true);
+      auto mma_s = [](uint32_t d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
+        if constexpr (kFp8) mma_ss_f8(d, ad, bd, id, acc); else mma_ss(d, ad, bd, id, acc);
+      };
+      auto mma_t = [](uint32_t d, uint32_t at, uint64_t bd, uint32_t id, uint32_t acc) {
+        if constexpr (kFp8) mma_ts_f8(d, at, bd, id, acc); else mma_ts(d, at, bd, id, acc);
+      };
       auto tS = [&](int t) { return tmem + (t ? L::kTmS1 : L::kTmS0); };
       auto tO = [&](int t) { return tmem + (t ? L::kTmO1 : L::kTmO0); };
 
@@ -288,31 +306,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dV = smem_desc_sw128(sV, L::kChunkBytes, 1024);
       constexpr uint64_t kTileStep = L::kTileBytes >> 4;
 
-      // S_t = Q_t K^T over d in 16-wide steps (K-major operands, 128B swizzle)
+      // S_t = Q_t K^T over d in 32-byte steps (K-major operands, 128B swizzle)
       auto issue_qk = [&](int t, int s) {
         uint64_t a0 = dQ + static_cast<uint64_t>(t) * kTileStep;
         uint64_t b0 = dK + static_cast<uint64_t>(s) * kTileStep;
         const uint32_t d = tS(t);
-        // 16-element K steps: +32 B within a 128-byte swizzle row, then the next 64-column chunk
+        // K steps of 32 bytes (16 bf16 or 32 fp8 elements) within a 128-byte
+        // swizzle row, then the next 128-byte chunk of d
 #pragma unroll 1
         for (int c = 0; c < L::kChunks; ++c) {
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4)
-            mma_ss(d, a0 + 2 * k4, b0 + 2 * k4, idesc_qk, (c | k4) != 0);
+            mma_s(d, a0 + 2 * k4, b0 + 2 * k4, idesc_qk, (c | k4) != 0);
           a0 += L::kChunkBytes >> 4;
           b0 += L::kChunkBytes >> 4;
         }
       };
-      // O_t += P_t V over one half (64 keys) of the tile in 16-row steps
-      // (P from TMEM, V MN-major)
+      // O_t += P_t V over one half (64 keys) of the tile, 16 (bf16) or 32
+      // (fp8) keys per MMA (P from TMEM: 8 columns per step either way; V
+      // MN-major, one 128-byte row per key)
       auto issue_pv_half = [&](int t, int s, int half, bool acc) {
+        constexpr int kPerHalf = (kBN / 2) / L::kKeysPerMma;
         const uint64_t b0 = dV + static_cast<uint64_t>(s) * kTileStep;
         const uint32_t d = tO(t), a = tS(t);
 #pragma unroll
-        for (int k4 = 0; k4 < kBN / 32; ++k4) {
-          const int kk = half * (kBN / 32) + k4;
-          mma_ts(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
-                 (acc || kk > 0) ? 1u : 0u);
+        for (int k4 = 0; k4 < kPerHalf; ++k4) {
+          const int kk = half * kPerHalf + k4;
+          mma_t(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * L::kKeysPerMma * 128) >> 4), idesc_pv,
+                (acc || kk > 0) ? 1u : 0u);
         }
       };
 
@@ -401,13 +422,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       // exp2((s - m) * c2) for 32 column pairs [64h, 64h + 64), packed to bf16
-      // pairs; masked columns get exactly 0.  Returns the sum of the values.
+      // pairs (32 words) or to four E4M3 codes per word (fp8: 16 words);
+      // masked columns get exactly 0.  Returns the sum of the unrounded values.
       // The masked form is a separate specialisation so unmasked tiles carry
       // no per-element compare/select.
-      auto exp_half = [&](auto masked, int h, float negm, uint32_t (&pk)[32]) -> float {
+      auto exp_half = [&](auto masked, int h, float negm, uint32_t (&pk)[L::kPWords]) -> float {
         constexpr bool kMasked = decltype(masked)::value;
         const float2 c2v = make_float2(c2, c2), negv = make_float2(negm, negm);
         float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+        float2 pp_prev = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int c = h * 64 + 2 * i;
@@ -423,12 +446,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             pp.x = c < lim ? pp.x : 0.f;
             pp.y = c + 1 < lim ? pp.y : 0.f;
           }
-          if (i & 1) sb = fadd2(sb, pp); else sa = fadd2(sa, pp);
-          pk[i] = pack_bf16x2(pp.x, pp.y);
+          if (i & 1) {
+            sb = fadd2(sb, pp);
+          } else {
+            sa = fadd2(sa, pp);
+          }
+          if constexpr (kFp8) {
+            if (i & 1) pk[i >> 1] = pack_e4m3x4(pp_prev.x, pp_prev.y, pp.x, pp.y);
+            pp_prev = pp;
+          } else {
+            pk[i] = pack_bf16x2(pp.x, pp.y);
+          }
         }
         return (sa.x + sb.x) + (sa.y + sb.y);
       };
-      auto exp_half_any = [&](int h, float negm, uint32_t (&pk)[32]) -> float {
+      auto exp_half_any = [&](int h, float negm, uint32_t (&pk)[L::kPWords]) -> float {
         return need_mask ? exp_half(std::true_type{}, h, negm, pk) : exp_half(std::false_type{}, h, negm, pk);
       };
 
@@ -474,17 +506,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // while the second is computed.
       float psum;
       {
-        uint32_t pk[32];
+        uint32_t pk[L::kPWords];
         psum = exp_half_any(0, negm, pk);
-        tmem_st32(tS, pk);
+        if constexpr (kFp8) tmem_st16(tS, pk); else tmem_st32(tS, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR_PH(t));
       {
-        uint32_t pk[32];
+        uint32_t pk[L::kPWords];
         psum += exp_half_any(1, negm, pk);
-        tmem_st32(tS + 32, pk);
+        if constexpr (kFp8) tmem_st16(tS + L::kPWords, pk); else tmem_st32(tS + L::kPWords, pk);
       }
       l = alpha * l + psum;
 
@@ -504,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // output row: [B, Hq, Nq] (dense) or packed [total_q, Hq] (paged)
     const size_t orow = kPaged ? static_cast<size_t>(q_base + (store ? qrow : 0)) * a.Hq + hq
                                : (static_cast<size_t>(b) * a.Hq + hq) * Nq + qrow;
-    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    const float inv = (l > 0.f) ? (kFp8 ? a.v_descale / l : 1.f / l) : 0.f;
     __nv_bfloat16* optr = a.o + orow * D;
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
@@ -564,7 +596,7 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   if ((st = encode_rows_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
   if ((st = encode_rows_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
   static int attr_done[64] = {0};
-  cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, false>, L::kAlloc, attr_done);
+  cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, false, false>, L::kAlloc, attr_done);
   if (e != cudaSuccess) return fail(TA_ERR_CUDA, "prefill: shared-memory limit", e);
   PrefillArgs a = {};
   a.o = static_cast<__nv_bfloat16*>(o);
@@ -578,10 +610,11 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.v_descale = 1.f;
   a.status = device_status_ptr();
   if (!a.status) return fail(TA_ERR_CUDA, "prefill: device status word");
   const unsigned grid = static_cast<unsigned>(a.n_pairs) * static_cast<unsigned>(B * Hq);
-  prefill_fwd_kernel<D, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
+  prefill_fwd_kernel<D, false, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "prefill: launch", e);
 }
@@ -611,7 +644,7 @@ static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, cons
     if ((st = encode_bf16_tiled(&tv, v_cache, 4, dims, strides, box)) != TA_OK) return st;
   }
   static int attr_done[64] = {0};
-  cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, true>, L::kAlloc, attr_done);
+  cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, true, false>, L::kAlloc, attr_done);
   if (e != cudaSuccess) return fail(TA_ERR_CUDA, "paged prefill: shared-memory limit", e);
   PrefillArgs a = {};
   a.o = static_cast<__nv_bfloat16*>(o);
@@ -623,6 +656,7 @@ static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, cons
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.v_descale = 1.f;
   a.status = device_status_ptr();
   if (!a.status) return fail(TA_ERR_CUDA, "paged prefill: device status word");
   a.block_table = block_table;
@@ -635,9 +669,55 @@ static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, cons
   a.max_pages = max_pages;
   a.num_pages_total = num_pages_total;
   const unsigned grid = static_cast<unsigned>(a.n_pairs) * static_cast<unsigned>(num_seqs * Hq);
-  prefill_fwd_kernel<D, true><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
+  prefill_fwd_kernel<D, true, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "paged prefill: launch", e);
+}
+
+// FP8 (E4M3) inputs, d = 128: Q, K, V [B, H, N, 128] one byte per element.
+// The descales of q and k multiply every score, so they join the softmax
+// scale; v's multiplies O.
+ta_status launch_prefill_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+                             float v_descale, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nkv,
+                             float scale, int causal, cudaStream_t stream) {
+  constexpr int D = 128;
+  using L = PrefillLayout<D, true>;
+  if (B == 0 || Nq == 0) return TA_OK;
+  if (Nkv == 0) {
+    const size_t rows = static_cast<size_t>(B) * Hq * Nq;
+    const size_t n = rows * D;
+    empty_keys_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+        static_cast<__nv_bfloat16*>(o), lse, rows, D);
+    return cudaGetLastError() == cudaSuccess ? TA_OK : TA_ERR_CUDA;
+  }
+  CUtensorMap tq, tk, tv;
+  ta_status st;
+  if ((st = encode_u8_rows_3d(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
+  if ((st = encode_u8_rows_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_u8_rows_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
+  static int attr_done[64] = {0};
+  cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, false, true>, L::kAlloc, attr_done);
+  if (e != cudaSuccess) return fail(TA_ERR_CUDA, "fp8 prefill: shared-memory limit", e);
+  const float s = scale * q_descale * k_descale;
+  PrefillArgs a = {};
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nq = Nq;
+  a.Nkv = Nkv;
+  a.n_pairs = (Nq + 2 * kBM - 1) / (2 * kBM);
+  a.causal = causal;
+  a.scale = s;
+  a.scale_log2 = s * 1.4426950408889634f;
+  a.v_descale = v_descale;
+  a.status = device_status_ptr();
+  if (!a.status) return fail(TA_ERR_CUDA, "fp8 prefill: device status word");
+  const unsigned grid = static_cast<unsigned>(a.n_pairs) * static_cast<unsigned>(B * Hq);
+  prefill_fwd_kernel<D, false, true><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "fp8 prefill: launch", e);
 }
 
 ta_status launch_paged_prefill(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,

@@ -19,6 +19,10 @@ PFN_encodeTiled get_encode_tiled();
 // as zero.
 ta_status encode_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices);
 
+// The same for a one-byte-per-element array (FP8 codes) [slices, rows, d],
+// d = 128: 128-row x 128-column boxes (one 128-byte swizzle row per row).
+ta_status encode_u8_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices);
+
 // General bf16 tensor map (rank 2-5, 128-byte swizzle, zero fill out of
 // bounds); strides_bytes has rank - 1 entries.
 ta_status encode_bf16_tiled(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
@@ -58,6 +62,10 @@ bool make_decode_plan(int num_seqs, int Hq, int Hkv, int d, int max_pages, int p
 
 ta_status launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                          int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);
+
+ta_status launch_prefill_fp8(const void* q, const void* k, const void* v, float q_descale, float k_descale,
+                             float v_descale, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nkv,
+                             float scale, int causal, cudaStream_t stream);
 
 ta_status launch_paged_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
                               const int32_t* seq_lens, int page_size, int num_seqs, int Hq, int Hkv, int d,
