@@ -56,10 +56,14 @@ constexpr int kRegsSoftmax = 224;    // warpgroups 1-2 after setmaxnreg.inc
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
 static_assert(kRegsControl + 2 * kRegsSoftmax <= 512, "per sub-partition: one warp of each warpgroup");
 constexpr float kRescaleLog2 = 8.0f;   // skip O rescale while max grew by <= 2^8
-// Column pairs whose index i has bit (i % 8) set in kPolyMask compute 2^x on
-// the FMA pipe (exp2_poly2) instead of the MUFU unit.  Moving 1/8 to 4/8 of
-// them there was measured: none was faster on B200, so all stay on MUFU.
+// Column pairs whose index i has bit (i % 8) set in the mask compute 2^x on
+// the FMA pipe (exp2_poly2) instead of the MUFU unit.  bf16: moving 1/8 to 4/8
+// of them there was measured, none was faster on B200, so all stay on MUFU.
+// fp8: the products take half the tensor cycles and MUFU limits more; 3/8
+// (pairs 0, 2, 5 of every 8) measured fastest, +6.5% and +6.7% on two boxes
+// (1/8: +4%, 2/8: +5%, 4/8: +2%).
 constexpr unsigned kPolyMask = 0x00u;
+constexpr unsigned kPolyMaskFp8 = 0x25u;
 
 template <int D, bool kFp8 = false>
 struct PrefillLayout {
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c = h * 64 + 2 * i;
           const float2 x = ffma2(make_float2(s[c], s[c + 1]), c2v, negv);
           float2 pp;
-          if ((kPolyMask >> (i & 7)) & 1u) {
+          if (((kFp8 ? kPolyMaskFp8 : kPolyMask) >> (i & 7)) & 1u) {
             pp = exp2_poly2(x);
           } else {
             pp.x = ex2(x.x);
