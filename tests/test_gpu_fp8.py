@@ -138,3 +138,41 @@ def test_fp8_deterministic(torch_cuda):
     a = run_fp8(torch_cuda, q8, k8, v8, desc, True)
     b = run_fp8(torch_cuda, q8, k8, v8, desc, True)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_fp8_all_codes(torch_cuda):
+    """Q, K and V codes drawn uniformly from every finite E4M3 code (subnormals
+    and +-448 included), descaled to |x| <= 1: the tensor cores must read the
+    whole format as the oracle's decoder does."""
+    rng = np.random.Generator(np.random.PCG64(77))
+    finite = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    B, Hq, Hkv, Nq, Nkv = 1, 2, 1, 300, 300
+    q8 = rng.choice(finite, size=(B, Hq, Nq, 128))
+    k8 = rng.choice(finite, size=(B, Hkv, Nkv, 128))
+    v8 = rng.choice(finite, size=(B, Hkv, Nkv, 128))
+    desc = (1 / 448, 1 / 448, 1 / 448)
+    for causal in (True, False):
+        o, lse = run_fp8(torch_cuda, q8, k8, v8, desc, causal)
+        o_ref, lse_ref = oracle.attn_fp8(q8, k8, v8, desc, causal)
+        fp8_bar(o, o_ref, lse, lse_ref, 1.0, f"fp8 all codes causal={causal}")
+
+
+def test_fp8_rising_scores_exact(torch_cuda):
+    """Integer scores that rise along the keys (0, 1, ..., 15 in steps every 32
+    keys), so the running max grows tile by tile: weights reach 2^8 against a
+    stale max before the O rescale.  With scale ln 2 every weight is a power of
+    two and exact in E4M3, so the bf16 bar applies."""
+    B, H, N = 1, 1, 512
+    one = inputs.f32_to_e4m3_bits(np.array([1.0], dtype=np.float32))[0]
+    q8 = np.zeros((B, H, N, 128), dtype=np.uint8)
+    q8[..., 0] = one
+    k8 = np.zeros((B, H, N, 128), dtype=np.uint8)
+    k8[0, 0, :, 0] = inputs.f32_to_e4m3_bits((np.arange(N) // 32).astype(np.float32))
+    rng = np.random.Generator(np.random.PCG64(78))
+    v8, dv = inputs.quantize_e4m3(rng.standard_normal(N * 128).astype(np.float32))
+    v8 = v8.reshape(B, H, N, 128)
+    desc = (1.0, 1.0, dv)
+    for causal in (False, True):
+        o, lse = run_fp8(torch_cuda, q8, k8, v8, desc, causal, math.log(2.0))
+        o_ref, lse_ref = oracle.attn_fp8(q8, k8, v8, desc, causal, scale=math.log(2.0))
+        parity(o, o_ref, lse, lse_ref, f"fp8 rising scores causal={causal}")
