@@ -37,7 +37,8 @@ def parity(o_gpu, o_ref, lse_gpu=None, lse_ref=None, what=""):
         lr = np.asarray(lse_ref, dtype=np.float64)
         both = np.isneginf(lg) & np.isneginf(lr)
         assert np.array_equal(np.isneginf(lg), np.isneginf(lr)), f"{what}: -inf lse pattern differs"
-        d = np.abs(np.where(both, 0.0, lg - lr))
+        with np.errstate(invalid="ignore"):     # -inf - -inf on rows with no key; masked by `both`
+            d = np.abs(np.where(both, 0.0, lg - lr))
         lse_err = float(d.max()) if d.size else 0.0
     assert max_abs <= MAX_ABS, f"{what}: max-abs {max_abs:.3e} > {MAX_ABS}"
     assert rel <= REL_L2 or denom == 0, f"{what}: rel-L2 {rel:.3e} > {REL_L2}"

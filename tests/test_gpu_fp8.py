@@ -59,7 +59,8 @@ def fp8_bar(o, o_ref, lse, lse_ref, vmax, what):
     rel = float(np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref))
     both = np.isneginf(lse) & np.isneginf(lse_ref)
     assert np.array_equal(np.isneginf(lse), np.isneginf(lse_ref)), f"{what}: -inf lse pattern differs"
-    lerr = float(np.abs(np.where(both, 0.0, lse - lse_ref)).max())
+    with np.errstate(invalid="ignore"):
+        lerr = float(np.abs(np.where(both, 0.0, lse - lse_ref)).max())
     bound = vmax / 16 + np.abs(o_ref).max() / 256
     assert np.all(np.isfinite(o)), f"{what}: non-finite output"
     assert max_abs <= bound, f"{what}: max-abs {max_abs:.3e} > {bound:.3e}"
