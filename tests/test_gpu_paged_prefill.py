@@ -49,6 +49,7 @@ CASES = [
     ([200, 77], [333, 77], 8, 2, 128, 32),                             # GQA group 4
     ([64, 512], [64, 700], 2, 1, 64, 64),                              # d = 64, 64-token pages
     ([300], [200], 2, 2, 128, 16),                                     # more queries than keys: masked rows
+    ([300, 5, 700], [300, 900, 1200], 6, 2, 128, 16),                  # GQA group 3: consecutive-tile pairs
 ]
 
 

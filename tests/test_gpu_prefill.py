@@ -46,6 +46,8 @@ CASES = [
     (1, 2, 2, 200, 333, 128, False),
     (2, 8, 2, 384, 384, 128, True),       # GQA group 4
     (1, 4, 1, 130, 130, 64, True),        # GQA group 4, d = 64, ragged
+    (1, 4, 2, 700, 900, 128, True),       # GQA group 2: head-paired tiles, Nq < Nkv
+    (1, 6, 2, 333, 333, 128, True),       # GQA group 3: consecutive-tile pairs
     (1, 1, 1, 1, 700, 128, False),        # one query row
     (1, 1, 1, 1, 700, 128, True),
     (1, 1, 1, 513, 129, 128, False),

@@ -95,7 +95,8 @@ struct PrefillArgs {
   __nv_bfloat16* o;
   float* lse;
   int B, Hq, Hkv, Nq, Nkv;
-  int n_pairs;       // ceil(Nq / 256)
+  int n_units;       // work units along the queries: ceil(Nq / 256) pairs, or ceil(Nq / 128) tiles (head_pair)
+  int head_pair;     // 1: a CTA takes one 128-row tile of two query heads sharing a KV head (GQA, even group)
   int causal;
   float scale;       // natural-log scale (for lse)
   float scale_log2;  // scale * log2(e)
@@ -150,14 +151,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: heavy (late) query pairs first so causal tails are short.
-  // Dense: (pair, batch, head).  Paged: (pair, sequence, head), with the
+  // ---- work item: heavy (late) query units first so causal tails are short.
+  // A CTA's two 128-row query tiles are two consecutive tiles of one head, or
+  // (head_pair) the same tile of two query heads of one GQA group: both then
+  // read the same K/V stream and have the same number of K/V tiles, so the
+  // two softmax warpgroups always have equal work.
+  // Dense: (unit, batch, head[s]).  Paged: (unit, sequence, head[s]), with the
   // sequence's query and key counts read (and range-checked) here.
-  const int bh_count = (kPaged ? a.num_seqs : a.B) * a.Hq;
-  const int pair = a.n_pairs - 1 - static_cast<int>(blockIdx.x) / bh_count;
+  const int heads_per_item = a.head_pair ? 2 : 1;
+  const int hx_count = a.Hq / heads_per_item;
+  const int bh_count = (kPaged ? a.num_seqs : a.B) * hx_count;
+  const int unit = a.n_units - 1 - static_cast<int>(blockIdx.x) / bh_count;
   const int bh = static_cast<int>(blockIdx.x) % bh_count;
-  const int b = bh / a.Hq, hq = bh % a.Hq;   // b = sequence when paged
-  const int hkv = hq / (a.Hq / a.Hkv);
+  const int b = bh / hx_count;                             // b = sequence when paged
+  const int hq_0 = (bh % hx_count) * heads_per_item;      // query head of tile 0
+  const int hq_1 = hq_0 + heads_per_item - 1;             // query head of tile 1
+  const int hkv = hq_0 / (a.Hq / a.Hkv);
   int Nq = a.Nq, Nkv = a.Nkv;
   int q_base = 0;                  // packed row of the sequence's first query (paged)
   if constexpr (kPaged) {
@@ -169,13 +178,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     lo = min(max(lo, 0), a.total_q);
     hi = min(max(hi, lo), min(a.total_q, lo + a.max_q_len));
     len = min(max(len, 0), a.max_pages * a.page_size);
-    if (bad && threadIdx.x == 0 && pair == 0 && hq == 0) atomicOr(a.status, bad);
+    if (bad && threadIdx.x == 0 && unit == 0 && hq_0 == 0) atomicOr(a.status, bad);
     q_base = lo;
     Nq = hi - lo;
     Nkv = len;
   }
-  const int q0_0 = pair * 2 * kBM, q0_1 = q0_0 + kBM;
-  if (kPaged && q0_0 >= Nq) return;   // this sequence has fewer query pairs (uniform per CTA)
+  const int q0_0 = a.head_pair ? unit * kBM : unit * 2 * kBM;
+  const int q0_1 = a.head_pair ? q0_0 : q0_0 + kBM;
+  if (kPaged && q0_0 >= Nq) return;   // this sequence has fewer query units (uniform per CTA)
   const int nt_0 = kv_tiles_for(q0_0, Nq, Nkv, a.causal), nt_1 = kv_tiles_for(q0_1, Nq, Nkv, a.causal);
   const int n_max = max(nt_0, nt_1);
 
@@ -215,18 +225,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     setmaxnreg_dec<kRegsControl>();
     if (warp == 0 && lane == 0) {
     // ======================= TMA producer =======================
-      const int zq = b * a.Hq + hq, zk = b * a.Hkv + hkv;
+      const int zk = b * a.Hkv + hkv;
       const uint32_t qbytes = static_cast<uint32_t>((q0_0 < Nq) + (q0_1 < Nq)) * L::kTileBytes;
       mbar_arrive_expect_tx(BAR_Q(), qbytes);
       for (int t = 0; t < 2; ++t) {
         const int q0 = t ? q0_1 : q0_0;
+        const int hq = t ? hq_1 : hq_0;
         if (q0 >= Nq) continue;
         for (int c = 0; c < L::kChunks; ++c) {
           if constexpr (kPaged)   // packed [total_q, Hq, d]: box of 128 rows of one head
             tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, hq,
                         q_base + q0);
           else
-            tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, q0, zq);
+            tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, q0,
+                        b * a.Hq + hq);
         }
       }
       // Physical pages of K/V tile j (paged): the table entries are read
@@ -390,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;                       // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;                // row within the tile
     const int q0 = t ? q0_1 : q0_0;                     // first query row of the tile
+    const int hq = t ? hq_1 : hq_0;                     // query head of the tile
     const int qrow = q0 + row;                          // query index
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + (t == 0 ? L::kTmS0 : L::kTmS1) + lane_off;
@@ -580,6 +593,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Work units: with an even number of query heads per KV head, a CTA takes one
+// 128-row tile of two heads of a group (equal work for both softmax
+// warpgroups, no half-empty last pair); otherwise two consecutive tiles of one
+// head.  max_q is Nq (dense) or the longest query chunk (paged).
+static void set_units(PrefillArgs& a, int Hq, int Hkv, int max_q) {
+  a.head_pair = ((Hq / Hkv) % 2 == 0) ? 1 : 0;
+  a.n_units = a.head_pair ? (max_q + kBM - 1) / kBM : (max_q + 2 * kBM - 1) / (2 * kBM);
+}
+
 // Output for shapes with no keys at all: O = 0, lse = -inf.
 __global__ void empty_keys_kernel(__nv_bfloat16* o, float* lse, size_t rows, int d) {
   const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
@@ -610,14 +632,14 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   a.Hkv = Hkv;
   a.Nq = Nq;
   a.Nkv = Nkv;
-  a.n_pairs = (Nq + 2 * kBM - 1) / (2 * kBM);
+  set_units(a, Hq, Hkv, Nq);
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.v_descale = 1.f;
   a.status = device_status_ptr();
   if (!a.status) return fail(TA_ERR_CUDA, "prefill: device status word");
-  const unsigned grid = static_cast<unsigned>(a.n_pairs) * static_cast<unsigned>(B * Hq);
+  const unsigned grid = static_cast<unsigned>(a.n_units) * static_cast<unsigned>(B * Hq / (a.head_pair + 1));
   prefill_fwd_kernel<D, false, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "prefill: launch", e);
@@ -656,7 +678,7 @@ static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, cons
   a.B = 1;
   a.Hq = Hq;
   a.Hkv = Hkv;
-  a.n_pairs = (max_q_len + 2 * kBM - 1) / (2 * kBM);
+  set_units(a, Hq, Hkv, max_q_len);
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
@@ -672,7 +694,7 @@ static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, cons
   a.page_size = page_size;
   a.max_pages = max_pages;
   a.num_pages_total = num_pages_total;
-  const unsigned grid = static_cast<unsigned>(a.n_pairs) * static_cast<unsigned>(num_seqs * Hq);
+  const unsigned grid = static_cast<unsigned>(a.n_units) * static_cast<unsigned>(num_seqs * Hq / (a.head_pair + 1));
   prefill_fwd_kernel<D, true, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "paged prefill: launch", e);
@@ -711,14 +733,14 @@ ta_status launch_prefill_fp8(const void* q, const void* k, const void* v, float 
   a.Hkv = Hkv;
   a.Nq = Nq;
   a.Nkv = Nkv;
-  a.n_pairs = (Nq + 2 * kBM - 1) / (2 * kBM);
+  set_units(a, Hq, Hkv, Nq);
   a.causal = causal;
   a.scale = s;
   a.scale_log2 = s * 1.4426950408889634f;
   a.v_descale = v_descale;
   a.status = device_status_ptr();
   if (!a.status) return fail(TA_ERR_CUDA, "fp8 prefill: device status word");
-  const unsigned grid = static_cast<unsigned>(a.n_pairs) * static_cast<unsigned>(B * Hq);
+  const unsigned grid = static_cast<unsigned>(a.n_units) * static_cast<unsigned>(B * Hq / (a.head_pair + 1));
   prefill_fwd_kernel<D, false, true><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "fp8 prefill: launch", e);
