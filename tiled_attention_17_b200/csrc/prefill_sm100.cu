@@ -6,9 +6,9 @@
 // (Gemini 3 Flash kernel-fusion post, sections 1-3; FlashAttention
 // optimisation article, sections 3.1-3.2 and 7.1).
 //
-// CTA = two 128-row query tiles of one (batch, query head) sharing one K/V
-// stream.  The kernel has two instantiations: dense [B, H, N, d] tensors, and
-// (kPaged) varlen query rows of several sequences packed as [total_q, Hq, d]
+// CTA = two 128-row query tiles sharing one K/V stream (two tiles of one head,
+// or one tile of two GQA heads).  Instantiations: dense [B, H, N, d] bf16; FP8
+// (kFp8) E4M3 inputs; (kPaged) varlen query rows packed as [total_q, Hq, d]
 // against K/V gathered page by page from a paged cache through a block table
 // (chunked prefill, LLM-inference article section 3.2; PagedAttention,
 // GPU-optimisation tag page).  Warp roles (384 threads, three warpgroups):
