@@ -1,0 +1,54 @@
+"""Host logic of bench.py's roofline reporting (CPU only): the DRAM traffic it
+reports comes from a committed ncu capture and only while the captured
+kernel's source is unchanged."""
+import json
+import os
+
+import pytest
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def _records():
+    with open(TRAFFIC) as f:
+        return {k: v for k, v in json.load(f).items() if not k.startswith("_")}
+
+
+@pytest.mark.parametrize("kernel", sorted(_records()))
+def test_traffic_record_is_complete(kernel):
+    rec = _records()[kernel]
+    assert os.path.exists(os.path.join(ROOT, "tiled_attention_17_b200", "csrc", rec["source_file"]))
+    assert rec["dram_bytes_per_unit"] > 0
+    capture = os.path.join(ROOT, rec["capture"])
+    assert os.path.exists(capture), f"{kernel}: capture summary {rec['capture']} missing"
+    # the summary states the command it came from
+    assert "ncu " in open(capture).read()
+
+
+@pytest.mark.parametrize("kernel", sorted(_records()))
+def test_traffic_reported_only_for_the_captured_source(kernel):
+    """A record is reported (scaled by the units) while its kernel source is the
+    one it was captured from, and as null once that source has changed."""
+    rec = _records()[kernel]
+    got = bench.recorded_traffic(kernel, rec["source_file"], 2.0)
+    if rec["source_sha256_16"] == bench.kernel_source_hash(rec["source_file"]):
+        assert got == pytest.approx(2.0 * rec["dram_bytes_per_unit"])
+    else:
+        assert got is None
+
+
+def test_stale_or_missing_record_reports_null(monkeypatch):
+    rec = _records()["prefill_fwd_kernel"]
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda fname: "0" * 16)
+    assert bench.recorded_traffic("prefill_fwd_kernel", rec["source_file"], 1.0) is None
+    monkeypatch.undo()
+    assert bench.recorded_traffic("no_such_kernel", rec["source_file"], 1.0) is None
+
+
+def test_roofline_fraction():
+    r = bench.roofline("tensor", 830.0, 1660.0, "TFLOP/s", None)
+    assert r == {"bound": "tensor", "achieved": 830.0, "peak": 1660.0, "unit": "TFLOP/s", "frac": 0.5,
+                 "traffic": None}
