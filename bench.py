@@ -199,6 +199,18 @@ def prefill_sample_rows(stride: int, shift: int = 0):
     return rows, flops
 
 
+def host_cpu_model() -> str:
+    """The host CPU's model name (first 'model name' line of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_oracle_sample(q, k, v, stride: int):
     import oracle
     rows, flops = prefill_sample_rows(stride)
@@ -206,6 +218,7 @@ def cpu_oracle_sample(q, k, v, stride: int):
     oracle.attn(q, k, v, True, scale=PREFILL.scale, rows=rows)
     dt = time.perf_counter() - t0
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "cpu_model": host_cpu_model(), "hardware_threads": os.cpu_count(),
             "sample": f"fp64 oracle on every {stride}th query row of all {PREFILL.B}x{PREFILL.Hq} heads of the "
                       f"causal prefill workload ({rows.size} rows, {flops / 1e9:.1f} GFLOP, {dt:.1f} s)"}
 
@@ -238,6 +251,7 @@ def run_reference(args):
         "config": {"workload": "causal prefill B=4 Hq=Hkv=16 N=4096 d=128 bf16 (bounded row sample per step)",
                    "parallelism": "host cores"},
         "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "cpu_model": host_cpu_model(), "hardware_threads": os.cpu_count(),
                          "sample": f"every {stride}th query row per step ({len(rows)} rows)"},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

@@ -52,3 +52,13 @@ def test_roofline_fraction():
     r = bench.roofline("tensor", 830.0, 1660.0, "TFLOP/s", None)
     assert r == {"bound": "tensor", "achieved": 830.0, "peak": 1660.0, "unit": "TFLOP/s", "frac": 0.5,
                  "traffic": None}
+
+
+def test_cpu_baseline_sample_runs_on_host():
+    """The CPU-baseline leg (the oracle on a row sample of the causal workload)
+    runs on the host alone and states its cores and CPU model."""
+    from tiled_attention_17_b200 import inputs
+    q, k, v = inputs.prefill_inputs(bench.PREFILL)
+    cpu = bench.cpu_oracle_sample(q, k, v, 2048)
+    assert cpu["kind"] == "oracle" and cpu["value"] > 0 and cpu["cores"] >= 1
+    assert cpu["cpu_model"] and cpu["hardware_threads"] >= 1
