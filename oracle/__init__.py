@@ -13,7 +13,6 @@ from __future__ import annotations
 
 import ctypes
 import math
-import os
 
 import numpy as np
 

@@ -3,7 +3,6 @@ timing, distinct per-rank inputs, and the reference arm running on rank 0 only."
 import os
 import socket
 
-import pytest
 import torch.multiprocessing as mp
 
 
@@ -55,7 +54,6 @@ def test_reference_arm_only_rank0_prints(monkeypatch, capsys):
 
 
 def test_sample_rows_cover_all_depths():
-    import numpy as np
     import bench
     rows, flops = bench.prefill_sample_rows(4)
     c = bench.PREFILL
