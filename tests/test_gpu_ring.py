@@ -25,13 +25,14 @@ def torch_cuda():
 @pytest.mark.parametrize("B,Hq,Hkv,N,d,shards", [(1, 4, 2, 1024, 128, 4), (2, 2, 2, 900, 128, 3),
                                                  (1, 8, 2, 512, 64, 2)])
 @pytest.mark.parametrize("causal", [True, False])
-def test_ring_emulated_matches_whole_sequence(torch_cuda, B, Hq, Hkv, N, d, shards, causal):
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+def test_ring_emulated_matches_whole_sequence(torch_cuda, B, Hq, Hkv, N, d, shards, causal, layout):
     from tiled_attention_17_b200 import ring
     q, k, v = random_prefill(B, Hq, Hkv, N, N, d, seed=N + shards)
-    o, lse = ring.ring_attention_emulated(to_dev(q), to_dev(k), to_dev(v), shards, causal)
+    o, lse = ring.ring_attention_emulated(to_dev(q), to_dev(k), to_dev(v), shards, causal, layout=layout)
     torch_cuda.cuda.synchronize()
     o_ref, lse_ref = oracle.attn(q, k, v, causal)
-    parity(bf16_to_f64(o), o_ref, lse.cpu().numpy(), lse_ref, f"ring {B, Hq, Hkv, N, d, shards, causal}")
+    parity(bf16_to_f64(o), o_ref, lse.cpu().numpy(), lse_ref, f"ring {layout} {B, Hq, Hkv, N, d, shards, causal}")
 
 
 def test_merge_of_key_halves(torch_cuda):

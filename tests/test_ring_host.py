@@ -148,3 +148,24 @@ def test_hop_masks():
     from tiled_attention_17_b200.ring import hop_mask
     assert hop_mask(2, 1, True) == "full" and hop_mask(2, 2, True) == "causal" and hop_mask(2, 3, True) is None
     assert all(hop_mask(r, s, False) == "full" for r in range(3) for s in range(3))
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+@pytest.mark.parametrize("shards", [2, 3, 4])
+@pytest.mark.parametrize("causal", [True, False])
+def test_emulated_ring_schedule(layout, shards, causal):
+    """The one-process emulation of the ring (the form the GPU tests run with the
+    CUDA kernels), here with the oracle per hop and an fp64 merge: the
+    reassembled output equals whole-sequence attention."""
+    import torch
+    import oracle
+    from tiled_attention_17_b200 import ring
+    from tiled_attention_17_b200.inputs import random_prefill
+    N = 6 * shards
+    q, k, v = random_prefill(1, 4, 2, N, N, 3, seed=60 + shards)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16))
+    o, lse = ring.ring_attention_emulated(t(q), t(k), t(v), shards, causal, scale=0.8, layout=layout,
+                                          attend=_oracle_attend, accumulator=_Fp64Accumulator)
+    o_ref, lse_ref = oracle.attn(q, k, v, causal, scale=0.8)
+    assert np.allclose(o, o_ref, rtol=0, atol=1e-12)
+    assert np.allclose(lse, lse_ref, rtol=0, atol=1e-12)

@@ -213,32 +213,62 @@ def _ring_attention_zigzag(q, k, v, causal, scale, group, attend, accumulator):
     return np.concatenate([o0, o1], axis=2), np.concatenate([l0, l1], axis=2)
 
 
-def ring_attention_emulated(q, k, v, shards: int, causal: bool, scale: float | None = None):
+def ring_attention_emulated(q, k, v, shards: int, causal: bool, scale: float | None = None,
+                            layout: str = "contiguous", attend=None, accumulator=None):
     """The ring schedule of `ring_attention` for `shards` virtual ranks in one
-    process (no communication): shard r of q attends to the K/V shards in the
-    order rank r would receive them.  Returns the full-sequence (o, lse).
-    For checking the per-hop masks and the merge kernels on one GPU."""
+    process (no communication): each virtual rank's queries attend to the K/V
+    shards in the order that rank would receive them.  Returns the
+    full-sequence (o, lse) in sequence order.  For checking the per-hop masks
+    and the merge kernels on one GPU; `attend` and `accumulator` default to the
+    CUDA kernels (other implementations exercise the schedule on the CPU)."""
     import torch
     B, Hq, N, d = q.shape
-    if N % shards:
-        raise ValueError("sequence length must divide into the shards")
-    n = N // shards
+    attend = attend or _cuda_attend
+    acc_cls = accumulator or _CudaAccumulator
     if scale is None:
         scale = d ** -0.5
-    outs, lses = [], []
+    cat = lambda xs, dim: (torch.cat(xs, dim=dim) if isinstance(xs[0], torch.Tensor)
+                           else __import__("numpy").concatenate(xs, axis=dim))
+    if layout == "contiguous":
+        if N % shards:
+            raise ValueError("sequence length must divide into the shards")
+        n = N // shards
+        outs, lses = [], []
+        for r in range(shards):
+            qr = q[:, :, r * n:(r + 1) * n].contiguous()
+            acc = acc_cls(qr)
+            for h in range(shards):
+                src = (r - h) % shards
+                mode = hop_mask(r, src, causal)
+                if mode is None:
+                    continue
+                ks = k[:, :, src * n:(src + 1) * n].contiguous()
+                vs = v[:, :, src * n:(src + 1) * n].contiguous()
+                o_part, lse_part = attend(qr, ks, vs, mode == "causal", scale)
+                acc.merge(o_part, lse_part)
+            o, lse = acc.finish()
+            outs.append(o)
+            lses.append(lse)
+        return cat(outs, 2), cat(lses, 2)
+    if layout != "zigzag":
+        raise ValueError(f"unknown layout {layout!r}")
+    if N % (2 * shards):
+        raise ValueError("sequence length must divide into 2 * shards chunks")
+    c = N // (2 * shards)
+    chunk = lambda t, ch: t[:, :, ch * c:(ch + 1) * c].contiguous()
+    by_chunk = {}
     for r in range(shards):
-        qr = q[:, :, r * n:(r + 1) * n].contiguous()
-        acc = _CudaAccumulator(qr)
-        for h in range(shards):
-            src = (r - h) % shards
-            mode = hop_mask(r, src, causal)
-            if mode is None:
-                continue
-            ks = k[:, :, src * n:(src + 1) * n].contiguous()
-            vs = v[:, :, src * n:(src + 1) * n].contiguous()
-            o_part, lse_part = _cuda_attend(qr, ks, vs, mode == "causal", scale)
-            acc.merge(o_part, lse_part)
-        o, lse = acc.finish()
-        outs.append(o)
-        lses.append(lse)
-    return torch.cat(outs, dim=2), torch.cat(lses, dim=2)
+        for qc in zigzag_chunks(r, shards):
+            qs = chunk(q, qc)
+            acc = acc_cls(qs)
+            for h in range(shards):
+                src = (r - h) % shards
+                for kc in zigzag_chunks(src, shards):
+                    mode = chunk_mask(qc, kc, causal)
+                    if mode is None:
+                        continue
+                    o_part, lse_part = attend(qs, chunk(k, kc), chunk(v, kc), mode == "causal", scale)
+                    acc.merge(o_part, lse_part)
+            by_chunk[qc] = acc.finish()
+    order = range(2 * shards)
+    return cat([by_chunk[i][0] for i in order], 2), cat([by_chunk[i][1] for i in order], 2)
