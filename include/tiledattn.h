@@ -13,9 +13,10 @@
  * article, sections 2.1 and 3.1-3.2.
  *
  * Conventions shared by every call
- *  - All Q/K/V/O arrays are bfloat16, dense, row-major, with 16-byte aligned
- *    base pointers (128-byte alignment recommended; FlashAttention article 5.2,
- *    kernel-fusion post "data layout").  lse arrays are float32.
+ *  - All Q/K/V/O arrays are bfloat16 (attn_fwd_fp8: Q/K/V as E4M3 codes),
+ *    dense, row-major, with 16-byte aligned base pointers (128-byte alignment
+ *    recommended; FlashAttention article 5.2, kernel-fusion post "data
+ *    layout").  lse arrays are float32.
  *  - Pointers are DEVICE pointers unless stated otherwise.  The caller owns
  *    every buffer and the stream.  No call allocates memory or synchronises;
  *    work is enqueued on `stream` and the call returns.

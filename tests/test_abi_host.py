@@ -227,3 +227,38 @@ def test_merge_validation(lib):
     assert fin(a, a, 16, 96) == "TA_ERR_UNSUPPORTED"
     assert fin(a, a + 4, 16, 128) == "TA_ERR_INVALID_ARG"
     assert fin(a, a, 0, 128) == "TA_OK"
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/tiledattn.h compiles as C11 with warnings as errors, and a C
+    program linked against libtiledattn.so reaches the host-side paths (no GPU
+    needed: argument checks return before any CUDA call)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    from tiled_attention_17_b200 import build as libbuild
+    lib = libbuild.build()
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "consumer.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "tiledattn.h"
+int main(void) {
+    void *p = (void *)(size_t)256;   /* aligned, never dereferenced: rejected first */
+    if (attn_fwd(p, p, p, p, NULL, 1, 3, 2, 128, 128, 128, 0.1f, 0, NULL) != TA_ERR_INVALID_ARG) return 1;
+    if (attn_fwd_fp8(p, p, p, 1.f, 1.f, 1.f, p, NULL, 1, 1, 1, 128, 128, 64, 0.1f, 1, NULL) != TA_ERR_UNSUPPORTED)
+        return 2;
+    if (attn_bwd_workspace_size(1, 1, 1) == 0) return 3;
+    if (strcmp(ta_status_string(TA_OK), "TA_OK") != 0) return 4;
+    printf("version %d\n", ta_version());
+    return ta_version() > 0 ? 0 : 5;
+}
+""")
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(lib)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                    str(src), "-o", str(exe), f"-L{libdir}", "-ltiledattn", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stderr)
