@@ -211,7 +211,11 @@ ta_status attn_bwd(const void *q, const void *k, const void *v, const void *o, c
 
 /*
  * Bytes of device workspace attn_paged_decode needs for these sizes (256-byte
- * aligned).  Pure host arithmetic; returns 0 for invalid sizes.
+ * aligned); returns 0 for invalid sizes.  Host arithmetic on the sizes and the
+ * current device's SM count (the split plan aims at 8 CTAs per SM; 148 is
+ * assumed when no device can be queried), so query it with the device
+ * current that the decode call will run on.  Hkv, which the pages' call
+ * sketch leaves out, fixes the number of CTAs per split and so the plan.
  */
 size_t attn_paged_decode_workspace_size(int num_seqs, int Hq, int Hkv, int d,
                                         int max_pages, int page_size);
@@ -262,11 +266,15 @@ ta_status attn_paged_decode(const void *q, const void *k_cache, const void *v_ca
  * every GPU that loads the library's code holds it until the process exits).
  * The call allocates nothing.  Sizes whose attn_paged_decode_workspace_size
  * exceeds 64 MiB return TA_ERR_UNSUPPORTED before anything is enqueued (the
- * reason is in ta_last_error).  The first call on each device looks up the
- * scratch array's device address (with that device current) and caches it;
- * make that first call before any stream capture.  Every call on a device
- * shares the one array: calls that may overlap on the GPU (different streams,
- * no ordering between them) race and give wrong results; serialise them.  The
+ * reason is in ta_last_error).  The first call in each CUDA context (on each
+ * device, with that device current) looks up the scratch array's device
+ * address and caches it under the context's unique id; make that first call
+ * before any stream capture.  A context created later (for example after
+ * cudaDeviceReset, or a non-primary context the caller makes current) gets
+ * its own lookup on its first call, so no stale address is used.  Every call
+ * on a device shares the one array: calls that may overlap on the GPU
+ * (different streams, no ordering between them) race and give wrong results;
+ * serialise them.  The
  * status word that attn_paged_decode_check reads lives in that shared array
  * and is not exposed for this entry point; bad table entries and lengths are
  * still clamped on the device.
@@ -286,12 +294,14 @@ ta_status attn_paged_decode_noalloc(const void *q, const void *k_cache, const vo
 ta_status attn_paged_decode_check(const void *workspace, unsigned *flags, ta_stream_t stream);
 
 /*
- * Test/diagnostic export: writes the logical K and V rows of (seq, hkv),
- * gathered through the block table by the same device gather routine that
- * attn_paged_decode uses, to k_out/v_out [max_pages * page_size, d] bf16
- * (rows >= seq_lens[seq] are left untouched).  Same layouts and limits as
- * attn_paged_decode; bad entries are clamped and flagged in the library status
- * word (ta_device_status).
+ * Test/diagnostic export: writes the logical K and V rows of (seq, hkv) to
+ * k_out/v_out [max_pages * page_size, d] bf16 (rows >= seq_lens[seq] are left
+ * untouched).  The rows are gathered split by split and chunk by chunk with
+ * the device functions both attn_paged_decode split kernels use: the split's
+ * block-table entries staged in shared memory, then one bulk copy per
+ * (page, KV head) of each 64-token chunk.  Same layouts and limits as
+ * attn_paged_decode; an entry outside the pool reads physical page 0 and is
+ * flagged in the library status word (ta_device_status), as in decode.
  */
 ta_status attn_paged_gather_debug(const void *k_cache, const void *v_cache,
                                   const int32_t *block_table, const int32_t *seq_lens,

@@ -85,27 +85,75 @@ def test_decode_long_split_merge(torch_cuda):
     check_decode(torch_cuda, inp, "long split merge")
 
 
-def test_gather_bit_exact(torch_cuda):
+GATHER_CASES = [
+    # page_size, d, lens: partial last pages, lengths that span several splits
+    # (a split is 1024 tokens, 64 pages at page 8) and the split boundaries
+    (8, 128, [1, 37, 513, 1030]),
+    (16, 128, [1, 37, 1024, 1025, 3000]),
+    (32, 128, [31, 33, 2100]),
+    (64, 128, [70, 1, 4097]),
+    (8, 64, [5, 200, 600]),
+    (64, 64, [130]),
+]
+
+
+@pytest.mark.parametrize("ps,d,lens", GATHER_CASES)
+def test_gather_bit_exact(torch_cuda, ps, d, lens):
+    """The gathered logical K/V rows equal the oracle's explicitly gathered rows
+    bit for bit.  attn_paged_gather_debug runs the decode kernels' own
+    split-table load and chunk copies (both decode split kernels use them)."""
     torch = torch_cuda
     from tiled_attention_17_b200 import binding
-    for ps, d, lens in [(16, 128, [1, 37, 1030]), (8, 64, [5, 200]), (64, 128, [70, 1])]:
-        inp = small_paged(len(lens), 4, 2, d, ps, lens, seed=ps + d)
-        q, kc, vc, bt, sl = to_dev_paged(torch, inp)
-        max_pages = inp.block_table.shape[1]
-        for s in range(len(lens)):
-            for h in range(2):
-                ko = torch.zeros((max_pages * ps, d), dtype=torch.bfloat16, device="cuda")
-                vo = torch.zeros_like(ko)
-                binding.attn_paged_gather_debug(kc, vc, bt, sl, s, h, ps, 2, d, max_pages,
-                                                inp.k_cache.shape[0], ko, vo)
-                torch.cuda.synchronize()
-                kr, vr = oracle.paged_gather(inp.k_cache, inp.v_cache, inp.block_table, inp.seq_lens, s, h)
-                L = lens[s]
-                kg = ko[:L].cpu().view(torch.int16).numpy().view(np.uint16)
-                vg = vo[:L].cpu().view(torch.int16).numpy().view(np.uint16)
-                assert np.array_equal(kg, kr) and np.array_equal(vg, vr), (ps, d, s, h)
+    Hkv = 2
+    inp = small_paged(len(lens), 4 * Hkv, Hkv, d, ps, lens, seed=ps + d + len(lens))
+    q, kc, vc, bt, sl = to_dev_paged(torch, inp)
+    max_pages = inp.block_table.shape[1]
+    binding.ta_device_status(reset=True)
+    for s in range(len(lens)):
+        for h in range(Hkv):
+            ko = torch.zeros((max_pages * ps, d), dtype=torch.bfloat16, device="cuda")
+            vo = torch.zeros_like(ko)
+            binding.attn_paged_gather_debug(kc, vc, bt, sl, s, h, ps, Hkv, d, max_pages,
+                                            inp.k_cache.shape[0], ko, vo)
+            torch.cuda.synchronize()
+            kr, vr = oracle.paged_gather(inp.k_cache, inp.v_cache, inp.block_table, inp.seq_lens, s, h)
+            L = lens[s]
+            kg = ko[:L].cpu().view(torch.int16).numpy().view(np.uint16)
+            vg = vo[:L].cpu().view(torch.int16).numpy().view(np.uint16)
+            assert np.array_equal(kg, kr) and np.array_equal(vg, vr), (ps, d, s, h)
+            # rows past the sequence are never written
+            assert torch.all(ko[L:] == 0) and torch.all(vo[L:] == 0)
     code, flags = binding.ta_device_status(reset=True)
     assert code == 0 and flags == 0
+
+
+@pytest.mark.parametrize("ps", [8, 16, 32, 64])
+def test_gather_bad_entry_clamped_bit_exact(torch_cuda, ps):
+    """A table entry outside the pool is never dereferenced: its page reads as
+    physical page 0 (bit-exact against the oracle's gather through the same
+    table with that entry replaced by 0) and the status word is flagged."""
+    torch = torch_cuda
+    from tiled_attention_17_b200 import binding
+    d, Hkv, L = 128, 2, 5 * ps + 3
+    inp = small_paged(1, 8, Hkv, d, ps, [L], seed=40 + ps)
+    bad = inp.block_table.copy()
+    bad[0, 2] = inp.num_pages_total + 11
+    fixed = bad.copy()
+    fixed[0, 2] = 0
+    kc, vc = to_dev(inp.k_cache), to_dev(inp.v_cache)
+    bt, sl = torch.from_numpy(bad).cuda(), torch.from_numpy(inp.seq_lens).cuda()
+    max_pages = bad.shape[1]
+    binding.ta_device_status(reset=True)
+    for h in range(Hkv):
+        ko = torch.zeros((max_pages * ps, d), dtype=torch.bfloat16, device="cuda")
+        vo = torch.zeros_like(ko)
+        binding.attn_paged_gather_debug(kc, vc, bt, sl, 0, h, ps, Hkv, d, max_pages, inp.num_pages_total, ko, vo)
+        torch.cuda.synchronize()
+        kr, vr = oracle.paged_gather(inp.k_cache, inp.v_cache, fixed, inp.seq_lens, 0, h)
+        assert np.array_equal(ko[:L].cpu().view(torch.int16).numpy().view(np.uint16), kr)
+        assert np.array_equal(vo[:L].cpu().view(torch.int16).numpy().view(np.uint16), vr)
+    code, flags = binding.ta_device_status(reset=True)
+    assert binding.STATUS_NAMES[code] == "TA_ERR_BAD_BLOCK_TABLE" and flags & binding.TA_DEV_BAD_BLOCK_TABLE
 
 
 def test_decode_cross_entry_identity_table(torch_cuda):

@@ -8,8 +8,9 @@
 //   2.1  a CTA stages the scattered pages of its range into shared memory;
 //        here each (page, KV head) is one contiguous page_size*d*2-byte span,
 //        so one TMA bulk copy moves it and every byte read is used;
-//   2.3  the split's block-table entries are loaded into registers of the
-//        issuing warp before the gather loop (index prefetch);
+//   2.3  the split's block-table entries are loaded once, before the gather
+//        loop, into a shared-memory table that every copy reads (index
+//        prefetch);
 //   2.4  the gather is fused with the dot products q.k, the online softmax
 //        and the weighted sum of V; nothing gathered is written back.
 // Splits are merged by their log-sum-exp, which is exact because the online
@@ -43,6 +44,7 @@ constexpr int kRowsPerWarp = kChunkTokens / kConsumerWarps;
 constexpr int kSplitThreads = 32 * (kConsumerWarps + 1);   // + one TMA producer warp
 constexpr int kGatherThreads = 128;        // gather-debug kernel
 constexpr int kMaxG = 8;
+constexpr int kMaxSplitPages = 64;         // block-table entries one split stages
 
 template <int D>
 struct DecodeLayout {
@@ -61,7 +63,8 @@ struct DecodeLayout {
   static constexpr int kArea = kRing > kStates * kMaxG * (D + 2) * 4 ? kRing : kStates * kMaxG * (D + 2) * 4;
   static constexpr int kBar = kArea;                    // full[S], empty[S]
   static constexpr int kAbort = kBar + 2 * kDecStages * 8;
-  static constexpr int kBytes = kAbort + 16;
+  static constexpr int kTable = kAbort + 16;            // the split's block-table entries
+  static constexpr int kBytes = kTable + kMaxSplitPages * 4;
 };
 
 struct DecodeArgs {
@@ -83,42 +86,52 @@ __device__ __forceinline__ int clamp_len(int len, const DecodeArgs& a) {
   return len < 0 ? 0 : (len > cap ? cap : len);
 }
 
-// The page gather shared by decode and the gather-debug export.  Warp-wide:
-// every lane of the calling warp must call it.  Stages the `npg` pages
-// starting at split-local page `first` into dstK/dstV (consecutive, in page
-// order) and arms `bar` with their byte count.  tbl0/tbl1 hold the split's
-// prefetched block-table entries (entry i sits in lane i % 32, register i / 32).
-// Entries outside [0, num_pages_total) are replaced by page 0 and flagged.
+// ---------------------------------------------------------------------------
+// The page gather, shared by both split kernels and the gather-debug export
+// (so the export checks the addressing the decode kernels run).
+// ---------------------------------------------------------------------------
+// Index prefetch (paged gather article, section 2.3): the block-table entries
+// of one split's pages are loaded once into the shared-memory table `tbl` and
+// checked there; every copy of the split then reads its page id from the
+// table.  Entries outside [0, num_pages_total) are replaced by page 0 (never
+// dereferenced) and flagged.  Thread i of the caller's `count` participating
+// threads loads entries i, i + count, ...; the caller synchronises before the
+// table is read.
+__device__ __forceinline__ void load_split_table(const DecodeArgs& a, int seq, int split_first_page, int npages,
+                                                 int* tbl, int i0, int count) {
+  const int32_t* row = a.block_table + static_cast<size_t>(seq) * a.max_pages + split_first_page;
+  for (int i = i0; i < npages; i += count) {
+    int pg = __ldg(row + i);
+    if (pg < 0 || pg >= a.num_pages_total) {
+      atomicOr(a.status, kDevBadBlockTable);
+      pg = 0;
+    }
+    tbl[i] = pg;
+  }
+}
+
+// The copies of one chunk (paged gather article, section 2.1): pages
+// [first, first + npg) of the split's table, each (page, KV head) one
+// contiguous page_size * D * 2-byte span, land back to back in dstK / dstV
+// (so chunk row r is token r of the chunk); `bar` is armed with their byte
+// count.  Warp-wide: every lane of the calling warp must call it; lane i < npg
+// copies page first + i.
 template <int D>
-__device__ __forceinline__ void gather_pages(const DecodeArgs& a, int hkv, int first, int npg, int tbl0, int tbl1,
-                                             uint32_t dstK, uint32_t dstV, uint32_t bar, unsigned* flag_word) {
+__device__ __forceinline__ void gather_chunk(const DecodeArgs& a, int hkv, const int* tbl, int first, int npg,
+                                             uint32_t dstK, uint32_t dstV, uint32_t bar) {
   const int lane = threadIdx.x & 31;
   const uint32_t page_bytes = static_cast<uint32_t>(a.page_size) * D * 2;
   if (lane == 0) mbar_arrive_expect_tx(bar, 2u * npg * page_bytes);
   __syncwarp();
-  const int idx = first + lane;
-  const int v0 = __shfl_sync(0xffffffffu, tbl0, idx & 31);
-  const int v1 = __shfl_sync(0xffffffffu, tbl1, idx & 31);
   if (lane < npg) {
-    int pg = (idx < 32) ? v0 : v1;
-    if (pg < 0 || pg >= a.num_pages_total) {
-      atomicOr(flag_word, kDevBadBlockTable);
-      pg = 0;
-    }
-    const size_t off = (static_cast<size_t>(pg) * a.Hkv + hkv) * page_bytes;
+    const size_t off = (static_cast<size_t>(tbl[first + lane]) * a.Hkv + hkv) * page_bytes;
     bulk_load(dstK + lane * page_bytes, a.k_cache + off, page_bytes, bar);
     bulk_load(dstV + lane * page_bytes, a.v_cache + off, page_bytes, bar);
   }
 }
 
-// Loads the block-table entries of pages [first_page, first_page + npages)
-// of `seq` into two registers per lane (index prefetch).
-__device__ __forceinline__ void prefetch_table(const DecodeArgs& a, int seq, int first_page, int npages, int& tbl0,
-                                               int& tbl1) {
-  const int lane = threadIdx.x & 31;
-  const int32_t* row = a.block_table + static_cast<size_t>(seq) * a.max_pages + first_page;
-  tbl0 = lane < npages ? __ldg(row + lane) : -1;
-  tbl1 = lane + 32 < npages ? __ldg(row + lane + 32) : -1;
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
@@ -217,8 +230,9 @@ __global__ void __launch_bounds__(kSplitThreads, (G <= 4 ? 2 : 1)) decode_split_
 
   if (warp == kConsumerWarps) {
     // ======================= producer warp =======================
-    int tbl0, tbl1;
-    prefetch_table(a, seq, split_first_page, split_npages, tbl0, tbl1);   // index prefetch
+    int* tbl = reinterpret_cast<int*>(smem + L::kTable);
+    load_split_table(a, seq, split_first_page, split_npages, tbl, lane, 32);   // index prefetch
+    __syncwarp();
     int c = 0;
     for (; c < n_chunks; ++c) {
       const int stage = c % kDecStages;
@@ -227,7 +241,7 @@ __global__ void __launch_bounds__(kSplitThreads, (G <= 4 ? 2 : 1)) decode_split_
       const int first = c * pages_per_chunk;
       const int npg = min(pages_per_chunk, split_npages - first);
       const uint32_t st = sbase + stage * L::kStageBytes;
-      gather_pages<D>(a, hkv, first, npg, tbl0, tbl1, st, st + L::kChunkBytes, FULL(stage), a.status);
+      gather_chunk<D>(a, hkv, tbl, first, npg, st, st + L::kChunkBytes, FULL(stage));
     }
     // drain: no copy into this CTA's shared memory may be in flight at exit
     if (lane == 0)
@@ -380,7 +394,7 @@ struct G4Layout {
   static constexpr int kMerge = kStates * 4 * (D + 2) * 4;       // 33 KB, reuses the ring
   static constexpr int kProb = kRing;                            // [8 warps][2 seg][16] floats
   static constexpr int kTable = kProb + kG4Warps * 2 * 16 * 4;   // split's block-table entries
-  static constexpr int kBar = kTable + 64 * 4;                   // full[3]
+  static constexpr int kBar = kTable + kMaxSplitPages * 4;       // full[3]
   static constexpr int kCnt = kBar + kDecStages * 8;             // per-stage finish counters
   static constexpr int kMisc = kCnt + kDecStages * 4;            // abort flag, issued-chunk count
   static constexpr int kBytes = kMisc + 16;
@@ -391,25 +405,6 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel_shared(uint32_t addr, uint3
   uint32_t old;
   asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
   return old;
-}
-
-__device__ __forceinline__ void fence_proxy_async_shared() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Page copies for one chunk, page ids read from the shared-memory table.
-// Warp-wide; lane i < npg copies page i of the chunk.
-__device__ __forceinline__ void gather_chunk_g4(const DecodeArgs& a, int hkv, const int* tbl, int first, int npg,
-                                                uint32_t dstK, uint32_t dstV, uint32_t bar) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t page_bytes = static_cast<uint32_t>(a.page_size) * G4Layout::kRowBytes;
-  if (lane == 0) mbar_arrive_expect_tx(bar, 2u * npg * page_bytes);
-  __syncwarp();
-  if (lane < npg) {
-    const size_t off = (static_cast<size_t>(tbl[first + lane]) * a.Hkv + hkv) * page_bytes;
-    bulk_load(dstK + lane * page_bytes, a.k_cache + off, page_bytes, bar);
-    bulk_load(dstV + lane * page_bytes, a.v_cache + off, page_bytes, bar);
-  }
 }
 
 __global__ void __launch_bounds__(kG4Threads, 2) decode_split_g4_kernel(const DecodeArgs a) {
@@ -450,19 +445,12 @@ __global__ void __launch_bounds__(kG4Threads, 2) decode_split_g4_kernel(const De
     *issued = min(kDecStages, n_chunks);
     fence_mbar_init();
   }
-  if (tid < split_npages) {
-    int pg = __ldg(a.block_table + static_cast<size_t>(seq) * a.max_pages + split_first_page + tid);
-    if (pg < 0 || pg >= a.num_pages_total) {
-      atomicOr(a.status, kDevBadBlockTable);
-      pg = 0;
-    }
-    tbl[tid] = pg;
-  }
+  load_split_table(a, seq, split_first_page, split_npages, tbl, tid, kG4Threads);
   __syncthreads();
   if (warp < kDecStages && warp < n_chunks) {
     const int first = warp * pages_per_chunk;
     const uint32_t st = sbase + warp * L::kStageBytes;
-    gather_chunk_g4(a, hkv, tbl, first, min(pages_per_chunk, split_npages - first), st, st + L::kChunkBytes,
+    gather_chunk<D>(a, hkv, tbl, first, min(pages_per_chunk, split_npages - first), st, st + L::kChunkBytes,
                     FULL(warp));
   }
 
@@ -604,7 +592,7 @@ __global__ void __launch_bounds__(kG4Threads, 2) decode_split_g4_kernel(const De
         fence_proxy_async_shared();   // generic reads of the stage before the async copies into it
         const int first = cn * pages_per_chunk;
         const uint32_t st = sbase + stage * L::kStageBytes;
-        gather_chunk_g4(a, hkv, tbl, first, min(pages_per_chunk, split_npages - first), st, st + L::kChunkBytes,
+        gather_chunk<D>(a, hkv, tbl, first, min(pages_per_chunk, split_npages - first), st, st + L::kChunkBytes,
                         FULL(stage));
         if (lane == 0) atomicMax(issued, cn + 1);
       }
@@ -686,38 +674,51 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeArgs a,
   if (col == 0 && lse) lse[orow] = mx + __logf(tot);
 }
 
-// Gather-debug: same gather routine, result written out contiguously.
+// Gather-debug: the sequence's pages gathered split by split and chunk by
+// chunk with the decode kernels' own table load and chunk copies, then written
+// out contiguously.
 template <int D>
 __global__ void __launch_bounds__(kGatherThreads) gather_debug_kernel(const DecodeArgs a, int seq, int hkv,
                                                                    __nv_bfloat16* k_out, __nv_bfloat16* v_out) {
   using L = DecodeLayout<D>;
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar = sbase + L::kBar;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  int* tbl = reinterpret_cast<int*>(smem + L::kTable);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int len = clamp_len(__ldg(a.seq_lens + seq), a);
+  const int raw_len = __ldg(a.seq_lens + seq);
+  const int len = clamp_len(raw_len, a);
   if (tid == 0) {
+    if (raw_len != len) atomicOr(a.status, kDevBadSeqLen);
     mbar_init(bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
   const int pages_per_chunk = kChunkTokens / a.page_size;
-  const int npages = (len + a.page_size - 1) / a.page_size;
+  const int split_tokens = a.split_pages * a.page_size;
   int phase = 0;
-  for (int g0 = 0; g0 < npages; g0 += 64) {       // table prefetch covers 64 pages
-    const int gn = min(64, npages - g0);
-    int tbl0 = -1, tbl1 = -1;
-    if (warp == 0) prefetch_table(a, seq, g0, gn, tbl0, tbl1);
-    for (int first = 0; first < gn; first += pages_per_chunk) {
-      const int npg = min(pages_per_chunk, gn - first);
-      if (warp == 0)
-        gather_pages<D>(a, hkv, first, npg, tbl0, tbl1, sbase, sbase + L::kChunkBytes, bar, a.status);
+  for (int t_begin = 0, split = 0; t_begin < len; t_begin += split_tokens, ++split) {
+    const int t_end = min(len, t_begin + split_tokens);
+    const int split_npages = (t_end - t_begin + a.page_size - 1) / a.page_size;
+    load_split_table(a, seq, split * a.split_pages, split_npages, tbl, tid, kGatherThreads);
+    __syncthreads();
+    for (int first = 0; first < split_npages; first += pages_per_chunk) {
+      const int npg = min(pages_per_chunk, split_npages - first);
+      if (warp == 0) {
+        fence_proxy_async_shared();   // earlier generic reads of the staging area before the async copies
+        gather_chunk<D>(a, hkv, tbl, first, npg, sbase, sbase + L::kChunkBytes, bar);
+      }
       const bool ok = mbar_wait(bar, phase & 1u, a.status, abort_flag);
       phase++;
-      if (__syncthreads_or(!ok)) return;
-      const int t0 = (g0 + first) * a.page_size;
+      if (__syncthreads_or(!ok)) {
+        // a wait gave up: let the copies in flight land before leaving
+        if (tid == 0) mbar_wait(bar, (phase - 1) & 1u, nullptr, nullptr, kWaitLimitNs);
+        __syncthreads();
+        return;
+      }
+      const int t0 = t_begin + first * a.page_size;
       const int rows = min(npg * a.page_size, len - t0);
       const int words = rows * D / 8;   // 16-byte words
       for (int w = tid; w < words; w += kGatherThreads) {
@@ -828,8 +829,10 @@ ta_status launch_gather_debug(const void* k_cache, const void* v_cache, const in
                               int max_pages, int num_pages_total, void* k_out, void* v_out, cudaStream_t stream) {
   unsigned* status = device_status_ptr();
   if (!status) return TA_ERR_CUDA;
+  // splits as the decode plan forms them for a batch that fills the GPU
+  const int split_pages = (1024 / page_size < kMaxSplitPages) ? 1024 / page_size : kMaxSplitPages;
   DecodeArgs a = make_args(nullptr, k_cache, v_cache, block_table, seq_lens, page_size, seq + 1, Hkv, Hkv, max_pages,
-                           num_pages_total, 1.f, 64, 1, nullptr, nullptr, status);
+                           num_pages_total, 1.f, split_pages, 1, nullptr, nullptr, status);
   static int done128[64] = {0}, done64[64] = {0};
   if (d == 128) {
     if (ensure_smem_limit(gather_debug_kernel<128>, DecodeLayout<128>::kBytes, done128) != cudaSuccess)
@@ -852,13 +855,26 @@ ta_status launch_selftest_wait(unsigned limit_us, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? TA_OK : TA_ERR_CUDA;
 }
 
+// SMs of the current device; 148 (B200) when no device can be queried, so a
+// size query made without a GPU still gets the plan a B200 would use.
+static int current_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0) {
+    cudaGetLastError();   // clear the non-sticky error of the failed query
+    return 148;
+  }
+  return n;
+}
+
 bool make_decode_plan(int num_seqs, int Hq, int Hkv, int d, int max_pages, int page_size, DecodePlan* plan) {
   if (page_size != 8 && page_size != 16 && page_size != 32 && page_size != 64) return false;
   if (num_seqs < 0 || Hq <= 0 || Hkv <= 0 || max_pages <= 0 || (d != 64 && d != 128)) return false;
   const int chunk_pages = kChunkTokens / page_size;
   int sp = 1024 / page_size;
-  if (sp > 64) sp = 64;                 // the table prefetch holds 64 entries per split
-  const long long target = 8LL * 148;   // enough CTAs to balance uneven lengths
+  if (sp > kMaxSplitPages) sp = kMaxSplitPages;   // the split's table holds 64 entries
+  // enough CTAs to balance uneven lengths: 8 per SM of the current device
+  const long long target = 8LL * current_sm_count();
   auto splits_for = [&](int p) { return (max_pages + p - 1) / p; };
   while (sp > chunk_pages && static_cast<long long>(num_seqs) * Hkv * splits_for(sp) < target) sp /= 2;
   if (sp < chunk_pages) sp = chunk_pages;
