@@ -22,18 +22,56 @@ static_assert(kDevTimeout == TA_DEV_TIMEOUT && kDevBadBlockTable == TA_DEV_BAD_B
 // the library is loaded on).  Bits: TA_DEV_*.
 __device__ unsigned g_status_word;
 
-unsigned* device_status_ptr() {
-  static unsigned* ptrs[64] = {nullptr};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> g(mu);
-  if (!ptrs[dev]) {
+using PFN_ctxGetCurrent = CUresult (*)(CUcontext*);
+using PFN_ctxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+bool current_context_id(unsigned long long* id) {
+  static PFN_ctxGetCurrent get_current = nullptr;
+  static PFN_ctxGetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<unsigned*>(p);
-  }
-  return ptrs[dev];
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_ctxGetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_ctxGetId>(p);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+bool ContextAddressCache::find(unsigned long long ctx, void** out) {
+  std::lock_guard<std::mutex> g(mu_);
+  for (int i = 0; i < kSlots; ++i)
+    if (ptrs_[i] && ids_[i] == ctx) {
+      *out = ptrs_[i];
+      return true;
+    }
+  return false;
+}
+
+void ContextAddressCache::insert(unsigned long long ctx, void* p) {
+  std::lock_guard<std::mutex> g(mu_);
+  ids_[next_] = ctx;
+  ptrs_[next_] = p;
+  next_ = (next_ + 1) % kSlots;
+}
+
+unsigned* device_status_ptr() {
+  static ContextAddressCache cache;
+  unsigned long long ctx = 0;
+  void* p = nullptr;
+  if (current_context_id(&ctx) && cache.find(ctx, &p)) return static_cast<unsigned*>(p);
+  if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess || p == nullptr) return nullptr;
+  // the lookup made the device's primary context current if none was
+  if (current_context_id(&ctx)) cache.insert(ctx, p);
+  return static_cast<unsigned*>(p);
 }
 
 PFN_encodeTiled get_encode_tiled() {

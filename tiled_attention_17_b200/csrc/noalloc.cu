@@ -10,14 +10,13 @@
 //
 // The scratch is one file-scope __device__ array of kNoAllocScratchBytes.  In
 // host code the array's name is only a host-side stand-in, so its device
-// address is looked up with cudaGetSymbolAddress, once per device with that
-// device current, and cached.  The call then forwards to attn_paged_decode
-// with that address as the workspace, so the kernels, validation and launch
-// path are exactly those of attn_paged_decode.
+// address is looked up with cudaGetSymbolAddress once per CUDA context (on
+// each device, with that device current) and cached.  The call then forwards
+// to attn_paged_decode with that address as the workspace, so the kernels,
+// validation and launch path are exactly those of attn_paged_decode.
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 
 #include "tiledattn_internal.h"
 
@@ -29,24 +28,24 @@ constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;   // 64 MiB
 // word until the next call overwrites them.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of the scratch array on the current device (looked up on the
-// first call per device, with that device current).
+// Device address of the scratch array in the calling thread's current
+// context.  The host-side name g_noalloc_scratch is only a stand-in, so the
+// address is looked up with cudaGetSymbolAddress, with the device (and the
+// context that will run the kernels) current, on the first call in each
+// context, and cached under that context's unique identifier.  A context
+// created later (after cudaDeviceReset, or one the caller makes current) gets
+// a lookup of its own, never a stale address.
 static ta_status noalloc_scratch(void** out) {
-  static void* ptrs[64] = {nullptr};
-  static std::mutex mu;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail(TA_ERR_CUDA, "attn_paged_decode_noalloc: cudaGetDevice", e);
-  if (dev < 0 || dev >= 64) return fail(TA_ERR_UNSUPPORTED, "attn_paged_decode_noalloc: device index >= 64");
-  std::lock_guard<std::mutex> g(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return fail(TA_ERR_CUDA, "attn_paged_decode_noalloc: cudaGetSymbolAddress of the scratch array", e);
-    ptrs[dev] = p;
-  }
-  *out = ptrs[dev];
+  static ContextAddressCache cache;
+  unsigned long long ctx = 0;
+  if (current_context_id(&ctx) && cache.find(ctx, out)) return TA_OK;
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr)
+    return fail(TA_ERR_CUDA, "attn_paged_decode_noalloc: cudaGetSymbolAddress of the scratch array", e);
+  // the lookup made the device's primary context current if none was
+  if (current_context_id(&ctx)) cache.insert(ctx, p);
+  *out = p;
   return TA_OK;
 }
 

@@ -5,6 +5,8 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "tiledattn.h"
 
 namespace ta {
@@ -33,8 +35,31 @@ ta_status encode_bf16_tiled(CUtensorMap* map, const void* base, int rank, const 
 ta_status fail(ta_status code, const char* where, cudaError_t err = cudaSuccess);
 ta_status fail_cu(ta_status code, const char* where, int cu_result);
 
-// Device address of the library status word on the current device.
+// Device address of the library status word in the current context.
 unsigned* device_status_ptr();
+
+// Unique identifier (cuCtxGetId) of the CUDA context current on the calling
+// thread.  Identifiers are never reused within a process, so a cache keyed by
+// one never serves an address from a context that was destroyed (for example
+// by cudaDeviceReset).  Returns false if no context is current or the driver
+// entry points are unavailable.
+bool current_context_id(unsigned long long* id);
+
+// Small per-context cache of device addresses of __device__ variables (their
+// host-side names are only stand-ins; the address comes from
+// cudaGetSymbolAddress in the context that will use it).
+class ContextAddressCache {
+ public:
+  bool find(unsigned long long ctx, void** out);
+  void insert(unsigned long long ctx, void* p);
+
+ private:
+  static constexpr int kSlots = 16;
+  std::mutex mu_;
+  unsigned long long ids_[kSlots] = {};
+  void* ptrs_[kSlots] = {};
+  int next_ = 0;
+};
 
 // Raise a kernel's dynamic shared-memory limit once per device.
 // `done` is the caller's per-kernel, per-device record.
