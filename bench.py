@@ -7,10 +7,13 @@ One step = one pass of the whole hot path over one batch of synthetic input:
     16-token pages, lengths uniform on [512, 32768] (attn_paged_decode + combine).
 The headline metric is the prefill's TFLOP/s (visible (q, k) pairs, both
 contractions, 2 flop per multiply-add); the decode's KV GB/s is reported in
-the same line under "decode"; the backward pass (attn_bwd on the prefill
-workload) and a varlen chunked prefill over the paged cache
-(attn_paged_prefill) are timed on their own after the step and reported under
-"backward" and "paged_prefill".  Inputs are
+the same line under "decode".  Timed on their own after the step: the other
+two prefill workloads (long: N=16384 non-causal with sharp key peaks; gqa:
+Hq=32 over Hkv=8, N=8192 causal) under "long" and "gqa", the backward pass
+(attn_bwd on the prefill workload) under "backward", a varlen chunked prefill
+over the paged cache (attn_paged_prefill) under "paged_prefill" and the FP8
+prefill under "fp8_prefill".  The CPU-baseline leg also compares the step's
+prefill output with the oracle on every row ("parity").  Inputs are
 resident in HBM when timing starts;
 L2 (126 MB) is flushed by writing a 256 MB buffer before every step, outside
 the kernels' event brackets.  Kernel times are CUDA events on the launching
@@ -211,16 +214,40 @@ def host_cpu_model() -> str:
     return "unknown"
 
 
-def cpu_oracle_sample(q, k, v, stride: int):
+def parity_metrics(o_gpu, o_ref, lse_gpu, lse_ref) -> dict:
+    """Max-abs and relative L2 error of O and max absolute lse error over the
+    rows given (the parity bar: 2e-2, 5e-3, 1e-3)."""
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    lg = np.asarray(lse_gpu, dtype=np.float64)
+    lr = np.asarray(lse_ref, dtype=np.float64)
+    both = np.isneginf(lg) & np.isneginf(lr)
+    with np.errstate(invalid="ignore"):
+        lse_err = float(np.abs(np.where(both, 0.0, lg - lr)).max())
+    max_abs = float(np.abs(o_gpu - o_ref).max())
+    rel = float(np.linalg.norm(o_gpu - o_ref) / np.linalg.norm(o_ref))
+    return {"max_abs": max_abs, "rel_l2": rel, "lse_abs": lse_err,
+            "pass": bool(max_abs <= 2e-2 and rel <= 5e-3 and lse_err <= 1e-3)}
+
+
+def cpu_oracle_sample(q, k, v, stride: int, o_gpu=None, lse_gpu=None):
+    """The oracle on every `stride`-th row of the causal workload, timed on the
+    host cores; with the GPU's output of the same rows given, also the parity
+    of that output against the oracle's (over all rows when stride is 1)."""
     import oracle
     rows, flops = prefill_sample_rows(stride)
     t0 = time.perf_counter()
-    oracle.attn(q, k, v, True, scale=PREFILL.scale, rows=rows)
+    o_ref, lse_ref = oracle.attn(q, k, v, True, scale=PREFILL.scale, rows=rows)
     dt = time.perf_counter() - t0
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "cpu_model": host_cpu_model(), "hardware_threads": os.cpu_count(),
-            "sample": f"fp64 oracle on every {stride}th query row of all {PREFILL.B}x{PREFILL.Hq} heads of the "
-                      f"causal prefill workload ({rows.size} rows, {flops / 1e9:.1f} GFLOP, {dt:.1f} s)"}
+    out = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+           "cpu_model": host_cpu_model(), "hardware_threads": os.cpu_count(),
+           "sample": f"fp64 oracle on every {stride}th query row of all {PREFILL.B}x{PREFILL.Hq} heads of the "
+                     f"causal prefill workload ({rows.size} rows, {flops / 1e9:.1f} GFLOP, {dt:.1f} s)"}
+    if o_gpu is not None:
+        par = parity_metrics(o_gpu.reshape(-1, PREFILL.d)[rows], o_ref, lse_gpu.reshape(-1)[rows], lse_ref)
+        par["rows"] = f"{rows.size} of {PREFILL.B * PREFILL.Hq * PREFILL.Nq}"
+        out["parity"] = par
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -365,9 +392,19 @@ def run_ours(args):
     if not args.no_fp8:
         fp8 = run_fp8_prefill(args, torch, binding, dev, stream, flush, dist, rank, world, peaks)
 
+    # ---- the other two prefill workloads (timed on their own, after the step)
+    legs = {}
+    if not args.no_prefill_legs:
+        for name in ("long", "gqa"):
+            legs[name] = run_prefill_leg(args, torch, binding, dev, stream, flush, dist, rank, world, peaks, name)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_sample(q_h, k_h, v_h, args.cpu_stride)
+        # the step's output (every step writes the same o and lse) against the
+        # oracle on the same rows
+        o_step = o.float().cpu().numpy()
+        lse_step = lse.cpu().numpy()
+        cpu = cpu_oracle_sample(q_h, k_h, v_h, args.cpu_stride, o_step, lse_step)
 
     if rank == 0:
         pre_per_gpu = pre_flops / (t_pre * 1e-3) / 1e12
@@ -388,6 +425,8 @@ def run_ours(args):
                                             recorded_traffic("decode_split_g4_kernel", "decode_paged.cu",
                                                              float(dinp.seq_lens.sum()))),
                        "e2e": dec_e2e},
+            "long": legs.get("long"),
+            "gqa": legs.get("gqa"),
             "backward": bwd,
             "paged_prefill": paged,
             "fp8_prefill": fp8,
@@ -399,12 +438,58 @@ def run_ours(args):
             "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "parity": cpu.get("parity") if cpu else None,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def run_prefill_leg(args, torch, binding, dev, stream, flush, dist, rank, world, peaks, name):
+    """attn_fwd on another prefill workload (long: B=1, H=8, N=16384,
+    non-causal, every 64th key row x4; gqa: B=2, Hq=32, Hkv=8, N=8192,
+    causal): CUDA events around each call, L2 flushed before every call, max
+    over ranks."""
+    c = inputs.PREFILL_CONFIGS[name]
+    q_h, k_h, v_h = inputs.prefill_inputs(c, seed=rank_seed(inputs.CONFIG_SEEDS[name], rank))
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = bf(q_h), bf(k_h), bf(v_h)
+    del q_h, k_h, v_h
+    o = torch.empty_like(q)
+    lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+
+    def call():
+        binding.attn_fwd(q, k, v, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nkv, c.d, c.scale, int(c.causal), stream)
+
+    for _ in range(3):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(dist, dev.index)
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+    (t,) = max_over_ranks([t], dist, device=dev)
+    flops = accounting.prefill_flops(c.B, c.Hq, c.Nq, c.Nkv, c.d, c.causal)
+    per_gpu = flops / (t * 1e-3) / 1e12
+    workload = (f"B={c.B} Hq={c.Hq} Hkv={c.Hkv} N={c.Nq} d={c.d} {'causal' if c.causal else 'non-causal'}"
+                + (f", key rows j%{c.peak_rows_every}==0 x{c.peak_factor:g}" if c.peak_rows_every else ""))
+    return {"value": per_gpu * world, "unit": "TFLOP/s", "ms": t, "steps": steps, "workload": workload,
+            "flops_per_call_per_gpu": flops, "gpu_launches_per_call": 1,
+            "roofline": roofline("tensor", per_gpu, peaks["bf16_tflops"], "TFLOP/s",
+                                 recorded_traffic(f"prefill_fwd_kernel_{name}", "prefill_sm100.cu",
+                                                  float(c.B * c.Hq)))}
 
 
 PAGED_MIX = dict(num_seqs=32, q_lo=1, q_hi=2048, prefix_lo=0, prefix_hi=8192, Hq=32, Hkv=8, d=128, page_size=16)
@@ -636,7 +721,8 @@ def timed(torch, stream, fn, steps):
 
 def run_ncu_case(args):
     """A small, self-contained case for a profiler capture of one kernel:
-    prefill = the causal workload (about 270 MB on the device); decode = 16
+    prefill = the causal workload (about 270 MB on the device); long and gqa =
+    those prefill workloads (about 135 and 340 MB); decode = 16
     sequences with the benchmark's length distribution (about 1.1 GB, larger
     than L2).  Runs `--reps` launches and exits."""
     import torch
@@ -675,14 +761,14 @@ def run_ncu_case(args):
         o, lse = binding.attention(q, k, v, True, c.scale)
         for _ in range(args.reps):
             binding.attention_backward(q, k, v, o, lse, dout, True, c.scale)
-    elif args.ncu_case == "prefill":
-        c = PREFILL
+    elif args.ncu_case in ("prefill", "long", "gqa"):
+        c = PREFILL if args.ncu_case == "prefill" else inputs.PREFILL_CONFIGS[args.ncu_case]
         q_h, k_h, v_h = inputs.prefill_inputs(c)
         q, k, v = dev_bf16(q_h), dev_bf16(k_h), dev_bf16(v_h)
         o = torch.empty_like(q)
         lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
         for _ in range(args.reps):
-            binding.attn_fwd(q, k, v, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nkv, c.d, c.scale, 1)
+            binding.attn_fwd(q, k, v, o, lse, c.B, c.Hq, c.Hkv, c.Nq, c.Nkv, c.d, c.scale, int(c.causal))
     else:
         import dataclasses
         D = dataclasses.replace(DECODE, num_seqs=16)
@@ -712,7 +798,9 @@ def main(argv=None):
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-paged-prefill", action="store_true")
     ap.add_argument("--no-fp8", action="store_true")
-    ap.add_argument("--ncu-case", choices=["prefill", "decode", "backward", "paged", "fp8"], default=None,
+    ap.add_argument("--no-prefill-legs", action="store_true", help="skip the long and gqa prefill legs")
+    ap.add_argument("--ncu-case", choices=["prefill", "long", "gqa", "decode", "backward", "paged", "fp8"],
+                    default=None,
                     help="run a small single-kernel case for a profiler capture and exit")
     ap.add_argument("--reps", type=int, default=4)
     args = ap.parse_args(argv)

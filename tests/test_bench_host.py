@@ -62,3 +62,25 @@ def test_cpu_baseline_sample_runs_on_host():
     cpu = bench.cpu_oracle_sample(q, k, v, 2048)
     assert cpu["kind"] == "oracle" and cpu["value"] > 0 and cpu["cores"] >= 1
     assert cpu["cpu_model"] and cpu["hardware_threads"] >= 1
+
+
+def test_cpu_baseline_parity_compares_the_given_output():
+    """With the GPU's output given, the CPU-baseline leg reports the parity of
+    that output on the rows it evaluated: exact for the oracle's own values,
+    failing once one element is off by more than the max-abs bar."""
+    import numpy as np
+
+    import oracle
+    from tiled_attention_17_b200 import inputs
+    c = bench.PREFILL
+    q, k, v = inputs.prefill_inputs(c)
+    rows, _ = bench.prefill_sample_rows(2048)
+    o_ref, lse_ref = oracle.attn(q, k, v, True, scale=c.scale, rows=rows)
+    o_full = np.zeros((c.B * c.Hq * c.Nq, c.d))
+    lse_full = np.zeros(c.B * c.Hq * c.Nq)
+    o_full[rows], lse_full[rows] = o_ref, lse_ref
+    par = bench.cpu_oracle_sample(q, k, v, 2048, o_full, lse_full)["parity"]
+    assert par["pass"] and par["max_abs"] == 0.0 and par["lse_abs"] == 0.0
+    o_full[rows[5], 3] += 0.05
+    par = bench.cpu_oracle_sample(q, k, v, 2048, o_full, lse_full)["parity"]
+    assert not par["pass"] and abs(par["max_abs"] - 0.05) < 1e-9
