@@ -1,0 +1,95 @@
+"""The backward parity bar, checked against a model of the kernels' arithmetic (CPU).
+
+The backward kernels round to bfloat16 at three points: the probabilities P
+before dV = P^T dO, the score gradients dS = P o (dP - delta) before dK =
+scale dS^T Q and dQ = scale dS K, and the gradients themselves when stored;
+delta = rowsum(dO o O) uses the forward's bf16 output O.  Products accumulate
+in fp32, whose error is far below these roundings.  This file models exactly
+those rounding points in numpy (fp64 elsewhere) and compares with the exact
+fp64 oracle:
+
+* the modelled error is at the level of bf16 rounding (relative L2 about
+  2.5e-3, max error at most about 6e-3 of the largest gradient), and the GPU
+  bar (tests/test_gpu_backward.py: relative L2 <= 5e-3, max error <=
+  1.2e-2 of the largest gradient, the attention parity bar's 5e-3 for the
+  former) leaves about 2x headroom over it;
+* without the roundings the model equals the oracle, so the error it predicts
+  is the roundings' and nothing else.
+
+The model is test infrastructure: it shares nothing with the CUDA code and is
+not the oracle.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+from gpu_util import GRAD_MAX_REL, GRAD_REL_L2
+from tiled_attention_17_b200.inputs import bf16_bits_to_f32, f32_to_bf16_bits, grad_output, random_prefill
+
+
+def _bf16(x):
+    return bf16_bits_to_f32(f32_to_bf16_bits(np.asarray(x, dtype=np.float32))).astype(np.float64)
+
+
+def model_bwd(q, k, v, do, causal, scale, rnd=_bf16):
+    """Gradients with the kernels' rounding points (`rnd` applied there)."""
+    Q, K, V, dO = (bf16_bits_to_f32(x).astype(np.float64) for x in (q, k, v, do))
+    B, Hq, Nq, d = Q.shape
+    Hkv, Nkv = K.shape[1], K.shape[2]
+    G = Hq // Hkv
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    i, j = np.arange(Nq)[:, None], np.arange(Nkv)[None, :]
+    mask = (j <= i + (Nkv - Nq)) if causal else np.ones((Nq, Nkv), dtype=bool)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            S = np.where(mask, Q[b, h] @ K[b, hk].T * scale, -np.inf)
+            m = S.max(axis=1, keepdims=True)
+            seen = np.isfinite(m)
+            E = np.exp(S - np.where(seen, m, 0.0))
+            P = np.where(seen, E / np.where(seen, E.sum(axis=1, keepdims=True), 1.0), 0.0)
+            O = rnd(P @ V[b, hk])                               # forward output as stored
+            dP = dO[b, h] @ V[b, hk].T
+            dS = P * (dP - (dO[b, h] * O).sum(axis=1, keepdims=True))
+            dV[b, hk] += rnd(P).T @ dO[b, h]
+            dK[b, hk] += scale * rnd(dS).T @ Q[b, h]
+            dQ[b, h] = scale * rnd(dS) @ K[b, hk]
+    return rnd(dQ), rnd(dK), rnd(dV)
+
+
+def _errors(g, ref):
+    return (np.linalg.norm(g - ref) / np.linalg.norm(ref), np.abs(g - ref).max() / np.abs(ref).max())
+
+
+CASES = [
+    (1, 1, 1, 256, 256, 64, False),
+    (1, 2, 2, 640, 640, 128, True),
+    (1, 2, 2, 333, 200, 128, False),
+    (2, 8, 2, 384, 384, 128, True),      # GQA group 4
+    (1, 4, 1, 130, 130, 64, True),
+    (1, 1, 1, 1, 700, 128, False),       # one query row
+    (1, 2, 1, 300, 100, 128, True),      # rows with no visible key
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nkv,d,causal", CASES)
+def test_backward_bar_covers_modelled_error(B, Hq, Hkv, Nq, Nkv, d, causal):
+    q, k, v = random_prefill(B, Hq, Hkv, Nq, Nkv, d, seed=Nq * 5 + Nkv + d + causal)
+    do = grad_output(q.shape, seed=Nq + 17 * Nkv)
+    scale = d ** -0.5
+    ref = oracle.attn_bwd(q, k, v, do, causal, scale=scale)
+    for name, g, r in zip(("dq", "dk", "dv"), model_bwd(q, k, v, do, causal, scale), ref):
+        rel, mx = _errors(g, r)
+        assert 1e-3 < rel < GRAD_REL_L2 / 1.8, (name, rel)      # bf16 level, 1.8x under the bar
+        assert mx < GRAD_MAX_REL / 1.8, (name, mx)
+
+
+def test_model_without_roundings_is_exact():
+    q, k, v = random_prefill(1, 4, 2, 200, 260, 64, seed=7)
+    do = grad_output(q.shape, seed=8)
+    for causal in (False, True):
+        ref = oracle.attn_bwd(q, k, v, do, causal)
+        for g, r in zip(model_bwd(q, k, v, do, causal, 64 ** -0.5, rnd=lambda x: x), ref):
+            assert np.abs(g - r).max() <= 1e-10 * np.abs(r).max()
