@@ -45,14 +45,6 @@ def varlen_prefill_flops(q_lens, kv_lens, Hq: int, d: int, causal: bool) -> floa
     return 4.0 * Hq * d * sum(visible_pairs(int(a), int(b), causal) for a, b in zip(q_lens, kv_lens))
 
 
-def prefill_min_bytes(B: int, Hq: int, Hkv: int, Nq: int, Nkv: int, d: int, lse: bool = True) -> int:
-    """Q, K, V read once, O (and lse) written once, bf16 tensors."""
-    b = 2 * (B * Hq * Nq * d) * 2 + 2 * (B * Hkv * Nkv * d) * 2
-    if lse:
-        b += 4 * B * Hq * Nq
-    return b
-
-
 def decode_kv_bytes(seq_lens, Hkv: int, d: int) -> int:
     return int(np.asarray(seq_lens, dtype=np.int64).clip(min=0).sum()) * Hkv * d * 2 * 2
 

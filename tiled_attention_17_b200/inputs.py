@@ -310,23 +310,6 @@ def paged_inputs(cfg: DecodeConfig = DECODE_CONFIG, seed: int | None = None, wit
     return inp
 
 
-def gather_pages_for(inp: PagedInputs, seqs) -> dict:
-    """Regenerate only the pool pages that the given sequences use.
-
-    Returns {physical_slot: (k_page, v_page)} with pages shaped [Hkv, page, d].
-    """
-    out = {}
-    for s in seqs:
-        n = (int(inp.seq_lens[s]) + inp.cfg.page_size - 1) // inp.cfg.page_size
-        for slot in inp.block_table[s, :n]:
-            slot = int(slot)
-            if slot not in out:
-                k = pool_pages(inp.cfg, inp.seed, 1, slot, 1)[0]
-                v = pool_pages(inp.cfg, inp.seed, 2, slot, 1)[0]
-                out[slot] = (k, v)
-    return out
-
-
 # --------------------------------------------------------------------------
 # Varlen prefill over the paged cache
 # --------------------------------------------------------------------------
