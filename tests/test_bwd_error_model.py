@@ -93,3 +93,18 @@ def test_model_without_roundings_is_exact():
         ref = oracle.attn_bwd(q, k, v, do, causal)
         for g, r in zip(model_bwd(q, k, v, do, causal, 64 ** -0.5, rnd=lambda x: x), ref):
             assert np.abs(g - r).max() <= 1e-10 * np.abs(r).max()
+
+
+def test_backward_bar_covers_modelled_error_sharp_peaks():
+    """Every 64th key row x4 (the long workload's structure): the weights are more
+    peaked, dS concentrates on fewer keys and the modelled error grows to about
+    3.9e-3; the bar still sits above it (1.25x)."""
+    from tiled_attention_17_b200 import inputs
+    cfg = inputs.PrefillConfig("peaks", 1, 2, 2, 1024, 1024, 128, False, 64, 4.0)
+    q, k, v = inputs.prefill_inputs(cfg, seed=98)
+    do = grad_output(q.shape, seed=3)
+    ref = oracle.attn_bwd(q, k, v, do, False)
+    for name, g, r in zip(("dq", "dk", "dv"), model_bwd(q, k, v, do, False, 128 ** -0.5), ref):
+        rel, mx = _errors(g, r)
+        assert 1e-3 < rel < GRAD_REL_L2 / 1.25, (name, rel)
+        assert mx < GRAD_MAX_REL / 2, (name, mx)
