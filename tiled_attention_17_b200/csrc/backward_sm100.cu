@@ -22,8 +22,9 @@
 // of 5) but needs no atomics, so the gradients are deterministic.
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator and
-// single-thread tcgen05.mma issuer, warps 4-11 two warpgroups for the
-// elementwise work and the epilogue: thread (h, row) owns one tile row's
+// tcgen05.mma issuer (the whole warp runs the loop, one elected lane
+// issues), warps 4-11 two warpgroups for the elementwise work and the
+// epilogue: thread (h, row) owns one tile row's
 // columns [64h, 64h + 64).  The elementwise steps need no row reduction (the
 // row statistics come precomputed), so the two halves never exchange data;
 // each writes its bf16 result over the TMEM columns it read, and the
@@ -77,12 +78,13 @@ struct BwdArgs {
 
 // K-major operand tile (128 rows x D, 128-byte swizzle): descriptor of the
 // tile, +2 per 16-element step inside a 64-column chunk, +chunk to the next.
-__device__ __forceinline__ void mma_kmajor_tile(uint32_t d_tmem, uint64_t a0, uint64_t b0, int chunks,
+__device__ __forceinline__ void mma_kmajor_tile(bool leader, uint32_t d_tmem, uint64_t a0, uint64_t b0, int chunks,
                                                 uint32_t idesc, bool acc) {
 #pragma unroll 1
   for (int c = 0; c < chunks; ++c) {
 #pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) mma_ss(d_tmem, a0 + 2 * k4, b0 + 2 * k4, idesc, (acc || (c | k4) != 0));
+    for (int k4 = 0; k4 < 4; ++k4)
+      if (leader) mma_ss(d_tmem, a0 + 2 * k4, b0 + 2 * k4, idesc, (acc || (c | k4) != 0));
     a0 += (kT * 128) >> 4;
     b0 += (kT * 128) >> 4;
   }
@@ -91,11 +93,12 @@ __device__ __forceinline__ void mma_kmajor_tile(uint32_t d_tmem, uint64_t a0, ui
 // D += A B with A = 128 x 128 bf16 in TMEM (packed pairs: K = 0..63 in the 32
 // columns at a_lo, K = 64..127 in the 32 columns at a_hi) and B = an MN-major
 // 128-row x D tile in shared memory (K = its rows).
-__device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint64_t b0,
+__device__ __forceinline__ void mma_tmem_a(bool leader, uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint64_t b0,
                                            uint32_t idesc, bool acc) {
 #pragma unroll
   for (int kk = 0; kk < kT / 16; ++kk)
-    mma_ts(d_tmem, (kk < 4 ? a_lo : a_hi - 32) + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc,
+    if (leader)
+      mma_ts(d_tmem, (kk < 4 ? a_lo : a_hi - 32) + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc,
            (acc || kk > 0) ? 1u : 0u);
 }
 
@@ -260,49 +263,56 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bulk_load(sb + L::kVec + (s * 2 + 0) * kT * 4, a.lse2 + vrow, kT * 4, BAR_QF(s));
       bulk_load(sb + L::kVec + (s * 2 + 1) * kT * 4, a.delta + vrow, kT * 4, BAR_QF(s));
     }
-  } else if (n_items > 0 && warp == 1 && lane == 0) {
+  } else if (n_items > 0 && warp == 1) {
     // ======================= MMA issuer =======================
+    // The whole warp runs the issue loop (warp-uniform descriptors and
+    // waits); the elected lane issues the MMAs and their commits.
+    const bool leader = elect_one_sync();
+    auto commit = [&](uint32_t bar) {
+      if (leader) mma_commit(bar);
+      __syncwarp();
+    };
     constexpr uint32_t idesc_s = idesc_bf16_f32(kT, kT, false);   // 128 x 128, K-major B
     constexpr uint32_t idesc_acc = idesc_bf16_f32(kT, D, true);   // 128 x D, MN-major B
     const uint64_t dK = smem_desc_sw128(sK, 16, 1024), dV = smem_desc_sw128(sV, 16, 1024);
     const uint64_t dQk = smem_desc_sw128(sQ, 16, 1024), dDOk = smem_desc_sw128(sDO, 16, 1024);
     const uint64_t dQm = smem_desc_sw128(sQ, T::kChunkBytes, 1024), dDOm = smem_desc_sw128(sDO, T::kChunkBytes, 1024);
     constexpr uint64_t kStep = T::kTileBytes >> 4;
-    bool ok = mbar_wait(BAR_KV, 0, a.status, abort_flag);
-    ok = ok && mbar_wait(BAR_QF(0), 0, a.status, abort_flag);
+    bool ok = mbar_wait_warp(BAR_KV, 0, a.status, abort_flag);
+    ok = ok && mbar_wait_warp(BAR_QF(0), 0, a.status, abort_flag);
     if (ok) {
       tc_fence_after();
       // S^T = K Q^T and dP^T = V dO^T for the first item
-      mma_kmajor_tile(tmem + L::kTmS, dK, dQk, T::kChunks, idesc_s, false);
-      mma_commit(BAR_SF);
-      mma_kmajor_tile(tmem + L::kTmDP, dV, dDOk, T::kChunks, idesc_s, false);
-      mma_commit(BAR_DPF);
+      mma_kmajor_tile(leader, tmem + L::kTmS, dK, dQk, T::kChunks, idesc_s, false);
+      commit(BAR_SF);
+      mma_kmajor_tile(leader, tmem + L::kTmDP, dV, dDOk, T::kChunks, idesc_s, false);
+      commit(BAR_DPF);
     }
     for (int it = 0; it < n_items && ok; ++it) {
       const int s = it & 1, s1 = s ^ 1;
       const uint32_t ph = it & 1u;
       // dV += P^T dO once P^T is in TMEM
-      if (!(ok = mbar_wait(BAR_PF, ph, a.status, abort_flag))) break;
+      if (!(ok = mbar_wait_warp(BAR_PF, ph, a.status, abort_flag))) break;
       tc_fence_after();
-      mma_tmem_a(tmem + L::kTmDV, tmem + L::kTmS, tmem + L::kTmS + 64, dDOm + s * kStep, idesc_acc, it > 0);
+      mma_tmem_a(leader, tmem + L::kTmDV, tmem + L::kTmS, tmem + L::kTmS + 64, dDOm + s * kStep, idesc_acc, it > 0);
       // next item's S^T: the S buffer is free once the dV product above has read P^T
       if (it + 1 < n_items) {
-        if (!(ok = mbar_wait(BAR_QF(s1), ((it + 1) >> 1) & 1u, a.status, abort_flag))) break;
+        if (!(ok = mbar_wait_warp(BAR_QF(s1), ((it + 1) >> 1) & 1u, a.status, abort_flag))) break;
         tc_fence_after();
-        mma_kmajor_tile(tmem + L::kTmS, dK, dQk + s1 * kStep, T::kChunks, idesc_s, false);
-        mma_commit(BAR_SF);
+        mma_kmajor_tile(leader, tmem + L::kTmS, dK, dQk + s1 * kStep, T::kChunks, idesc_s, false);
+        commit(BAR_SF);
       }
       // dK += dS^T Q once dS^T is in TMEM
-      if (!(ok = mbar_wait(BAR_DSF, ph, a.status, abort_flag))) break;
+      if (!(ok = mbar_wait_warp(BAR_DSF, ph, a.status, abort_flag))) break;
       tc_fence_after();
-      mma_tmem_a(tmem + L::kTmDK, tmem + L::kTmDP, tmem + L::kTmDP + 64, dQm + s * kStep, idesc_acc, it > 0);
-      mma_commit(BAR_QE(s));   // this stage's Q, dO, lse and delta are read once these land
+      mma_tmem_a(leader, tmem + L::kTmDK, tmem + L::kTmDP, tmem + L::kTmDP + 64, dQm + s * kStep, idesc_acc, it > 0);
+      commit(BAR_QE(s));   // this stage's Q, dO, lse and delta are read once these land
       if (it + 1 < n_items) {
-        mma_kmajor_tile(tmem + L::kTmDP, dV, dDOk + s1 * kStep, T::kChunks, idesc_s, false);
-        mma_commit(BAR_DPF);
+        mma_kmajor_tile(leader, tmem + L::kTmDP, dV, dDOk + s1 * kStep, T::kChunks, idesc_s, false);
+        commit(BAR_DPF);
       }
     }
-    if (ok) mma_commit(BAR_ACC);
+    if (ok) commit(BAR_ACC);
   }
   } else {
     setmaxnreg_inc<kBwdRegsWork>();
@@ -555,24 +565,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int c = 0; c < T::kChunks; ++c)
         tma_load_3d(sV + sv * T::kTileBytes + c * T::kChunkBytes, &tmV, BAR_VF(sv), c * 64, j * kT, zk);
     }
-  } else if (n > 0 && warp == 1 && lane == 0) {
+  } else if (n > 0 && warp == 1) {
     // ======================= MMA issuer =======================
+    // The whole warp runs the issue loop (warp-uniform descriptors and
+    // waits); the elected lane issues the MMAs and their commits.
+    const bool leader = elect_one_sync();
+    auto commit = [&](uint32_t bar) {
+      if (leader) mma_commit(bar);
+      __syncwarp();
+    };
     constexpr uint32_t idesc_s = idesc_bf16_f32(kT, kT, false);
     constexpr uint32_t idesc_acc = idesc_bf16_f32(kT, D, true);
     const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024), dDO = smem_desc_sw128(sDO, 16, 1024);
     const uint64_t dKk = smem_desc_sw128(sK, 16, 1024), dVk = smem_desc_sw128(sV, 16, 1024);
     const uint64_t dKm = smem_desc_sw128(sK, T::kChunkBytes, 1024);
     constexpr uint64_t kStep = T::kTileBytes >> 4;
-    bool ok = mbar_wait(BAR_Q, 0, a.status, abort_flag);
-    ok = ok && mbar_wait(BAR_KF(0), 0, a.status, abort_flag);
-    ok = ok && mbar_wait(BAR_VF(0), 0, a.status, abort_flag);
+    bool ok = mbar_wait_warp(BAR_Q, 0, a.status, abort_flag);
+    ok = ok && mbar_wait_warp(BAR_KF(0), 0, a.status, abort_flag);
+    ok = ok && mbar_wait_warp(BAR_VF(0), 0, a.status, abort_flag);
     if (ok) {
       tc_fence_after();
-      mma_kmajor_tile(tmem + L::kTmS, dQ, dKk, T::kChunks, idesc_s, false);     // S = Q K_0^T
-      mma_commit(BAR_SF);
-      mma_kmajor_tile(tmem + L::kTmDP, dDO, dVk, T::kChunks, idesc_s, false);   // dP = dO V_0^T
-      mma_commit(BAR_DPF);
-      if (kSV < n) mma_commit(BAR_VE(0));   // release a slot only when a later load reuses it
+      mma_kmajor_tile(leader, tmem + L::kTmS, dQ, dKk, T::kChunks, idesc_s, false);     // S = Q K_0^T
+      commit(BAR_SF);
+      mma_kmajor_tile(leader, tmem + L::kTmDP, dDO, dVk, T::kChunks, idesc_s, false);   // dP = dO V_0^T
+      commit(BAR_DPF);
+      if (kSV < n) commit(BAR_VE(0));   // release a slot only when a later load reuses it
     }
     for (int j = 0; j < n && ok; ++j) {
       const int sk = j % kSK, sk1 = (j + 1) % kSK, sv1 = (j + 1) % kSV;
@@ -580,25 +597,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t phk1 = ((j + 1) / kSK) & 1u, phv1 = ((j + 1) / kSV) & 1u;
       // next S and dP as soon as the work warps hold this tile's in registers
       if (j + 1 < n) {
-        if (!(ok = mbar_wait(BAR_LOADED, ph, a.status, abort_flag))) break;
-        if (!(ok = mbar_wait(BAR_KF(sk1), phk1, a.status, abort_flag))) break;
+        if (!(ok = mbar_wait_warp(BAR_LOADED, ph, a.status, abort_flag))) break;
+        if (!(ok = mbar_wait_warp(BAR_KF(sk1), phk1, a.status, abort_flag))) break;
         tc_fence_after();
-        mma_kmajor_tile(tmem + L::kTmS, dQ, dKk + sk1 * kStep, T::kChunks, idesc_s, false);
-        mma_commit(BAR_SF);
-        if (!(ok = mbar_wait(BAR_VF(sv1), phv1, a.status, abort_flag))) break;
+        mma_kmajor_tile(leader, tmem + L::kTmS, dQ, dKk + sk1 * kStep, T::kChunks, idesc_s, false);
+        commit(BAR_SF);
+        if (!(ok = mbar_wait_warp(BAR_VF(sv1), phv1, a.status, abort_flag))) break;
         tc_fence_after();
-        mma_kmajor_tile(tmem + L::kTmDP, dDO, dVk + sv1 * kStep, T::kChunks, idesc_s, false);
-        mma_commit(BAR_DPF);
-        if (j + 1 + kSV < n) mma_commit(BAR_VE(sv1));
+        mma_kmajor_tile(leader, tmem + L::kTmDP, dDO, dVk + sv1 * kStep, T::kChunks, idesc_s, false);
+        commit(BAR_DPF);
+        if (j + 1 + kSV < n) commit(BAR_VE(sv1));
       }
       // dQ += dS K_j once dS is in its buffer
-      if (!(ok = mbar_wait(BAR_DSF, ph, a.status, abort_flag))) break;
+      if (!(ok = mbar_wait_warp(BAR_DSF, ph, a.status, abort_flag))) break;
       tc_fence_after();
-      mma_tmem_a(tmem + L::kTmDQ, tmem + L::kTmDS, tmem + L::kTmDS + 32, dKm + sk * kStep, idesc_acc, j > 0);
-      mma_commit(BAR_DSE);
-      if (j + kSK < n) mma_commit(BAR_KE(sk));
+      mma_tmem_a(leader, tmem + L::kTmDQ, tmem + L::kTmDS, tmem + L::kTmDS + 32, dKm + sk * kStep, idesc_acc, j > 0);
+      commit(BAR_DSE);
+      if (j + kSK < n) commit(BAR_KE(sk));
     }
-    if (ok) mma_commit(BAR_ACC);
+    if (ok) commit(BAR_ACC);
   }
   } else {
     setmaxnreg_inc<kBwdRegsWork>();

@@ -13,7 +13,8 @@
 // (chunked prefill, LLM-inference article section 3.2; PagedAttention,
 // GPU-optimisation tag page).  Warp roles (384 threads, three warpgroups):
 //   warp 0      TMA producer: Q tiles once, then K_j / V_j into a smem ring
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warp 1      TMEM allocator + tcgen05.mma issuer (whole warp, one elected
+//               lane issues)
 //   warps 2-3   idle after setup
 //   warps 4-7   softmax warpgroup for query tile 0 (one thread per row)
 //   warps 8-11  softmax warpgroup for query tile 1
@@ -34,6 +35,7 @@
 // the result is unchanged because numerator and denominator share the stale
 // max.  lse = m * scale + ln(l) is written per row (the row max and
 // normaliser kept for a recomputing backward, kernel-fusion post section 4).
+// Dense bf16 tiles leave O / l through the tile's Q buffer and TMA stores.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -128,9 +130,14 @@ __device__ __forceinline__ int kv_tiles_for(int q0, int Nq, int Nkv, int causal)
 template <int D, bool kPaged, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                       const PrefillArgs a) {
   static_assert(!(kPaged && kFp8), "fp8 inputs: dense layout only");
   using L = PrefillLayout<D, kFp8>;
+  // Dense bf16: O leaves through shared memory and TMA stores.  Paged query
+  // tiles end mid-tile at other sequences' rows and FP8's Q buffer is half a
+  // bf16 O tile, so those store per thread.
+  constexpr bool kTmaStoreO = !kPaged && !kFp8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -211,6 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    if constexpr (kTmaStoreO) prefetch_tmap(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
@@ -301,15 +309,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(BAR_KF(s), ph, a.status, abort_flag);
         mbar_wait(BAR_VF(s), ph, a.status, abort_flag);
       }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
     // ======================= MMA issuer =======================
+      // The whole warp runs the issue loop (warp-uniform descriptors and
+      // waits); the elected lane issues the MMAs and their commits.
+      const bool leader = elect_one_sync();
       constexpr uint32_t idesc_qk = kFp8 ? idesc_e4m3_f32(kBM, kBN, false) : idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = kFp8 ? idesc_e4m3_f32(kBM, D, true) : idesc_bf16_f32(kBM, D, true);
-      auto mma_s = [](uint32_t d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
+      auto mma_s = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
+        if (!leader) return;
         if constexpr (kFp8) mma_ss_f8(d, ad, bd, id, acc); else mma_ss(d, ad, bd, id, acc);
       };
-      auto mma_t = [](uint32_t d, uint32_t at, uint64_t bd, uint32_t id, uint32_t acc) {
+      auto mma_t = [&](uint32_t d, uint32_t at, uint64_t bd, uint32_t id, uint32_t acc) {
+        if (!leader) return;
         if constexpr (kFp8) mma_ts_f8(d, at, bd, id, acc); else mma_ts(d, at, bd, id, acc);
+      };
+      // commits come from the lane that issued the MMAs they cover
+      auto commit = [&](uint32_t bar) {
+        if (leader) mma_commit(bar);
+        __syncwarp();
       };
       auto tS = [&](int t) { return tmem + (t ? L::kTmS1 : L::kTmS0); };
       auto tO = [&](int t) { return tmem + (t ? L::kTmO1 : L::kTmO0); };
@@ -353,17 +371,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
-      bool ok = mbar_wait(BAR_Q(), 0, a.status, abort_flag);
+      bool ok = mbar_wait_warp(BAR_Q(), 0, a.status, abort_flag);
       if (ok && n_max > 0) {
-        ok = mbar_wait(BAR_KF(0), 0, a.status, abort_flag);
+        ok = mbar_wait_warp(BAR_KF(0), 0, a.status, abort_flag);
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
             if ((t ? nt_1 : nt_0) > 0) {
               issue_qk(t, 0);
-              mma_commit(BAR_SF(t));
+              commit(BAR_SF(t));
             }
-          if (L::kStages < n_max) mma_commit(BAR_KE(0));  // only if a later load reuses stage 0
+          if (L::kStages < n_max) commit(BAR_KE(0));  // only if a later load reuses stage 0
         }
       }
       for (int j = 0; j < n_max && ok; ++j) {
@@ -371,28 +389,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (j / L::kStages) & 1u;
         const int s1 = (j + 1) % L::kStages;
         const uint32_t ph1 = ((j + 1) / L::kStages) & 1u;
-        if (!(ok = mbar_wait(BAR_VF(s), ph, a.status, abort_flag))) break;
+        if (!(ok = mbar_wait_warp(BAR_VF(s), ph, a.status, abort_flag))) break;
         for (int t = 0; t < 2; ++t) {
           const int ntt = t ? nt_1 : nt_0;
           if (j >= ntt) continue;
-          if (!(ok = mbar_wait(BAR_PH(t), j & 1u, a.status, abort_flag))) break;
+          if (!(ok = mbar_wait_warp(BAR_PH(t), j & 1u, a.status, abort_flag))) break;
           tc_fence_after();
           issue_pv_half(t, s, 0, j > 0);
-          if (!(ok = mbar_wait(BAR_PR(t), j & 1u, a.status, abort_flag))) break;
+          if (!(ok = mbar_wait_warp(BAR_PR(t), j & 1u, a.status, abort_flag))) break;
           tc_fence_after();
           issue_pv_half(t, s, 1, true);
-          mma_commit(BAR_OD(t));
+          commit(BAR_OD(t));
           if (j + 1 < ntt) {
-            if (!(ok = mbar_wait(BAR_KF(s1), ph1, a.status, abort_flag))) break;
+            if (!(ok = mbar_wait_warp(BAR_KF(s1), ph1, a.status, abort_flag))) break;
             issue_qk(t, s1);
-            mma_commit(BAR_SF(t));
+            commit(BAR_SF(t));
           }
         }
         if (!ok) break;
         // release a stage only when a later load will reuse it, so no commit
         // is left pending on a barrier nobody waits for at exit
-        if (j + L::kStages < n_max) mma_commit(BAR_VE(s));
-        if (j + 1 + L::kStages < n_max) mma_commit(BAR_KE(s1));
+        if (j + L::kStages < n_max) commit(BAR_VE(s));
+        if (j + 1 + L::kStages < n_max) commit(BAR_KE(s1));
       }
     }
   } else {
@@ -554,19 +572,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t orow = kPaged ? static_cast<size_t>(q_base + (store ? qrow : 0)) * a.Hq + hq
                                : (static_cast<size_t>(b) * a.Hq + hq) * Nq + qrow;
     const float inv = (l > 0.f) ? (kFp8 ? a.v_descale / l : 1.f / l) : 0.f;
-    __nv_bfloat16* optr = a.o + orow * D;
+    if constexpr (kTmaStoreO) {
+      // O / l as bf16 into this tile's Q buffer, in the 128-byte-swizzled
+      // layout of the O tensor map's 64-column boxes, then one TMA store per
+      // box (rows past Nq are clipped by the map).  The Q buffer is free:
+      // this tile's last MMA has completed, or, with no K/V tile, its Q load
+      // has landed.
+      if (!have && q0 < Nq) mbar_wait(BAR_Q(), 0, a.status, abort_flag);
+      uint8_t* stage = smem + L::kQ + t * L::kTileBytes;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t orr[32];
-      if (have && ok) {
-        tmem_ld32(tO + c * 32, orr);
-        tmem_wait_ld();
-      } else {
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t orr[32];
+        if (have && ok) {
+          tmem_ld32(tO + c * 32, orr);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) orr[e] = 0u;
-      }
-      if (store) {
-        uint4* dst = reinterpret_cast<uint4*>(optr + c * 32);
+          for (int e = 0; e < 32; ++e) orr[e] = 0u;
+        }
+        uint8_t* rowp = stage + (c >> 1) * L::kChunkBytes + row * 128;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           uint4 w;
@@ -574,7 +598,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.y = pack_bf16x2(__uint_as_float(orr[8 * e + 2]) * inv, __uint_as_float(orr[8 * e + 3]) * inv);
           w.z = pack_bf16x2(__uint_as_float(orr[8 * e + 4]) * inv, __uint_as_float(orr[8 * e + 5]) * inv);
           w.w = pack_bf16x2(__uint_as_float(orr[8 * e + 6]) * inv, __uint_as_float(orr[8 * e + 7]) * inv);
-          dst[e] = w;
+          const int unit = (c & 1) * 4 + e;   // 16-byte unit of the 128-byte row, swizzled by row % 8
+          *reinterpret_cast<uint4*>(rowp + ((unit ^ (row & 7)) << 4)) = w;
+        }
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(1 + t, 128);
+      if (row == 0 && q0 < Nq) {
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_store_3d(&tmO, sQ + t * L::kTileBytes + c * L::kChunkBytes, c * L::kChunkElems, q0,
+                       b * a.Hq + hq);
+        bulk_commit_group();
+        bulk_wait_group_read0();   // the buffer must stay valid until the stores have read it
+      }
+    } else {
+      __nv_bfloat16* optr = a.o + orow * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t orr[32];
+        if (have && ok) {
+          tmem_ld32(tO + c * 32, orr);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) orr[e] = 0u;
+        }
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(optr + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(orr[8 * e + 0]) * inv, __uint_as_float(orr[8 * e + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(orr[8 * e + 2]) * inv, __uint_as_float(orr[8 * e + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(orr[8 * e + 4]) * inv, __uint_as_float(orr[8 * e + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(orr[8 * e + 6]) * inv, __uint_as_float(orr[8 * e + 7]) * inv);
+            dst[e] = w;
+          }
         }
       }
     }
@@ -621,6 +680,8 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   if ((st = encode_rows_3d(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
   if ((st = encode_rows_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
   if ((st = encode_rows_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
+  CUtensorMap to;   // O is stored through the same [B*Hq, Nq, d] box layout as Q
+  if ((st = encode_rows_3d(&to, o, D, Nq, B * Hq)) != TA_OK) return st;
   static int attr_done[64] = {0};
   cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, false, false>, L::kAlloc, attr_done);
   if (e != cudaSuccess) return fail(TA_ERR_CUDA, "prefill: shared-memory limit", e);
@@ -640,7 +701,7 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   a.status = device_status_ptr();
   if (!a.status) return fail(TA_ERR_CUDA, "prefill: device status word");
   const unsigned grid = static_cast<unsigned>(a.n_units) * static_cast<unsigned>(B * Hq / (a.head_pair + 1));
-  prefill_fwd_kernel<D, false, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
+  prefill_fwd_kernel<D, false, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, to, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "prefill: launch", e);
 }
@@ -695,7 +756,7 @@ static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, cons
   a.max_pages = max_pages;
   a.num_pages_total = num_pages_total;
   const unsigned grid = static_cast<unsigned>(a.n_units) * static_cast<unsigned>(num_seqs * Hq / (a.head_pair + 1));
-  prefill_fwd_kernel<D, true, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
+  prefill_fwd_kernel<D, true, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, tq, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "paged prefill: launch", e);
 }
@@ -741,7 +802,7 @@ ta_status launch_prefill_fp8(const void* q, const void* k, const void* v, float 
   a.status = device_status_ptr();
   if (!a.status) return fail(TA_ERR_CUDA, "fp8 prefill: device status word");
   const unsigned grid = static_cast<unsigned>(a.n_units) * static_cast<unsigned>(B * Hq / (a.head_pair + 1));
-  prefill_fwd_kernel<D, false, true><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
+  prefill_fwd_kernel<D, false, true><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, tq, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "fp8 prefill: launch", e);
 }

@@ -92,6 +92,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   }
 }
 
+// Warp-uniform form of mbar_wait for a warp whose lanes all run the same
+// control flow: every lane waits and all get the same answer, so a timeout
+// seen by one lane cannot split the warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, unsigned* status,
+                                               volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, abort_flag));
+}
+
+// One lane of a fully active warp (elect.sync): the lane that issues the
+// warp's tcgen05 operations.  Operands the whole warp computes beforehand are
+// warp-uniform, so the compiler keeps them in uniform registers and the
+// issuing lane does not move each descriptor over before every MMA.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t p;
+  asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}" : "=r"(p));
+  return p != 0;
+}
+
 // ----------------------------------------------------------------------------
 // TMA: tiled tensor loads (no multicast) and plain bulk copies
 // ----------------------------------------------------------------------------
@@ -110,6 +128,29 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
       : "memory");
+}
+
+// Shared -> global tiled TMA store of one box (bulk-group completion); rows
+// and columns outside the tensor map's extent are not written.
+__device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(src), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the committed bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Make this thread's generic-proxy writes to shared memory visible to later
+// async-proxy operations (TMA stores).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Barrier over `count` threads (a multiple of 32) with id 1-15.
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
