@@ -6,13 +6,17 @@
 // (Gemini 3 Flash kernel-fusion post, sections 1-3; FlashAttention
 // optimisation article, sections 3.1-3.2 and 7.1).
 //
-// CTA = two 128-row query tiles sharing one K/V stream (two tiles of one head,
-// or one tile of two GQA heads).  Instantiations: dense [B, H, N, d] bf16; FP8
+// Work item = two 128-row query tiles sharing one K/V stream (two tiles of one
+// head, or one tile of two GQA heads).  Dense and FP8 CTAs are persistent: after
+// their own item they take over the items of CTAs not yet launched (cluster
+// launch control), so the next item's loads and first Q.K^T overlap the
+// epilogue of the current one.  Instantiations: dense [B, H, N, d] bf16; FP8
 // (kFp8) E4M3 inputs; (kPaged) varlen query rows packed as [total_q, Hq, d]
 // against K/V gathered page by page from a paged cache through a block table
 // (chunked prefill, LLM-inference article section 3.2; PagedAttention,
 // GPU-optimisation tag page).  Warp roles (384 threads, three warpgroups):
-//   warp 0      TMA producer: Q tiles once, then K_j / V_j into a smem ring
+//   warp 0      TMA producer: Q tiles once per item, then K_j / V_j into a
+//               smem ring; makes the work requests
 //   warp 1      TMEM allocator + tcgen05.mma issuer (whole warp, one elected
 //               lane issues)
 //   warps 2-3   idle after setup
@@ -35,7 +39,6 @@
 // the result is unchanged because numerator and denominator share the stale
 // max.  lse = m * scale + ln(l) is written per row (the row max and
 // normaliser kept for a recomputing backward, kernel-fusion post section 4).
-// Dense bf16 tiles leave O / l through the tile's Q buffer and TMA stores.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -84,9 +87,11 @@ struct PrefillLayout {
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kBar = kV + kStages * kTileBytes;
   // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2], o_done[2],
-  // p_half[2] (first 64 keys of P written)
-  static constexpr int kNumBars = 1 + 4 * kStages + 8;
-  static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base (4 B) + abort flag (4 B)
+  // p_half[2] (first 64 keys of P written), item_full[2], item_empty[2] (work-request
+  // responses), q_free, o_free[2] (epilogue has read O), mma_done
+  static constexpr int kNumBars = 1 + 4 * kStages + 16;
+  static constexpr int kResp = (kBar + kNumBars * 8 + 15) & ~15;   // two 16-byte work-request responses
+  static constexpr int kMisc = kResp + 32;            // tmem base (4 B) + abort flag (4 B)
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;        // slack to align the base to 1024 B
   static constexpr uint32_t kTmemCols = 512;
@@ -130,14 +135,9 @@ __device__ __forceinline__ int kv_tiles_for(int q0, int Nq, int Nkv, int causal)
 template <int D, bool kPaged, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                       const PrefillArgs a) {
+                       const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
   static_assert(!(kPaged && kFp8), "fp8 inputs: dense layout only");
   using L = PrefillLayout<D, kFp8>;
-  // Dense bf16: O leaves through shared memory and TMA stores.  Paged query
-  // tiles end mid-tile at other sequences' rows and FP8's Q buffer is half a
-  // bf16 O tile, so those store per thread.
-  constexpr bool kTmaStoreO = !kPaged && !kFp8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -152,49 +152,78 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto BAR_PR = [&](int t) { return bar0 + 8u * (3 + 4 * L::kStages + t); };
   auto BAR_OD = [&](int t) { return bar0 + 8u * (5 + 4 * L::kStages + t); };
   auto BAR_PH = [&](int t) { return bar0 + 8u * (7 + 4 * L::kStages + t); };
+  auto BAR_ITF = [&](int s) { return bar0 + 8u * (9 + 4 * L::kStages + s); };
+  auto BAR_ITE = [&](int s) { return bar0 + 8u * (11 + 4 * L::kStages + s); };
+  auto BAR_QE = [&]() { return bar0 + 8u * (13 + 4 * L::kStages); };
+  auto BAR_OF = [&](int t) { return bar0 + 8u * (14 + 4 * L::kStages + t); };
+  auto BAR_FIN = [&]() { return bar0 + 8u * (16 + 4 * L::kStages); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: heavy (late) query units first so causal tails are short.
-  // A CTA's two 128-row query tiles are two consecutive tiles of one head, or
-  // (head_pair) the same tile of two query heads of one GQA group: both then
-  // read the same K/V stream and have the same number of K/V tiles, so the
-  // two softmax warpgroups always have equal work.
-  // Dense: (unit, batch, head[s]).  Paged: (unit, sequence, head[s]), with the
-  // sequence's query and key counts read (and range-checked) here.
-  const int heads_per_item = a.head_pair ? 2 : 1;
-  const int hx_count = a.Hq / heads_per_item;
-  const int bh_count = (kPaged ? a.num_seqs : a.B) * hx_count;
-  const int unit = a.n_units - 1 - static_cast<int>(blockIdx.x) / bh_count;
-  const int bh = static_cast<int>(blockIdx.x) % bh_count;
-  const int b = bh / hx_count;                             // b = sequence when paged
-  const int hq_0 = (bh % hx_count) * heads_per_item;      // query head of tile 0
-  const int hq_1 = hq_0 + heads_per_item - 1;             // query head of tile 1
-  const int hkv = hq_0 / (a.Hq / a.Hkv);
-  int Nq = a.Nq, Nkv = a.Nkv;
-  int q_base = 0;                  // packed row of the sequence's first query (paged)
-  if constexpr (kPaged) {
-    int lo = a.cu_seqlens[b], hi = a.cu_seqlens[b + 1];
-    int len = a.seq_lens[b];
-    unsigned bad = 0;
-    if (lo < 0 || lo > a.total_q || hi < lo || hi > a.total_q || hi - lo > a.max_q_len) bad |= kDevBadSeqLen;
-    if (len < 0 || len > a.max_pages * a.page_size) bad |= kDevBadSeqLen;
-    lo = min(max(lo, 0), a.total_q);
-    hi = min(max(hi, lo), min(a.total_q, lo + a.max_q_len));
-    len = min(max(len, 0), a.max_pages * a.page_size);
-    if (bad && threadIdx.x == 0 && unit == 0 && hq_0 == 0) atomicOr(a.status, bad);
-    q_base = lo;
-    Nq = hi - lo;
-    Nkv = len;
+  // ---- work items.  A CTA starts with item blockIdx.x and then takes over
+  // the items of CTAs that have not launched yet (cluster launch control: a
+  // successful try_cancel hands over the cancelled CTA's index).  Each SM so
+  // runs a sequence of items in launch order, heaviest first, and the next
+  // item's loads and first product overlap the current item's epilogue.  An
+  // item's two 128-row query tiles are two consecutive tiles of one head, or
+  // (head_pair) the same tile of two query heads of one GQA group: both read
+  // the same K/V stream.  Dense: (unit, batch, head[s]).  Paged: (unit,
+  // sequence, head[s]), with the sequence's query and key counts read (and
+  // range-checked) here; units past a sequence's queries are empty items.
+  struct Item {
+    int b, hq_0, hq_1, hkv, Nq, Nkv, q_base, q0_0, q0_1, nt_0, nt_1, n_max;
+    bool valid;
+  };
+  auto decode_item = [&](int idx, bool report) {
+    Item it;
+    const int heads_per_item = a.head_pair ? 2 : 1;
+    const int hx_count = a.Hq / heads_per_item;
+    const int bh_count = (kPaged ? a.num_seqs : a.B) * hx_count;
+    const int unit = a.n_units - 1 - idx / bh_count;
+    const int bh = idx % bh_count;
+    it.b = bh / hx_count;                             // sequence when paged
+    it.hq_0 = (bh % hx_count) * heads_per_item;      // query head of tile 0
+    it.hq_1 = it.hq_0 + heads_per_item - 1;          // query head of tile 1
+    it.hkv = it.hq_0 / (a.Hq / a.Hkv);
+    it.Nq = a.Nq;
+    it.Nkv = a.Nkv;
+    it.q_base = 0;                                   // packed row of the sequence's first query (paged)
+    if constexpr (kPaged) {
+      int lo = a.cu_seqlens[it.b], hi = a.cu_seqlens[it.b + 1];
+      int len = a.seq_lens[it.b];
+      unsigned bad = 0;
+      if (lo < 0 || lo > a.total_q || hi < lo || hi > a.total_q || hi - lo > a.max_q_len) bad |= kDevBadSeqLen;
+      if (len < 0 || len > a.max_pages * a.page_size) bad |= kDevBadSeqLen;
+      lo = min(max(lo, 0), a.total_q);
+      hi = min(max(hi, lo), min(a.total_q, lo + a.max_q_len));
+      len = min(max(len, 0), a.max_pages * a.page_size);
+      if (bad && report && unit == 0 && it.hq_0 == 0) atomicOr(a.status, bad);
+      it.q_base = lo;
+      it.Nq = hi - lo;
+      it.Nkv = len;
+    }
+    it.q0_0 = a.head_pair ? unit * kBM : unit * 2 * kBM;
+    it.q0_1 = a.head_pair ? it.q0_0 : it.q0_0 + kBM;
+    it.valid = !(kPaged && it.q0_0 >= it.Nq);
+    it.nt_0 = it.valid ? kv_tiles_for(it.q0_0, it.Nq, it.Nkv, a.causal) : 0;
+    it.nt_1 = it.valid ? kv_tiles_for(it.q0_1, it.Nq, it.Nkv, a.causal) : 0;
+    it.n_max = max(it.nt_0, it.nt_1);
+    return it;
+  };
+  // Dense and FP8 CTAs take further items; a paged CTA runs its own item
+  // only (about half of a varlen grid are empty units past their sequence's
+  // queries, which exit at once instead of costing a work request each).
+  constexpr bool kPersistent = !kPaged;
+  if constexpr (!kPersistent) {
+    if (!decode_item(static_cast<int>(blockIdx.x), false).valid) return;   // uniform per CTA
   }
-  const int q0_0 = a.head_pair ? unit * kBM : unit * 2 * kBM;
-  const int q0_1 = a.head_pair ? q0_0 : q0_0 + kBM;
-  if (kPaged && q0_0 >= Nq) return;   // this sequence has fewer query units (uniform per CTA)
-  const int nt_0 = kv_tiles_for(q0_0, Nq, Nkv, a.causal), nt_1 = kv_tiles_for(q0_1, Nq, Nkv, a.causal);
-  const int n_max = max(nt_0, nt_1);
+  // Work request k >= 1 (the item after the k-th) answers in slot k & 1; it is
+  // that slot's ((k - 1) >> 1)-th use.
+  const uint32_t sResp = sbase + L::kResp;
+  auto resp_parity = [](int k) { return static_cast<uint32_t>((k - 1) >> 1) & 1u; };
 
   // ---- setup
   if (threadIdx.x == 0) {
@@ -210,7 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(BAR_PR(t), 128);
       mbar_init(BAR_OD(t), 1);
       mbar_init(BAR_PH(t), 128);
+      mbar_init(BAR_ITF(t), 1);
+      mbar_init(BAR_ITE(t), 1 + 256);   // the MMA warp's leader and every softmax thread
+      mbar_init(BAR_OF(t), 128);
     }
+    mbar_init(BAR_QE(), 1);
+    mbar_init(BAR_FIN(), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -218,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
-    if constexpr (kTmaStoreO) prefetch_tmap(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
@@ -233,35 +266,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     setmaxnreg_dec<kRegsControl>();
     if (warp == 0 && lane == 0) {
     // ======================= TMA producer =======================
-      const int zk = b * a.Hkv + hkv;
-      const uint32_t qbytes = static_cast<uint32_t>((q0_0 < Nq) + (q0_1 < Nq)) * L::kTileBytes;
-      mbar_arrive_expect_tx(BAR_Q(), qbytes);
-      for (int t = 0; t < 2; ++t) {
-        const int q0 = t ? q0_1 : q0_0;
-        const int hq = t ? hq_1 : hq_0;
-        if (q0 >= Nq) continue;
-        for (int c = 0; c < L::kChunks; ++c) {
-          if constexpr (kPaged)   // packed [total_q, Hq, d]: box of 128 rows of one head
-            tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, hq,
-                        q_base + q0);
-          else
-            tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, q0,
-                        b * a.Hq + hq);
-        }
-      }
       // Physical pages of K/V tile j (paged): the table entries are read
       // together, once per tile, for both the K and the V copies.  Pages past
       // the sequence, and entries outside the pool (flagged), read page 0: the
       // pool's contents are finite and those keys are masked.
       constexpr int kMaxPagesPerTile = kBN / 8;
       int phys[kMaxPagesPerTile];
-      auto lookup_pages = [&](int j) {
+      auto lookup_pages = [&](const Item& it, int j) {
         if constexpr (kPaged) {
           const int per_tile = kBN / a.page_size;
-          const int32_t* row = a.block_table + static_cast<size_t>(b) * a.max_pages + j * per_tile;
+          const int32_t* row = a.block_table + static_cast<size_t>(it.b) * a.max_pages + j * per_tile;
 #pragma unroll
           for (int p = 0; p < kMaxPagesPerTile; ++p)
-            phys[p] = (p < per_tile && (j * per_tile + p) * a.page_size < Nkv) ? __ldg(row + p) : 0;
+            phys[p] = (p < per_tile && (j * per_tile + p) * a.page_size < it.Nkv) ? __ldg(row + p) : 0;
 #pragma unroll
           for (int p = 0; p < kMaxPagesPerTile; ++p)
             if (phys[p] < 0 || phys[p] >= a.num_pages_total) {
@@ -272,43 +289,90 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // K or V tile j into ring slot `dst`: one tile box (dense), or one box per
       // page (paged, pages from lookup_pages)
-      auto load_kv = [&](const CUtensorMap* tm, uint32_t dst, uint32_t bar, int j) {
+      auto load_kv = [&](const Item& it, const CUtensorMap* tm, uint32_t dst, uint32_t bar, int j) {
         if constexpr (kPaged) {
           const int per_tile = kBN / a.page_size;
 #pragma unroll
           for (int p = 0; p < kMaxPagesPerTile; ++p) {
             if (p >= per_tile) break;
             for (int c = 0; c < L::kChunks; ++c)
-              tma_load_4d(dst + c * L::kChunkBytes + p * a.page_size * 128, tm, bar, c * L::kChunkElems, 0, hkv,
+              tma_load_4d(dst + c * L::kChunkBytes + p * a.page_size * 128, tm, bar, c * L::kChunkElems, 0, it.hkv,
                           phys[p]);
           }
         } else {
           for (int c = 0; c < L::kChunks; ++c)
-            tma_load_3d(dst + c * L::kChunkBytes, tm, bar, c * L::kChunkElems, j * kBN, zk);
+            tma_load_3d(dst + c * L::kChunkBytes, tm, bar, c * L::kChunkElems, j * kBN, it.b * a.Hkv + it.hkv);
         }
       };
       bool ok = true;
-      for (int j = 0; j < n_max && ok; ++j) {
-        const int s = j % L::kStages;
-        const uint32_t ph = (j / L::kStages) & 1u;
-        lookup_pages(j);   // before the wait, so the table reads overlap it
-        ok = mbar_wait(BAR_KE(s), ph ^ 1u, a.status, abort_flag);
-        if (!ok) break;
-        mbar_arrive_expect_tx(BAR_KF(s), L::kTileBytes);
-        load_kv(&tmK, sK + s * L::kTileBytes, BAR_KF(s), j);
-        ok = mbar_wait(BAR_VE(s), ph ^ 1u, a.status, abort_flag);
-        if (!ok) break;
-        mbar_arrive_expect_tx(BAR_VF(s), L::kTileBytes);
-        load_kv(&tmV, sV + s * L::kTileBytes, BAR_VF(s), j);
+      uint32_t g = 0;            // K/V tiles loaded so far: ring slot g % S, use (g / S)
+      uint32_t gk = 0, gv = 0;   // K and V copies issued (for the drain)
+      int qi = 0;                // items whose Q tiles were loaded
+      int requested = 0;         // work requests made (the last one's answer is awaited before exit)
+      int answered = 0;
+      int idx = static_cast<int>(blockIdx.x);
+      for (int k = 0; idx >= 0 && ok; ++k) {
+        // ask for the item after this one now, so the answer is back by the time it is needed
+        if constexpr (kPersistent) {
+          const int kn = k + 1, sl = kn & 1;
+          if (kn >= 3 && !(ok = mbar_wait(BAR_ITE(sl), resp_parity(kn - 2), a.status, abort_flag))) break;
+          fence_proxy_async_smem();   // the slot's previous answer was read through the generic proxy
+          mbar_arrive_expect_tx(BAR_ITF(sl), 16);
+          clc_try_cancel(sResp + 16 * sl, BAR_ITF(sl));
+          requested = kn;
+        }
+        const Item it = decode_item(idx, true);
+        if (it.valid) {
+          // this buffer's previous Q tiles are free once the last Q.K^T reading them completed
+          if (qi > 0 && !(ok = mbar_wait(BAR_QE(), static_cast<uint32_t>(qi - 1) & 1u, a.status, abort_flag)))
+            break;
+          const uint32_t qbytes = static_cast<uint32_t>((it.q0_0 < it.Nq) + (it.q0_1 < it.Nq)) * L::kTileBytes;
+          mbar_arrive_expect_tx(BAR_Q(), qbytes);
+          for (int t = 0; t < 2; ++t) {
+            const int q0 = t ? it.q0_1 : it.q0_0;
+            const int hq = t ? it.hq_1 : it.hq_0;
+            if (q0 >= it.Nq) continue;
+            for (int c = 0; c < L::kChunks; ++c) {
+              if constexpr (kPaged)   // packed [total_q, Hq, d]: box of 128 rows of one head
+                tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, hq,
+                            it.q_base + q0);
+              else
+                tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, q0,
+                            it.b * a.Hq + hq);
+            }
+          }
+          ++qi;
+          for (int j = 0; j < it.n_max && ok; ++j, ++g) {
+            const int s = static_cast<int>(g % L::kStages);
+            const uint32_t ph = (g / L::kStages) & 1u;
+            lookup_pages(it, j);   // before the wait, so the table reads overlap it
+            if (!(ok = mbar_wait(BAR_KE(s), ph ^ 1u, a.status, abort_flag))) break;
+            mbar_arrive_expect_tx(BAR_KF(s), L::kTileBytes);
+            load_kv(it, &tmK, sK + s * L::kTileBytes, BAR_KF(s), j);
+            ++gk;
+            if (!(ok = mbar_wait(BAR_VE(s), ph ^ 1u, a.status, abort_flag))) break;
+            mbar_arrive_expect_tx(BAR_VF(s), L::kTileBytes);
+            load_kv(it, &tmV, sV + s * L::kTileBytes, BAR_VF(s), j);
+            ++gv;
+          }
+          if (!ok) break;
+        }
+        // the next item (or none)
+        if constexpr (!kPersistent) break;
+        const int kn = k + 1, sl = kn & 1;
+        if (!(ok = mbar_wait(BAR_ITF(sl), resp_parity(kn), a.status, abort_flag))) break;
+        answered = kn;
+        idx = clc_cancelled_ctaid_x(sResp + 16 * sl);
       }
-      // drain: make sure no copy into this CTA's smem is still in flight at exit
-      mbar_wait(BAR_Q(), 0, a.status, abort_flag);
-      for (int j = max(0, n_max - L::kStages); j < n_max; ++j) {
-        const int s = j % L::kStages;
-        const uint32_t ph = (j / L::kStages) & 1u;
-        mbar_wait(BAR_KF(s), ph, a.status, abort_flag);
-        mbar_wait(BAR_VF(s), ph, a.status, abort_flag);
-      }
+      // drain: no copy into this CTA's shared memory may still be in flight at exit
+      if (answered < requested)
+        mbar_wait(BAR_ITF(requested & 1), resp_parity(requested), nullptr, nullptr, kWaitLimitNs);
+      if (qi > 0) mbar_wait(BAR_Q(), static_cast<uint32_t>(qi - 1) & 1u, nullptr, nullptr, kWaitLimitNs);
+      constexpr uint32_t kS = L::kStages;
+      for (uint32_t gg = (gk > kS ? gk - kS : 0u); gg < gk; ++gg)
+        mbar_wait(BAR_KF(static_cast<int>(gg % kS)), (gg / kS) & 1u, nullptr, nullptr, kWaitLimitNs);
+      for (uint32_t gg = (gv > kS ? gv - kS : 0u); gg < gv; ++gg)
+        mbar_wait(BAR_VF(static_cast<int>(gg % kS)), (gg / kS) & 1u, nullptr, nullptr, kWaitLimitNs);
     } else if (warp == 1) {
     // ======================= MMA issuer =======================
       // The whole warp runs the issue loop (warp-uniform descriptors and
@@ -371,47 +435,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
-      bool ok = mbar_wait_warp(BAR_Q(), 0, a.status, abort_flag);
-      if (ok && n_max > 0) {
-        ok = mbar_wait_warp(BAR_KF(0), 0, a.status, abort_flag);
-        if (ok) {
+      bool ok = true;
+      uint32_t g = 0;              // K/V tiles consumed (ring position, as the producer's)
+      uint32_t steps[2] = {0, 0};  // K/V steps of each query tile so far: S/P/O barrier phases
+      int qi = 0;                  // items whose Q tiles were used
+      int idx = static_cast<int>(blockIdx.x);
+      for (int k = 0; idx >= 0 && ok; ++k) {
+        const Item it = decode_item(idx, false);
+        if (it.valid) {
+          if (!(ok = mbar_wait_warp(BAR_Q(), static_cast<uint32_t>(qi) & 1u, a.status, abort_flag))) break;
           tc_fence_after();
-          for (int t = 0; t < 2; ++t)
-            if ((t ? nt_1 : nt_0) > 0) {
-              issue_qk(t, 0);
-              commit(BAR_SF(t));
-            }
-          if (L::kStages < n_max) commit(BAR_KE(0));  // only if a later load reuses stage 0
-        }
-      }
-      for (int j = 0; j < n_max && ok; ++j) {
-        const int s = j % L::kStages;
-        const uint32_t ph = (j / L::kStages) & 1u;
-        const int s1 = (j + 1) % L::kStages;
-        const uint32_t ph1 = ((j + 1) / L::kStages) & 1u;
-        if (!(ok = mbar_wait_warp(BAR_VF(s), ph, a.status, abort_flag))) break;
-        for (int t = 0; t < 2; ++t) {
-          const int ntt = t ? nt_1 : nt_0;
-          if (j >= ntt) continue;
-          if (!(ok = mbar_wait_warp(BAR_PH(t), j & 1u, a.status, abort_flag))) break;
-          tc_fence_after();
-          issue_pv_half(t, s, 0, j > 0);
-          if (!(ok = mbar_wait_warp(BAR_PR(t), j & 1u, a.status, abort_flag))) break;
-          tc_fence_after();
-          issue_pv_half(t, s, 1, true);
-          commit(BAR_OD(t));
-          if (j + 1 < ntt) {
-            if (!(ok = mbar_wait_warp(BAR_KF(s1), ph1, a.status, abort_flag))) break;
-            issue_qk(t, s1);
-            commit(BAR_SF(t));
+          if (it.n_max > 0) {
+            const int s0 = static_cast<int>(g % L::kStages);
+            if (!(ok = mbar_wait_warp(BAR_KF(s0), (g / L::kStages) & 1u, a.status, abort_flag))) break;
+            tc_fence_after();
+            for (int t = 0; t < 2; ++t)
+              if ((t ? it.nt_1 : it.nt_0) > 0) {
+                issue_qk(t, s0);
+                commit(BAR_SF(t));
+              }
+            commit(BAR_KE(s0));
           }
+          if (it.n_max <= 1) commit(BAR_QE());   // no later Q.K^T of this item reads Q
+          for (int j = 0; j < it.n_max && ok; ++j) {
+            const uint32_t gj = g + static_cast<uint32_t>(j);
+            const int s = static_cast<int>(gj % L::kStages);
+            const uint32_t ph = (gj / L::kStages) & 1u;
+            const int s1 = static_cast<int>((gj + 1) % L::kStages);
+            const uint32_t ph1 = ((gj + 1) / L::kStages) & 1u;
+            if (!(ok = mbar_wait_warp(BAR_VF(s), ph, a.status, abort_flag))) break;
+            for (int t = 0; t < 2; ++t) {
+              const int ntt = t ? it.nt_1 : it.nt_0;
+              if (j >= ntt) continue;
+              const uint32_t c = steps[t];
+              // the first P.V of an item overwrites O_t: the previous item's
+              // epilogue must have read it
+              if (j == 0 && qi > 0 &&
+                  !(ok = mbar_wait_warp(BAR_OF(t), static_cast<uint32_t>(qi - 1) & 1u, a.status, abort_flag)))
+                break;
+              if (!(ok = mbar_wait_warp(BAR_PH(t), c & 1u, a.status, abort_flag))) break;
+              tc_fence_after();
+              issue_pv_half(t, s, 0, j > 0);
+              if (!(ok = mbar_wait_warp(BAR_PR(t), c & 1u, a.status, abort_flag))) break;
+              tc_fence_after();
+              issue_pv_half(t, s, 1, true);
+              commit(BAR_OD(t));
+              if (j + 1 < ntt) {
+                if (!(ok = mbar_wait_warp(BAR_KF(s1), ph1, a.status, abort_flag))) break;
+                issue_qk(t, s1);
+                commit(BAR_SF(t));
+              }
+              steps[t] = c + 1;
+            }
+            if (!ok) break;
+            if (j + 2 == it.n_max) commit(BAR_QE());   // the item's last Q.K^T has been issued
+            commit(BAR_VE(s));
+            if (j + 1 < it.n_max) commit(BAR_KE(s1));
+          }
+          if (!ok) break;
+          g += static_cast<uint32_t>(it.n_max);
+          ++qi;
         }
-        if (!ok) break;
-        // release a stage only when a later load will reuse it, so no commit
-        // is left pending on a barrier nobody waits for at exit
-        if (j + L::kStages < n_max) commit(BAR_VE(s));
-        if (j + 1 + L::kStages < n_max) commit(BAR_KE(s1));
+        // the next item (or none)
+        if constexpr (!kPersistent) break;
+        const int kn = k + 1, sl = kn & 1;
+        if (!(ok = mbar_wait_warp(BAR_ITF(sl), resp_parity(kn), a.status, abort_flag))) break;
+        idx = clc_cancelled_ctaid_x(sResp + 16 * sl);
+        __syncwarp();
+        if (leader) mbar_arrive(BAR_ITE(sl));
       }
+      // no commit may still be pending when the CTA exits
+      commit(BAR_FIN());
+      mbar_wait_warp(BAR_FIN(), 0, nullptr, nullptr);
     }
   } else {
     setmaxnreg_inc<kRegsSoftmax>();
@@ -419,227 +514,207 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = (warp - kSoftmaxWarp0) / 4;           // query tile of this warpgroup
     const int quarter = warp & 3;                       // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;                // row within the tile
-    const int q0 = t ? q0_1 : q0_0;                     // first query row of the tile
-    const int hq = t ? hq_1 : hq_0;                     // query head of the tile
-    const int qrow = q0 + row;                          // query index
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + (t == 0 ? L::kTmS0 : L::kTmS1) + lane_off;
     const uint32_t tO = tmem + (t == 0 ? L::kTmO0 : L::kTmO1) + lane_off;
-    const int n = t ? nt_1 : nt_0;
-    const int off = Nkv - Nq;
-    // visible keys of this row: [0, vis_end)
-    const int vis_end = a.causal ? min(Nkv, qrow + off + 1) : Nkv;
     const float c2 = a.scale_log2;
-
-    float m = -INFINITY;  // running max of the raw scores q.k
-    float l = 0.f;        // running sum of exp2((s - m) * c2)
     bool ok = true;
+    uint32_t steps = 0;    // K/V steps of this tile so far: S/P/O barrier phases
+    int idx = static_cast<int>(blockIdx.x);
+    for (int k = 0; idx >= 0 && ok; ++k) {
+      const Item it = decode_item(idx, false);
+      if (it.valid) {
+        const int q0 = t ? it.q0_1 : it.q0_0;               // first query row of the tile
+        const int hq = t ? it.hq_1 : it.hq_0;               // query head of the tile
+        const int qrow = q0 + row;                          // query index
+        const int Nq = it.Nq, Nkv = it.Nkv;
+        const int n = t ? it.nt_1 : it.nt_0;
+        const int off = Nkv - Nq;
+        // visible keys of this row: [0, vis_end)
+        const int vis_end = a.causal ? min(Nkv, qrow + off + 1) : Nkv;
 
-    for (int j = 0; j < n; ++j) {
-      ok = mbar_wait(BAR_SF(t), j & 1u, a.status, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
-      tmem_wait_ld();
-      float* s = reinterpret_cast<float*>(&sr[0][0]);
+        float m = -INFINITY;  // running max of the raw scores q.k
+        float l = 0.f;        // running sum of exp2((s - m) * c2)
 
-      // tile-uniform: does any row of this tile have masked keys in tile j?
-      const int kv0 = j * kBN;
-      const bool need_mask =
-          (kv0 + kBN > Nkv) || (a.causal && kv0 + kBN - 1 > q0 + off);
-      const int lim = vis_end - kv0;  // visible columns of this tile for this row: [0, lim)
-      if (need_mask) {
+        for (int j = 0; j < n; ++j) {
+          ok = mbar_wait(BAR_SF(t), (steps + j) & 1u, a.status, abort_flag);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t sr[4][32];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = c < lim ? s[c] : -INFINITY;
-      }
+          for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+          tmem_wait_ld();
+          float* s = reinterpret_cast<float*>(&sr[0][0]);
 
-      // exp2((s - m) * c2) for 32 column pairs [64h, 64h + 64), packed to bf16
-      // pairs (32 words) or to four E4M3 codes per word (fp8: 16 words);
-      // masked columns get exactly 0.  Returns the sum of the unrounded values.
-      // The masked form is a separate specialisation so unmasked tiles carry
-      // no per-element compare/select.
-      auto exp_half = [&](auto masked, int h, float negm, uint32_t (&pk)[L::kPWords]) -> float {
-        constexpr bool kMasked = decltype(masked)::value;
-        const float2 c2v = make_float2(c2, c2), negv = make_float2(negm, negm);
-        float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
-        float2 pp_prev = make_float2(0.f, 0.f);
+          // tile-uniform: does any row of this tile have masked keys in tile j?
+          const int kv0 = j * kBN;
+          const bool need_mask =
+              (kv0 + kBN > Nkv) || (a.causal && kv0 + kBN - 1 > q0 + off);
+          const int lim = vis_end - kv0;  // visible columns of this tile for this row: [0, lim)
+          if (need_mask) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int c = h * 64 + 2 * i;
-          const float2 x = ffma2(make_float2(s[c], s[c + 1]), c2v, negv);
-          float2 pp;
-          if (((kFp8 ? kPolyMaskFp8 : kPolyMask) >> (i & 7)) & 1u) {
-            pp = exp2_poly2(x);
-          } else {
-            pp.x = ex2(x.x);
-            pp.y = ex2(x.y);
+            for (int c = 0; c < 128; ++c) s[c] = c < lim ? s[c] : -INFINITY;
           }
-          if constexpr (kMasked) {
-            pp.x = c < lim ? pp.x : 0.f;
-            pp.y = c + 1 < lim ? pp.y : 0.f;
+
+          // exp2((s - m) * c2) for 32 column pairs [64h, 64h + 64), packed to bf16
+          // pairs (32 words) or to four E4M3 codes per word (fp8: 16 words);
+          // masked columns get exactly 0.  Returns the sum of the unrounded values.
+          // The masked form is a separate specialisation so unmasked tiles carry
+          // no per-element compare/select.
+          auto exp_half = [&](auto masked, int h, float negm, uint32_t (&pk)[L::kPWords]) -> float {
+            constexpr bool kMasked = decltype(masked)::value;
+            const float2 c2v = make_float2(c2, c2), negv = make_float2(negm, negm);
+            float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+            float2 pp_prev = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int c = h * 64 + 2 * i;
+              const float2 x = ffma2(make_float2(s[c], s[c + 1]), c2v, negv);
+              float2 pp;
+              if (((kFp8 ? kPolyMaskFp8 : kPolyMask) >> (i & 7)) & 1u) {
+                pp = exp2_poly2(x);
+              } else {
+                pp.x = ex2(x.x);
+                pp.y = ex2(x.y);
+              }
+              if constexpr (kMasked) {
+                pp.x = c < lim ? pp.x : 0.f;
+                pp.y = c + 1 < lim ? pp.y : 0.f;
+              }
+              if (i & 1) {
+                sb = fadd2(sb, pp);
+              } else {
+                sa = fadd2(sa, pp);
+              }
+              if constexpr (kFp8) {
+                if (i & 1) pk[i >> 1] = pack_e4m3x4(pp_prev.x, pp_prev.y, pp.x, pp.y);
+                pp_prev = pp;
+              } else {
+                pk[i] = pack_bf16x2(pp.x, pp.y);
+              }
+            }
+            return (sa.x + sb.x) + (sa.y + sb.y);
+          };
+          auto exp_half_any = [&](int h, float negm, uint32_t (&pk)[L::kPWords]) -> float {
+            return need_mask ? exp_half(std::true_type{}, h, negm, pk) : exp_half(std::false_type{}, h, negm, pk);
+          };
+
+          // row max of the tile, then the running max with a stale-max margin:
+          // the max is only moved (and O rescaled) when it grows by more than
+          // 2^8 in exp2 units; weights stay below 2^8 either way.
+          float mx;
+          {
+            float r0 = -INFINITY, r1 = -INFINITY, r2 = -INFINITY, r3 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 128; c += 8) {
+              r0 = fmax3(r0, s[c + 0], s[c + 1]);
+              r1 = fmax3(r1, s[c + 2], s[c + 3]);
+              r2 = fmax3(r2, s[c + 4], s[c + 5]);
+              r3 = fmax3(r3, s[c + 6], s[c + 7]);
+            }
+            mx = fmaxf(fmax3(r0, r1, r2), r3);
           }
-          if (i & 1) {
-            sb = fadd2(sb, pp);
-          } else {
-            sa = fadd2(sa, pp);
+          const float m_new = fmaxf(m, mx);
+          const bool upd = (m == -INFINITY) || ((m_new - m) * c2 > kRescaleLog2);
+          const float m_use = upd ? m_new : m;
+          const float alpha = (upd && m != -INFINITY) ? ex2((m - m_use) * c2) : (m == -INFINITY ? 0.f : 1.f);
+          const float negm = (m_use == -INFINITY) ? 0.f : -m_use * c2;
+          m = m_use;
+
+          // Rescale O before any of this tile's P.V lands on it.  The previous
+          // P.V has completed: the commit that signalled this S tile was issued
+          // after it and covers every earlier MMA.
+          if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t orr[32];
+              tmem_ld32(tO + c * 32, orr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+              tmem_st32(tO + c * 32, orr);
+            }
           }
-          if constexpr (kFp8) {
-            if (i & 1) pk[i >> 1] = pack_e4m3x4(pp_prev.x, pp_prev.y, pp.x, pp.y);
-            pp_prev = pp;
-          } else {
-            pk[i] = pack_bf16x2(pp.x, pp.y);
+
+          // P (bf16 pairs) into the first 64 columns of this tile's S region, one
+          // half (64 keys) at a time; the MMA warp starts P.V on the first half
+          // while the second is computed.
+          float psum;
+          {
+            uint32_t pk[L::kPWords];
+            psum = exp_half_any(0, negm, pk);
+            if constexpr (kFp8) tmem_st16(tS, pk); else tmem_st32(tS, pk);
           }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(BAR_PH(t));
+          {
+            uint32_t pk[L::kPWords];
+            psum += exp_half_any(1, negm, pk);
+            if constexpr (kFp8) tmem_st16(tS + L::kPWords, pk); else tmem_st32(tS + L::kPWords, pk);
+          }
+          l = alpha * l + psum;
+
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(BAR_PR(t));
         }
-        return (sa.x + sb.x) + (sa.y + sb.y);
-      };
-      auto exp_half_any = [&](int h, float negm, uint32_t (&pk)[L::kPWords]) -> float {
-        return need_mask ? exp_half(std::true_type{}, h, negm, pk) : exp_half(std::false_type{}, h, negm, pk);
-      };
 
-      // row max of the tile, then the running max with a stale-max margin:
-      // the max is only moved (and O rescaled) when it grows by more than
-      // 2^8 in exp2 units; weights stay below 2^8 either way.
-      float mx;
-      {
-        float r0 = -INFINITY, r1 = -INFINITY, r2 = -INFINITY, r3 = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 128; c += 8) {
-          r0 = fmax3(r0, s[c + 0], s[c + 1]);
-          r1 = fmax3(r1, s[c + 2], s[c + 3]);
-          r2 = fmax3(r2, s[c + 4], s[c + 5]);
-          r3 = fmax3(r3, s[c + 6], s[c + 7]);
+        // ---- epilogue: O / l -> bf16, lse = m * scale + ln(l)
+        const bool have = (n > 0) && ok;
+        if (have) {
+          ok = mbar_wait(BAR_OD(t), (steps + n - 1) & 1u, a.status, abort_flag);
+          ok = __all_sync(0xffffffffu, ok);
+          tc_fence_after();
         }
-        mx = fmaxf(fmax3(r0, r1, r2), r3);
-      }
-      const float m_new = fmaxf(m, mx);
-      const bool upd = (m == -INFINITY) || ((m_new - m) * c2 > kRescaleLog2);
-      const float m_use = upd ? m_new : m;
-      const float alpha = (upd && m != -INFINITY) ? ex2((m - m_use) * c2) : (m == -INFINITY ? 0.f : 1.f);
-      const float negm = (m_use == -INFINITY) ? 0.f : -m_use * c2;
-      m = m_use;
-
-      // Rescale O before any of this tile's P.V lands on it.  The previous
-      // P.V has completed: the commit that signalled this S tile was issued
-      // after it and covers every earlier MMA.
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        steps += static_cast<uint32_t>(n);
+        const bool store = qrow < Nq;
+        // output row: [B, Hq, Nq] (dense) or packed [total_q, Hq] (paged).  O
+        // leaves by 16-byte stores per thread: the Q buffer may already hold the
+        // next item's tiles.
+        const size_t orow = kPaged ? static_cast<size_t>(it.q_base + (store ? qrow : 0)) * a.Hq + hq
+                                   : (static_cast<size_t>(it.b) * a.Hq + hq) * Nq + qrow;
+        const float inv = (l > 0.f) ? (kFp8 ? a.v_descale / l : 1.f / l) : 0.f;
+        __nv_bfloat16* optr = a.o + orow * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t orr[32];
-          tmem_ld32(tO + c * 32, orr);
-          tmem_wait_ld();
+          if (have && ok) {
+            tmem_ld32(tO + c * 32, orr);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-          tmem_st32(tO + c * 32, orr);
-        }
-      }
-
-      // P (bf16 pairs) into the first 64 columns of this tile's S region, one
-      // half (64 keys) at a time; the MMA warp starts P.V on the first half
-      // while the second is computed.
-      float psum;
-      {
-        uint32_t pk[L::kPWords];
-        psum = exp_half_any(0, negm, pk);
-        if constexpr (kFp8) tmem_st16(tS, pk); else tmem_st32(tS, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(BAR_PH(t));
-      {
-        uint32_t pk[L::kPWords];
-        psum += exp_half_any(1, negm, pk);
-        if constexpr (kFp8) tmem_st16(tS + L::kPWords, pk); else tmem_st32(tS + L::kPWords, pk);
-      }
-      l = alpha * l + psum;
-
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(BAR_PR(t));
-    }
-
-    // ---- epilogue: O / l -> bf16, lse = m * scale + ln(l)
-    const bool have = (n > 0) && ok;
-    if (have) {
-      ok = mbar_wait(BAR_OD(t), (n - 1) & 1u, a.status, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      tc_fence_after();
-    }
-    const bool store = qrow < Nq;
-    // output row: [B, Hq, Nq] (dense) or packed [total_q, Hq] (paged)
-    const size_t orow = kPaged ? static_cast<size_t>(q_base + (store ? qrow : 0)) * a.Hq + hq
-                               : (static_cast<size_t>(b) * a.Hq + hq) * Nq + qrow;
-    const float inv = (l > 0.f) ? (kFp8 ? a.v_descale / l : 1.f / l) : 0.f;
-    if constexpr (kTmaStoreO) {
-      // O / l as bf16 into this tile's Q buffer, in the 128-byte-swizzled
-      // layout of the O tensor map's 64-column boxes, then one TMA store per
-      // box (rows past Nq are clipped by the map).  The Q buffer is free:
-      // this tile's last MMA has completed, or, with no K/V tile, its Q load
-      // has landed.
-      if (!have && q0 < Nq) mbar_wait(BAR_Q(), 0, a.status, abort_flag);
-      uint8_t* stage = smem + L::kQ + t * L::kTileBytes;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t orr[32];
-        if (have && ok) {
-          tmem_ld32(tO + c * 32, orr);
-          tmem_wait_ld();
-        } else {
+            for (int e = 0; e < 32; ++e) orr[e] = 0u;
+          }
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(optr + c * 32);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orr[e] = 0u;
-        }
-        uint8_t* rowp = stage + (c >> 1) * L::kChunkBytes + row * 128;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(orr[8 * e + 0]) * inv, __uint_as_float(orr[8 * e + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(orr[8 * e + 2]) * inv, __uint_as_float(orr[8 * e + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(orr[8 * e + 4]) * inv, __uint_as_float(orr[8 * e + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(orr[8 * e + 6]) * inv, __uint_as_float(orr[8 * e + 7]) * inv);
-          const int unit = (c & 1) * 4 + e;   // 16-byte unit of the 128-byte row, swizzled by row % 8
-          *reinterpret_cast<uint4*>(rowp + ((unit ^ (row & 7)) << 4)) = w;
-        }
-      }
-      fence_proxy_async_smem();
-      named_barrier_sync(1 + t, 128);
-      if (row == 0 && q0 < Nq) {
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_store_3d(&tmO, sQ + t * L::kTileBytes + c * L::kChunkBytes, c * L::kChunkElems, q0,
-                       b * a.Hq + hq);
-        bulk_commit_group();
-        bulk_wait_group_read0();   // the buffer must stay valid until the stores have read it
-      }
-    } else {
-      __nv_bfloat16* optr = a.o + orow * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t orr[32];
-        if (have && ok) {
-          tmem_ld32(tO + c * 32, orr);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) orr[e] = 0u;
-        }
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(optr + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(orr[8 * e + 0]) * inv, __uint_as_float(orr[8 * e + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(orr[8 * e + 2]) * inv, __uint_as_float(orr[8 * e + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(orr[8 * e + 4]) * inv, __uint_as_float(orr[8 * e + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(orr[8 * e + 6]) * inv, __uint_as_float(orr[8 * e + 7]) * inv);
-            dst[e] = w;
+            for (int e = 0; e < 4; ++e) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(orr[8 * e + 0]) * inv, __uint_as_float(orr[8 * e + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(orr[8 * e + 2]) * inv, __uint_as_float(orr[8 * e + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(orr[8 * e + 4]) * inv, __uint_as_float(orr[8 * e + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(orr[8 * e + 6]) * inv, __uint_as_float(orr[8 * e + 7]) * inv);
+              dst[e] = w;
+            }
           }
         }
-      }
-    }
-    if (store && a.lse) {
-      a.lse[orow] = (l > 0.f) ? fmaf(m, a.scale, __log2f(l) * 0.69314718055994531f) : -INFINITY;
-    }
+        // O_t has been read: the next item's first P.V may overwrite it
+        tc_fence_before();
+        mbar_arrive(BAR_OF(t));
+        if (store && a.lse) {
+          a.lse[orow] = (l > 0.f) ? fmaf(m, a.scale, __log2f(l) * 0.69314718055994531f) : -INFINITY;
+        }
+      }   // valid item
+      // the next item (or none)
+      if constexpr (!kPersistent) break;
+      const int kn = k + 1, sl = kn & 1;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(BAR_ITF(sl), resp_parity(kn), a.status, abort_flag));
+      if (!ok) break;
+      idx = clc_cancelled_ctaid_x(sResp + 16 * sl);
+      mbar_arrive(BAR_ITE(sl));
+    }   // items
   }
 
   // ---- teardown
@@ -680,8 +755,6 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   if ((st = encode_rows_3d(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
   if ((st = encode_rows_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
   if ((st = encode_rows_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
-  CUtensorMap to;   // O is stored through the same [B*Hq, Nq, d] box layout as Q
-  if ((st = encode_rows_3d(&to, o, D, Nq, B * Hq)) != TA_OK) return st;
   static int attr_done[64] = {0};
   cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, false, false>, L::kAlloc, attr_done);
   if (e != cudaSuccess) return fail(TA_ERR_CUDA, "prefill: shared-memory limit", e);
@@ -701,7 +774,7 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   a.status = device_status_ptr();
   if (!a.status) return fail(TA_ERR_CUDA, "prefill: device status word");
   const unsigned grid = static_cast<unsigned>(a.n_units) * static_cast<unsigned>(B * Hq / (a.head_pair + 1));
-  prefill_fwd_kernel<D, false, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, to, a);
+  prefill_fwd_kernel<D, false, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "prefill: launch", e);
 }
@@ -756,7 +829,7 @@ static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, cons
   a.max_pages = max_pages;
   a.num_pages_total = num_pages_total;
   const unsigned grid = static_cast<unsigned>(a.n_units) * static_cast<unsigned>(num_seqs * Hq / (a.head_pair + 1));
-  prefill_fwd_kernel<D, true, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, tq, a);
+  prefill_fwd_kernel<D, true, false><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "paged prefill: launch", e);
 }
@@ -802,7 +875,7 @@ ta_status launch_prefill_fp8(const void* q, const void* k, const void* v, float 
   a.status = device_status_ptr();
   if (!a.status) return fail(TA_ERR_CUDA, "fp8 prefill: device status word");
   const unsigned grid = static_cast<unsigned>(a.n_units) * static_cast<unsigned>(B * Hq / (a.head_pair + 1));
-  prefill_fwd_kernel<D, false, true><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, tq, a);
+  prefill_fwd_kernel<D, false, true><<<grid, kThreads, L::kAlloc, stream>>>(tq, tk, tv, a);
   e = cudaGetLastError();
   return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "fp8 prefill: launch", e);
 }

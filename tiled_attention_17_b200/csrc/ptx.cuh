@@ -130,27 +130,44 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint
       : "memory");
 }
 
-// Shared -> global tiled TMA store of one box (bulk-group completion); rows
-// and columns outside the tensor map's extent are not written.
-__device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int x, int y, int z) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(tmap)),
-               "r"(src), "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until the committed bulk stores have finished reading shared memory.
-__device__ __forceinline__ void bulk_wait_group_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// Make this thread's generic-proxy writes to shared memory visible to later
-// async-proxy operations (TMA stores).
+// Order this thread's earlier generic-proxy accesses to shared memory before
+// later async-proxy writes to it (TMA, cluster launch control responses).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// Barrier over `count` threads (a multiple of 32) with id 1-15.
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+
+// ----------------------------------------------------------------------------
+// Cluster launch control (sm_100): a running CTA takes over the work of a CTA
+// of the same grid that has not launched yet.
+// ----------------------------------------------------------------------------
+// Asks to cancel one not-yet-launched CTA; the 16-byte response lands at
+// `resp` (shared, 16-byte aligned) and completes 16 transaction bytes on
+// `bar`, which the caller armed with mbar_arrive_expect_tx(bar, 16).  Once a
+// response reports that nothing was cancelled, no further request may be made.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+  asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+                   resp),
+               "r"(bar)
+               : "memory");
+}
+// blockIdx.x of the CTA a response cancelled, or -1 if it cancelled none.
+__device__ __forceinline__ int clc_cancelled_ctaid_x(uint32_t resp) {
+  uint64_t lo, hi;
+  asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(lo), "=l"(hi) : "r"(resp) : "memory");
+  uint32_t cancelled;
+  asm volatile(
+      "{\n\t.reg .b128 R;\n\t.reg .pred P;\n\tmov.b128 R, {%1, %2};\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 P, R;\n\tselp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(cancelled)
+      : "l"(lo), "l"(hi));
+  if (!cancelled) return -1;
+  uint32_t x;
+  asm volatile(
+      "{\n\t.reg .b128 R;\n\tmov.b128 R, {%1, %2};\n\t"
+      "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %0, R;\n\t}"
+      : "=r"(x)
+      : "l"(lo), "l"(hi));
+  return static_cast<int>(x);
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
