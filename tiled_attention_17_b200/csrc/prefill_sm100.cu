@@ -182,8 +182,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int heads_per_item = a.head_pair ? 2 : 1;
     const int hx_count = a.Hq / heads_per_item;
     const int bh_count = (kPaged ? a.num_seqs : a.B) * hx_count;
-    const int unit = a.n_units - 1 - idx / bh_count;
-    const int bh = idx % bh_count;
+    // Dense: query units heaviest first across all heads (causal balance).
+    // Paged: stream-major, all units of one (sequence, head[s]) adjacent,
+    // heaviest first, so the CTAs running at once share one sequence's K/V
+    // in L2 (DRAM traffic 5.1 -> 1.1 GB on the chunked-prefill mix, about
+    // the algorithmic minimum) and its empty units come first and exit.
+    const int unit = kPaged ? a.n_units - 1 - idx % a.n_units : a.n_units - 1 - idx / bh_count;
+    const int bh = kPaged ? idx / a.n_units : idx % bh_count;
     it.b = bh / hx_count;                             // sequence when paged
     it.hq_0 = (bh % hx_count) * heads_per_item;      // query head of tile 0
     it.hq_1 = it.hq_0 + heads_per_item - 1;          // query head of tile 1
