@@ -105,6 +105,50 @@ __device__ __forceinline__ void mma_tmem_a(bool leader, uint32_t d_tmem, uint32_
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// P^T over 64 query columns of one key row: p_c = exp2(s_c c2 - lse2_c) as
+// bf16 pairs.  kMask zeroes the columns c < lo (causally hidden, or every
+// column of a key row past the keys).  The two forms are separate code
+// paths behind a warp-uniform branch: a compare-and-select per element on
+// every tile would cost more issue slots than the exponentials themselves.
+template <bool kMask>
+__device__ __forceinline__ void p_row_half(const float* sv, const float* l2v, float c2, int lo, uint32_t* pk) {
+#pragma unroll
+  for (int e4 = 0; e4 < 16; ++e4) {
+    const float4 l4 = *reinterpret_cast<const float4*>(l2v + 4 * e4);
+    const int c = 4 * e4;
+    float p0 = ex2(fmaf(sv[c + 0], c2, -l4.x)), p1 = ex2(fmaf(sv[c + 1], c2, -l4.y));
+    float p2 = ex2(fmaf(sv[c + 2], c2, -l4.z)), p3 = ex2(fmaf(sv[c + 3], c2, -l4.w));
+    if constexpr (kMask) {
+      p0 = c + 0 >= lo ? p0 : 0.f;
+      p1 = c + 1 >= lo ? p1 : 0.f;
+      p2 = c + 2 >= lo ? p2 : 0.f;
+      p3 = c + 3 >= lo ? p3 : 0.f;
+    }
+    pk[2 * e4] = pack_bf16x2(p0, p1);
+    pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
+  }
+}
+
+// dS over 64 key columns of one query row: P = exp2(s_c c2 - lse2), rounded
+// to bf16 as the dK/dV kernel rounds it, times (dP_c - delta).  kMask zeroes
+// the columns c >= lim (causally hidden or past the keys).
+template <bool kMask>
+__device__ __forceinline__ void ds_row_half(const float* sv, const float* dpv, float c2, float l2, float dl, int lim,
+                                            uint32_t* pk) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const int c = 2 * e;
+    float p0 = ex2(fmaf(sv[2 * e], c2, -l2));
+    float p1 = ex2(fmaf(sv[2 * e + 1], c2, -l2));
+    if constexpr (kMask) {
+      p0 = c < lim ? p0 : 0.f;
+      p1 = c + 1 < lim ? p1 : 0.f;
+    }
+    const uint32_t pb = pack_bf16x2(p0, p1);
+    pk[e] = pack_bf16x2(bf16lo(pb) * (dpv[2 * e] - dl), bf16hi(pb) * (dpv[2 * e + 1] - dl));
+  }
+}
+
 // ---------------------------------------------------------------------------
 // delta_i = dO_i . O_i and lse in log2 units per (padded) query row
 // ---------------------------------------------------------------------------
@@ -350,21 +394,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(tmem + L::kTmS + lane_off + h * 64 + 32, sr[1]);
         tmem_wait_ld();
         const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
-#pragma unroll
-        for (int e4 = 0; e4 < 16; ++e4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(l2v + 4 * e4);
-          const int c = 4 * e4;
-          float p0 = ex2(fmaf(sv[c + 0], c2, -l4.x)), p1 = ex2(fmaf(sv[c + 1], c2, -l4.y));
-          float p2 = ex2(fmaf(sv[c + 2], c2, -l4.z)), p3 = ex2(fmaf(sv[c + 3], c2, -l4.w));
-          if (need_mask) {
-            p0 = (row_ok && c + 0 >= lim) ? p0 : 0.f;
-            p1 = (row_ok && c + 1 >= lim) ? p1 : 0.f;
-            p2 = (row_ok && c + 2 >= lim) ? p2 : 0.f;
-            p3 = (row_ok && c + 3 >= lim) ? p3 : 0.f;
-          }
-          pk[2 * e4] = pack_bf16x2(p0, p1);
-          pk[2 * e4 + 1] = pack_bf16x2(p2, p3);
-        }
+        // lanes that need no mask have lim <= 0 and keep every column
+        if (__any_sync(0xffffffffu, need_mask))
+          p_row_half<true>(sv, l2v, c2, row_ok ? lim : 64, pk);
+        else
+          p_row_half<false>(sv, l2v, c2, 0, pk);
         tmem_st32(tmem + L::kTmS + lane_off + h * 64, pk);
       }
       tmem_wait_st();
@@ -653,19 +687,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive(BAR_LOADED);
         const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
         const float* dpv = reinterpret_cast<const float*>(&dr[0][0]);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = 2 * e;
-          float p0 = ex2(fmaf(sv[2 * e], c2, -l2));
-          float p1 = ex2(fmaf(sv[2 * e + 1], c2, -l2));
-          if (need_mask) {
-            p0 = c < lim ? p0 : 0.f;
-            p1 = c + 1 < lim ? p1 : 0.f;
-          }
-          // dS rounds P to bf16 first, as the dK/dV kernel does
-          const uint32_t pb = pack_bf16x2(p0, p1);
-          pk[e] = pack_bf16x2(bf16lo(pb) * (dpv[2 * e] - dl), bf16hi(pb) * (dpv[2 * e + 1] - dl));
-        }
+        if (need_mask)   // uniform across the CTA
+          ds_row_half<true>(sv, dpv, c2, l2, dl, lim, pk);
+        else
+          ds_row_half<false>(sv, dpv, c2, l2, dl, lim, pk);
       }
       // the previous dQ product must have read the dS buffer
       if (j > 0) {
