@@ -76,18 +76,26 @@ struct BwdArgs {
   unsigned* status;
 };
 
-// K-major operand tile (128 rows x D, 128-byte swizzle): descriptor of the
-// tile, +2 per 16-element step inside a 64-column chunk, +chunk to the next.
-__device__ __forceinline__ void mma_kmajor_tile(bool leader, uint32_t d_tmem, uint64_t a0, uint64_t b0, int chunks,
-                                                uint32_t idesc, bool acc) {
-#pragma unroll 1
-  for (int c = 0; c < chunks; ++c) {
+// The elected lane issues a whole product inside one branch: a branch per
+// MMA (the warp splitting and reconverging around every instruction) made
+// issue, at ~50 cycles per MMA, as slow as the tensor pipe executes a
+// 128 x 128 x 16 step, so the pipe sat idle between instructions.
+
+// D = A B^T with A, B K-major operand tiles (128 rows x D, 128-byte swizzle):
+// descriptor of the tile, +2 per 16-element step inside a 64-column chunk,
+// +chunk to the next.
+template <int kChunks>
+__device__ __forceinline__ void mma_kmajor_tile(bool leader, uint32_t d_tmem, uint64_t a0, uint64_t b0,
+                                                uint32_t idesc) {
+  if (leader) {
 #pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4)
-      if (leader) mma_ss(d_tmem, a0 + 2 * k4, b0 + 2 * k4, idesc, (acc || (c | k4) != 0));
-    a0 += (kT * 128) >> 4;
-    b0 += (kT * 128) >> 4;
+    for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4)
+        mma_ss(d_tmem, a0 + c * ((kT * 128) >> 4) + 2 * k4, b0 + c * ((kT * 128) >> 4) + 2 * k4, idesc,
+               (c | k4) != 0 ? 1u : 0u);
   }
+  __syncwarp();
 }
 
 // D += A B with A = 128 x 128 bf16 in TMEM (packed pairs: K = 0..63 in the 32
@@ -95,11 +103,14 @@ __device__ __forceinline__ void mma_kmajor_tile(bool leader, uint32_t d_tmem, ui
 // 128-row x D tile in shared memory (K = its rows).
 __device__ __forceinline__ void mma_tmem_a(bool leader, uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint64_t b0,
                                            uint32_t idesc, bool acc) {
+  if (leader) {
+    const uint32_t acc0 = acc ? 1u : 0u;
 #pragma unroll
-  for (int kk = 0; kk < kT / 16; ++kk)
-    if (leader)
+    for (int kk = 0; kk < kT / 16; ++kk)
       mma_ts(d_tmem, (kk < 4 ? a_lo : a_hi - 32) + kk * 8, b0 + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc,
-           (acc || kk > 0) ? 1u : 0u);
+             kk > 0 ? 1u : acc0);
+  }
+  __syncwarp();
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -327,9 +338,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) {
       tc_fence_after();
       // S^T = K Q^T and dP^T = V dO^T for the first item
-      mma_kmajor_tile(leader, tmem + L::kTmS, dK, dQk, T::kChunks, idesc_s, false);
+      mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dK, dQk, idesc_s);
       commit(BAR_SF);
-      mma_kmajor_tile(leader, tmem + L::kTmDP, dV, dDOk, T::kChunks, idesc_s, false);
+      mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dV, dDOk, idesc_s);
       commit(BAR_DPF);
     }
     for (int it = 0; it < n_items && ok; ++it) {
@@ -343,7 +354,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (it + 1 < n_items) {
         if (!(ok = mbar_wait_warp(BAR_QF(s1), ((it + 1) >> 1) & 1u, a.status, abort_flag))) break;
         tc_fence_after();
-        mma_kmajor_tile(leader, tmem + L::kTmS, dK, dQk + s1 * kStep, T::kChunks, idesc_s, false);
+        mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dK, dQk + s1 * kStep, idesc_s);
         commit(BAR_SF);
       }
       // dK += dS^T Q once dS^T is in TMEM
@@ -352,7 +363,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_tmem_a(leader, tmem + L::kTmDK, tmem + L::kTmDP, tmem + L::kTmDP + 64, dQm + s * kStep, idesc_acc, it > 0);
       commit(BAR_QE(s));   // this stage's Q, dO, lse and delta are read once these land
       if (it + 1 < n_items) {
-        mma_kmajor_tile(leader, tmem + L::kTmDP, dV, dDOk + s1 * kStep, T::kChunks, idesc_s, false);
+        mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dV, dDOk + s1 * kStep, idesc_s);
         commit(BAR_DPF);
       }
     }
@@ -619,9 +630,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     ok = ok && mbar_wait_warp(BAR_VF(0), 0, a.status, abort_flag);
     if (ok) {
       tc_fence_after();
-      mma_kmajor_tile(leader, tmem + L::kTmS, dQ, dKk, T::kChunks, idesc_s, false);     // S = Q K_0^T
+      mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dQ, dKk, idesc_s);     // S = Q K_0^T
       commit(BAR_SF);
-      mma_kmajor_tile(leader, tmem + L::kTmDP, dDO, dVk, T::kChunks, idesc_s, false);   // dP = dO V_0^T
+      mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dDO, dVk, idesc_s);   // dP = dO V_0^T
       commit(BAR_DPF);
       if (kSV < n) commit(BAR_VE(0));   // release a slot only when a later load reuses it
     }
@@ -634,11 +645,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!(ok = mbar_wait_warp(BAR_LOADED, ph, a.status, abort_flag))) break;
         if (!(ok = mbar_wait_warp(BAR_KF(sk1), phk1, a.status, abort_flag))) break;
         tc_fence_after();
-        mma_kmajor_tile(leader, tmem + L::kTmS, dQ, dKk + sk1 * kStep, T::kChunks, idesc_s, false);
+        mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dQ, dKk + sk1 * kStep, idesc_s);
         commit(BAR_SF);
         if (!(ok = mbar_wait_warp(BAR_VF(sv1), phv1, a.status, abort_flag))) break;
         tc_fence_after();
-        mma_kmajor_tile(leader, tmem + L::kTmDP, dDO, dVk + sv1 * kStep, T::kChunks, idesc_s, false);
+        mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dDO, dVk + sv1 * kStep, idesc_s);
         commit(BAR_DPF);
         if (j + 1 + kSV < n) commit(BAR_VE(sv1));
       }

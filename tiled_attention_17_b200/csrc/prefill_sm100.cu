@@ -385,12 +385,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool leader = elect_one_sync();
       constexpr uint32_t idesc_qk = kFp8 ? idesc_e4m3_f32(kBM, kBN, false) : idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = kFp8 ? idesc_e4m3_f32(kBM, D, true) : idesc_bf16_f32(kBM, D, true);
+      // The leader issues a whole product inside one branch: a branch around
+      // every MMA made issue about as slow as the tensor pipe's execution of
+      // a 128 x 128 x 16 step.
       auto mma_s = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
-        if (!leader) return;
         if constexpr (kFp8) mma_ss_f8(d, ad, bd, id, acc); else mma_ss(d, ad, bd, id, acc);
       };
       auto mma_t = [&](uint32_t d, uint32_t at, uint64_t bd, uint32_t id, uint32_t acc) {
-        if (!leader) return;
         if constexpr (kFp8) mma_ts_f8(d, at, bd, id, acc); else mma_ts(d, at, bd, id, acc);
       };
       // commits come from the lane that issued the MMAs they cover
@@ -416,14 +417,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d = tS(t);
         // K steps of 32 bytes (16 bf16 or 32 fp8 elements) within a 128-byte
         // swizzle row, then the next 128-byte chunk of d
+        if (leader) {
 #pragma unroll 1
-        for (int c = 0; c < L::kChunks; ++c) {
+          for (int c = 0; c < L::kChunks; ++c) {
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4)
-            mma_s(d, a0 + 2 * k4, b0 + 2 * k4, idesc_qk, (c | k4) != 0);
-          a0 += L::kChunkBytes >> 4;
-          b0 += L::kChunkBytes >> 4;
+            for (int k4 = 0; k4 < 4; ++k4)
+              mma_s(d, a0 + 2 * k4, b0 + 2 * k4, idesc_qk, (c | k4) != 0 ? 1u : 0u);
+            a0 += L::kChunkBytes >> 4;
+            b0 += L::kChunkBytes >> 4;
+          }
         }
+        __syncwarp();
       };
       // O_t += P_t V over one half (64 keys) of the tile, 16 (bf16) or 32
       // (fp8) keys per MMA (P from TMEM: 8 columns per step either way; V
@@ -432,12 +436,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kPerHalf = (kBN / 2) / L::kKeysPerMma;
         const uint64_t b0 = dV + static_cast<uint64_t>(s) * kTileStep;
         const uint32_t d = tO(t), a = tS(t);
+        if (leader) {
 #pragma unroll
-        for (int k4 = 0; k4 < kPerHalf; ++k4) {
-          const int kk = half * kPerHalf + k4;
-          mma_t(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * L::kKeysPerMma * 128) >> 4), idesc_pv,
-                (acc || kk > 0) ? 1u : 0u);
+          for (int k4 = 0; k4 < kPerHalf; ++k4) {
+            const int kk = half * kPerHalf + k4;
+            mma_t(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * L::kKeysPerMma * 128) >> 4), idesc_pv,
+                  (acc || kk > 0) ? 1u : 0u);
+          }
         }
+        __syncwarp();
       };
 
       bool ok = true;
