@@ -489,7 +489,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// dQ: one CTA per (query tile, batch, query head)
+// dQ: work items are (query tile, batch, query head), later query tiles
+// first.  A CTA runs its own item and then takes over the items of CTAs not
+// yet launched (cluster launch control: a successful try_cancel hands over
+// the cancelled CTA's index).  Its K/V ring and its S, dP and dS hand-offs
+// run on across items as one stream of key tiles: the next item's Q and dO
+// load as soon as the current item's last S and dP are issued, and the next
+// item's first S and dP follow the current item's last dQ product while the
+// work warps write that dQ out.  That overlaps each item's fixed cost (Q/dO
+// load latency, first products, dQ epilogue, CTA launch) with work.
 // ---------------------------------------------------------------------------
 template <int D>
 struct DqLayout {
@@ -502,10 +510,11 @@ struct DqLayout {
   static constexpr int kK = kDO + T::kTileBytes;
   static constexpr int kV = kK + kSK * T::kTileBytes;
   static constexpr int kBar = kV + kSV * T::kTileBytes;
-  // q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, loaded, dp_full, ds_full, ds_empty,
-  // acc_done
-  static constexpr int kNumBars = 17;
-  static constexpr int kMisc = kBar + kNumBars * 8;
+  // q_full, q_empty, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, loaded, dp_full, ds_full,
+  // ds_empty, acc_done, dq_empty, item_full[2], item_empty[2], fin
+  static constexpr int kNumBars = 2 + 2 * kSK + 2 * kSV + 7 + 4 + 1;
+  static constexpr int kResp = (kBar + kNumBars * 8 + 15) & ~15;   // two 16-byte work-request answers
+  static constexpr int kMisc = kResp + 32;
   static constexpr int kAlloc = kMisc + 16 + 1024;
   static_assert(kAlloc <= 232448, "dynamic shared memory per block");
   // TMEM: S | dP | dQ | dS (bf16, 64 columns)
@@ -532,32 +541,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sb = smem_u32(smem);
   const uint32_t sQ = sb + L::kQ, sDO = sb + L::kDO, sK = sb + L::kK, sV = sb + L::kV;
   const uint32_t bar0 = sb + L::kBar;
-  const uint32_t BAR_Q = bar0;
   constexpr int kSK = L::kSK, kSV = L::kSV;
-  auto BAR_KF = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto BAR_KE = [&](int s) { return bar0 + 8u * (1 + kSK + s); };
-  auto BAR_VF = [&](int s) { return bar0 + 8u * (1 + 2 * kSK + s); };
-  auto BAR_VE = [&](int s) { return bar0 + 8u * (1 + 2 * kSK + kSV + s); };
+  // q_empty: the item's last S and dP have read Q and dO
+  const uint32_t BAR_Q = bar0, BAR_QE = bar0 + 8u;
+  auto BAR_KF = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto BAR_KE = [&](int s) { return bar0 + 8u * (2 + kSK + s); };
+  auto BAR_VF = [&](int s) { return bar0 + 8u * (2 + 2 * kSK + s); };
+  auto BAR_VE = [&](int s) { return bar0 + 8u * (2 + 2 * kSK + kSV + s); };
   // loaded: S and dP of the current tile are in registers (both buffers may be
-  // overwritten); ds_empty: the dQ product has read the dS buffer
-  const uint32_t bar1 = bar0 + 8u * (1 + 2 * kSK + 2 * kSV);
+  // overwritten); ds_empty: the dQ product has read the dS buffer; dq_empty:
+  // the epilogue has read the dQ accumulator; item_full / item_empty: a work
+  // request's answer has landed / has been read by every consumer
+  const uint32_t bar1 = bar0 + 8u * (2 + 2 * kSK + 2 * kSV);
   const uint32_t BAR_SF = bar1, BAR_LOADED = bar1 + 8u, BAR_DPF = bar1 + 16u, BAR_DSF = bar1 + 24u,
-                 BAR_DSE = bar1 + 32u, BAR_ACC = bar1 + 40u;
+                 BAR_DSE = bar1 + 32u, BAR_ACC = bar1 + 40u, BAR_DQE = bar1 + 48u, BAR_FIN = bar1 + 88u;
+  auto BAR_ITF = [&](int s) { return bar1 + 56u + 8u * s; };
+  auto BAR_ITE = [&](int s) { return bar1 + 72u + 8u * s; };
+  const uint32_t sResp = sb + L::kResp;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // later query tiles (more visible keys under causal masking) first
+  struct Item {
+    int b, hq, hkv, bh, q0, n;
+  };
   const int bh_count = a.B * a.Hq;
-  const int qt = a.n_qt - 1 - static_cast<int>(blockIdx.x) / bh_count;
-  const int bh = static_cast<int>(blockIdx.x) % bh_count;
-  const int b = bh / a.Hq, hq = bh % a.Hq;
-  const int hkv = hq / (a.Hq / a.Hkv);
-  const int q0 = qt * kT;
-  const int n = key_tiles_for(q0, a);
+  auto decode_item = [&](int idx) {
+    Item it;
+    it.bh = idx % bh_count;
+    it.b = it.bh / a.Hq;
+    it.hq = it.bh % a.Hq;
+    it.hkv = it.hq / (a.Hq / a.Hkv);
+    it.q0 = (a.n_qt - 1 - idx / bh_count) * kT;
+    it.n = key_tiles_for(it.q0, a);
+    return it;
+  };
+  // Work request k >= 1 (the item after the k-th) answers in slot k & 1; it is
+  // that slot's ((k - 1) >> 1)-th use.
+  auto resp_parity = [](int k) { return static_cast<uint32_t>((k - 1) >> 1) & 1u; };
 
   if (threadIdx.x == 0) {
     mbar_init(BAR_Q, 1);
+    mbar_init(BAR_QE, 1);
     for (int s = 0; s < kSK; ++s) {
       mbar_init(BAR_KF(s), 1);
       mbar_init(BAR_KE(s), 1);
@@ -572,6 +597,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(BAR_DSF, 256);
     mbar_init(BAR_DSE, 1);
     mbar_init(BAR_ACC, 1);
+    mbar_init(BAR_DQE, 256);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR_ITF(s), 1);
+      mbar_init(BAR_ITE(s), 1 + 256);   // the MMA warp's leader and every work thread
+    }
+    mbar_init(BAR_FIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -591,26 +622,64 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
   if (warp < kWorkWarp0) {
   setmaxnreg_dec<kBwdRegsControl>();
-  if (n > 0 && warp == 0 && lane == 0) {
+  if (warp == 0 && lane == 0) {
     // ======================= TMA producer =======================
-    const int zq = b * a.Hq + hq, zk = b * a.Hkv + hkv;
-    mbar_arrive_expect_tx(BAR_Q, 2 * T::kTileBytes);
-    for (int c = 0; c < T::kChunks; ++c) {
-      tma_load_3d(sQ + c * T::kChunkBytes, &tmQ, BAR_Q, c * 64, q0, zq);
-      tma_load_3d(sDO + c * T::kChunkBytes, &tmDO, BAR_Q, c * 64, q0, zq);
+    bool ok = true;
+    uint32_t gk = 0, gv = 0;   // K and V tiles loaded so far: ring slot g % slots, use g / slots
+    int qi = 0;                // items whose Q and dO were loaded
+    int requested = 0, answered = 0;
+    int idx = static_cast<int>(blockIdx.x);
+    for (int k = 0; idx >= 0 && ok; ++k) {
+      // ask for the item after this one now, so the answer is back when it is needed
+      {
+        const int kn = k + 1, sl = kn & 1;
+        if (kn >= 3 && !(ok = mbar_wait(BAR_ITE(sl), resp_parity(kn - 2), a.status, abort_flag))) break;
+        fence_proxy_async_smem();   // the slot's previous answer was read through the generic proxy
+        mbar_arrive_expect_tx(BAR_ITF(sl), 16);
+        clc_try_cancel(sResp + 16 * sl, BAR_ITF(sl));
+        requested = kn;
+      }
+      const Item it = decode_item(idx);
+      if (it.n > 0) {
+        // the Q/dO buffer is free once the previous item's last S and dP completed
+        if (qi > 0 && !(ok = mbar_wait(BAR_QE, static_cast<uint32_t>(qi - 1) & 1u, a.status, abort_flag))) break;
+        const int zq = it.b * a.Hq + it.hq, zk = it.b * a.Hkv + it.hkv;
+        mbar_arrive_expect_tx(BAR_Q, 2 * T::kTileBytes);
+        for (int c = 0; c < T::kChunks; ++c) {
+          tma_load_3d(sQ + c * T::kChunkBytes, &tmQ, BAR_Q, c * 64, it.q0, zq);
+          tma_load_3d(sDO + c * T::kChunkBytes, &tmDO, BAR_Q, c * 64, it.q0, zq);
+        }
+        ++qi;
+        for (int j = 0; j < it.n; ++j) {
+          const int sk = static_cast<int>(gk % kSK), sv = static_cast<int>(gv % kSV);
+          if (!(ok = mbar_wait(BAR_KE(sk), ((gk / kSK) & 1u) ^ 1u, a.status, abort_flag))) break;
+          mbar_arrive_expect_tx(BAR_KF(sk), T::kTileBytes);
+          for (int c = 0; c < T::kChunks; ++c)
+            tma_load_3d(sK + sk * T::kTileBytes + c * T::kChunkBytes, &tmK, BAR_KF(sk), c * 64, j * kT, zk);
+          ++gk;
+          if (!(ok = mbar_wait(BAR_VE(sv), ((gv / kSV) & 1u) ^ 1u, a.status, abort_flag))) break;
+          mbar_arrive_expect_tx(BAR_VF(sv), T::kTileBytes);
+          for (int c = 0; c < T::kChunks; ++c)
+            tma_load_3d(sV + sv * T::kTileBytes + c * T::kChunkBytes, &tmV, BAR_VF(sv), c * 64, j * kT, zk);
+          ++gv;
+        }
+        if (!ok) break;
+      }
+      // the next item (or none)
+      const int kn = k + 1, sl = kn & 1;
+      if (!(ok = mbar_wait(BAR_ITF(sl), resp_parity(kn), a.status, abort_flag))) break;
+      answered = kn;
+      idx = clc_cancelled_ctaid_x(sResp + 16 * sl);
     }
-    for (int j = 0; j < n; ++j) {
-      const int sk = j % kSK, sv = j % kSV;
-      if (!mbar_wait(BAR_KE(sk), ((j / kSK) & 1u) ^ 1u, a.status, abort_flag)) break;
-      mbar_arrive_expect_tx(BAR_KF(sk), T::kTileBytes);
-      for (int c = 0; c < T::kChunks; ++c)
-        tma_load_3d(sK + sk * T::kTileBytes + c * T::kChunkBytes, &tmK, BAR_KF(sk), c * 64, j * kT, zk);
-      if (!mbar_wait(BAR_VE(sv), ((j / kSV) & 1u) ^ 1u, a.status, abort_flag)) break;
-      mbar_arrive_expect_tx(BAR_VF(sv), T::kTileBytes);
-      for (int c = 0; c < T::kChunks; ++c)
-        tma_load_3d(sV + sv * T::kTileBytes + c * T::kChunkBytes, &tmV, BAR_VF(sv), c * 64, j * kT, zk);
-    }
-  } else if (n > 0 && warp == 1) {
+    // drain: no copy into this CTA's shared memory may still be in flight at exit
+    if (answered < requested)
+      mbar_wait(BAR_ITF(requested & 1), resp_parity(requested), nullptr, nullptr, kWaitLimitNs);
+    if (qi > 0) mbar_wait(BAR_Q, static_cast<uint32_t>(qi - 1) & 1u, nullptr, nullptr, kWaitLimitNs);
+    for (uint32_t g = (gk > static_cast<uint32_t>(kSK) ? gk - kSK : 0u); g < gk; ++g)
+      mbar_wait(BAR_KF(static_cast<int>(g % kSK)), (g / kSK) & 1u, nullptr, nullptr, kWaitLimitNs);
+    for (uint32_t g = (gv > static_cast<uint32_t>(kSV) ? gv - kSV : 0u); g < gv; ++g)
+      mbar_wait(BAR_VF(static_cast<int>(g % kSV)), (g / kSV) & 1u, nullptr, nullptr, kWaitLimitNs);
+  } else if (warp == 1) {
     // ======================= MMA issuer =======================
     // The whole warp runs the issue loop (warp-uniform descriptors and
     // waits); the elected lane issues the MMAs and their commits.
@@ -625,42 +694,72 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t dKk = smem_desc_sw128(sK, 16, 1024), dVk = smem_desc_sw128(sV, 16, 1024);
     const uint64_t dKm = smem_desc_sw128(sK, T::kChunkBytes, 1024);
     constexpr uint64_t kStep = T::kTileBytes >> 4;
-    bool ok = mbar_wait_warp(BAR_Q, 0, a.status, abort_flag);
-    ok = ok && mbar_wait_warp(BAR_KF(0), 0, a.status, abort_flag);
-    ok = ok && mbar_wait_warp(BAR_VF(0), 0, a.status, abort_flag);
-    if (ok) {
+    // S = Q K^T and dP = dO V^T of the key tile in ring positions (gkk, gvv)
+    auto issue_s_dp = [&](uint32_t gkk, uint32_t gvv) -> bool {
+      const int sk = static_cast<int>(gkk % kSK), sv = static_cast<int>(gvv % kSV);
+      if (!mbar_wait_warp(BAR_KF(sk), (gkk / kSK) & 1u, a.status, abort_flag)) return false;
       tc_fence_after();
-      mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dQ, dKk, idesc_s);     // S = Q K_0^T
+      mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dQ, dKk + sk * kStep, idesc_s);
       commit(BAR_SF);
-      mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dDO, dVk, idesc_s);   // dP = dO V_0^T
-      commit(BAR_DPF);
-      if (kSV < n) commit(BAR_VE(0));   // release a slot only when a later load reuses it
-    }
-    for (int j = 0; j < n && ok; ++j) {
-      const int sk = j % kSK, sk1 = (j + 1) % kSK, sv1 = (j + 1) % kSV;
-      const uint32_t ph = j & 1u;
-      const uint32_t phk1 = ((j + 1) / kSK) & 1u, phv1 = ((j + 1) / kSV) & 1u;
-      // next S and dP as soon as the work warps hold this tile's in registers
-      if (j + 1 < n) {
-        if (!(ok = mbar_wait_warp(BAR_LOADED, ph, a.status, abort_flag))) break;
-        if (!(ok = mbar_wait_warp(BAR_KF(sk1), phk1, a.status, abort_flag))) break;
-        tc_fence_after();
-        mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dQ, dKk + sk1 * kStep, idesc_s);
-        commit(BAR_SF);
-        if (!(ok = mbar_wait_warp(BAR_VF(sv1), phv1, a.status, abort_flag))) break;
-        tc_fence_after();
-        mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dDO, dVk + sv1 * kStep, idesc_s);
-        commit(BAR_DPF);
-        if (j + 1 + kSV < n) commit(BAR_VE(sv1));
-      }
-      // dQ += dS K_j once dS is in its buffer
-      if (!(ok = mbar_wait_warp(BAR_DSF, ph, a.status, abort_flag))) break;
+      if (!mbar_wait_warp(BAR_VF(sv), (gvv / kSV) & 1u, a.status, abort_flag)) return false;
       tc_fence_after();
-      mma_tmem_a(leader, tmem + L::kTmDQ, tmem + L::kTmDS, tmem + L::kTmDS + 32, dKm + sk * kStep, idesc_acc, j > 0);
-      commit(BAR_DSE);
-      if (j + kSK < n) commit(BAR_KE(sk));
+      mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dDO, dVk + sv * kStep, idesc_s);
+      commit(BAR_DPF);
+      commit(BAR_VE(sv));   // V_j is read by dP_j only
+      return true;
+    };
+    bool ok = true;
+    uint32_t t = 0;            // key tiles of this CTA so far (S/dP/dS hand-off phases)
+    uint32_t gk = 0, gv = 0;   // K/V ring positions, as the producer's
+    int qi = 0;                // items with keys so far
+    int idx = static_cast<int>(blockIdx.x);
+    for (int k = 0; idx >= 0 && ok; ++k) {
+      const Item it = decode_item(idx);
+      if (it.n > 0) {
+        // the first tile's S and dP: the previous tile's are in registers and
+        // this item's Q and dO have landed
+        if (t > 0 && !(ok = mbar_wait_warp(BAR_LOADED, (t - 1) & 1u, a.status, abort_flag))) break;
+        if (!(ok = mbar_wait_warp(BAR_Q, static_cast<uint32_t>(qi) & 1u, a.status, abort_flag))) break;
+        if (!(ok = issue_s_dp(gk, gv))) break;
+        if (it.n == 1) commit(BAR_QE);
+        for (int j = 0; j < it.n; ++j) {
+          const uint32_t tj = t + static_cast<uint32_t>(j), gkj = gk + static_cast<uint32_t>(j);
+          // next S and dP as soon as the work warps hold this tile's in registers
+          if (j + 1 < it.n) {
+            if (!(ok = mbar_wait_warp(BAR_LOADED, tj & 1u, a.status, abort_flag))) break;
+            if (!(ok = issue_s_dp(gkj + 1, gv + static_cast<uint32_t>(j) + 1))) break;
+            if (j + 2 == it.n) commit(BAR_QE);   // the item's last S and dP: Q and dO are free
+          }
+          // dQ += dS K_j once dS is in its buffer; an item's first product
+          // overwrites the accumulator, which the previous epilogue must have read
+          if (!(ok = mbar_wait_warp(BAR_DSF, tj & 1u, a.status, abort_flag))) break;
+          if (j == 0 && qi > 0 &&
+              !(ok = mbar_wait_warp(BAR_DQE, static_cast<uint32_t>(qi - 1) & 1u, a.status, abort_flag)))
+            break;
+          tc_fence_after();
+          const int sk = static_cast<int>(gkj % kSK);
+          mma_tmem_a(leader, tmem + L::kTmDQ, tmem + L::kTmDS, tmem + L::kTmDS + 32, dKm + sk * kStep, idesc_acc,
+                     j > 0);
+          commit(BAR_DSE);
+          commit(BAR_KE(sk));   // K_j is read by S_j and dQ_j
+        }
+        if (!ok) break;
+        commit(BAR_ACC);
+        t += static_cast<uint32_t>(it.n);
+        gk += static_cast<uint32_t>(it.n);
+        gv += static_cast<uint32_t>(it.n);
+        ++qi;
+      }
+      // the next item (or none)
+      const int kn = k + 1, sl = kn & 1;
+      if (!(ok = mbar_wait_warp(BAR_ITF(sl), resp_parity(kn), a.status, abort_flag))) break;
+      idx = clc_cancelled_ctaid_x(sResp + 16 * sl);
+      __syncwarp();
+      if (leader) mbar_arrive(BAR_ITE(sl));
     }
-    if (ok) commit(BAR_ACC);
+    // no commit may still be pending when the CTA exits
+    commit(BAR_FIN);
+    mbar_wait_warp(BAR_FIN, 0, nullptr, nullptr);
   }
   } else {
     setmaxnreg_inc<kBwdRegsWork>();
@@ -668,83 +767,104 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int h = (warp - kWorkWarp0) / 4;         // key columns [64h, 64h + 64) of each tile
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int qrow = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float c2 = a.scale_log2;
-    const size_t vrow = static_cast<size_t>(bh) * (a.n_qt * kT) + qrow;   // padded rows exist for every r
-    const float l2 = a.lse2[vrow], dl = a.delta[vrow];
-    const int vis_end = a.causal ? min(a.Nkv, qrow + (a.Nkv - a.Nq) + 1) : a.Nkv;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const uint32_t ph = j & 1u;
-      ok = mbar_wait(BAR_SF, ph, a.status, abort_flag);
-      ok = ok && mbar_wait(BAR_DPF, ph, a.status, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const int lim = vis_end - j * kT - h * 64;   // visible key columns of this half: [0, lim)
-      const bool need_mask = (j * kT + kT > a.Nkv) || (a.causal && j * kT + kT - 1 > q0 + (a.Nkv - a.Nq));
-      uint32_t pk[32];
-      {
-        uint32_t sr[2][32], dr[2][32];
-        tmem_ld32(tmem + L::kTmS + lane_off + h * 64, sr[0]);
-        tmem_ld32(tmem + L::kTmS + lane_off + h * 64 + 32, sr[1]);
-        tmem_ld32(tmem + L::kTmDP + lane_off + h * 64, dr[0]);
-        tmem_ld32(tmem + L::kTmDP + lane_off + h * 64 + 32, dr[1]);
-        tmem_wait_ld();
-        // this half of S and dP is in registers: the next tile's products may
-        // overwrite both buffers once the other half has read its part too
+    uint32_t t = 0;   // key tiles of this CTA so far
+    int qi = 0;       // items with keys so far
+    int idx = static_cast<int>(blockIdx.x);
+    for (int k = 0; idx >= 0; ++k) {
+      const Item it = decode_item(idx);
+      const int q0 = it.q0, n = it.n;
+      const int qrow = q0 + r;
+      const size_t vrow = static_cast<size_t>(it.bh) * (a.n_qt * kT) + qrow;   // padded rows exist for every r
+      const float l2 = a.lse2[vrow], dl = a.delta[vrow];
+      const int vis_end = a.causal ? min(a.Nkv, qrow + (a.Nkv - a.Nq) + 1) : a.Nkv;
+      for (int j = 0; j < n && ok; ++j) {
+        const uint32_t tj = t + static_cast<uint32_t>(j);
+        const uint32_t ph = tj & 1u;
+        ok = mbar_wait(BAR_SF, ph, a.status, abort_flag);
+        ok = ok && mbar_wait(BAR_DPF, ph, a.status, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const int lim = vis_end - j * kT - h * 64;   // visible key columns of this half: [0, lim)
+        const bool need_mask = (j * kT + kT > a.Nkv) || (a.causal && j * kT + kT - 1 > q0 + (a.Nkv - a.Nq));
+        uint32_t pk[32];
+        {
+          uint32_t sr[2][32], dr[2][32];
+          tmem_ld32(tmem + L::kTmS + lane_off + h * 64, sr[0]);
+          tmem_ld32(tmem + L::kTmS + lane_off + h * 64 + 32, sr[1]);
+          tmem_ld32(tmem + L::kTmDP + lane_off + h * 64, dr[0]);
+          tmem_ld32(tmem + L::kTmDP + lane_off + h * 64 + 32, dr[1]);
+          tmem_wait_ld();
+          // this half of S and dP is in registers: the next tile's products may
+          // overwrite both buffers once the other half has read its part too
+          tc_fence_before();
+          mbar_arrive(BAR_LOADED);
+          const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+          const float* dpv = reinterpret_cast<const float*>(&dr[0][0]);
+          if (need_mask)   // uniform across the CTA
+            ds_row_half<true>(sv, dpv, c2, l2, dl, lim, pk);
+          else
+            ds_row_half<false>(sv, dpv, c2, l2, dl, lim, pk);
+        }
+        // the previous dQ product (of this or an earlier item) must have read the dS buffer
+        if (tj > 0) {
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_DSE, (tj - 1) & 1u, a.status, abort_flag)))) break;
+          tc_fence_after();
+        }
+        tmem_st32(tmem + L::kTmDS + lane_off + h * 32, pk);
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR_LOADED);
-        const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
-        const float* dpv = reinterpret_cast<const float*>(&dr[0][0]);
-        if (need_mask)   // uniform across the CTA
-          ds_row_half<true>(sv, dpv, c2, l2, dl, lim, pk);
-        else
-          ds_row_half<false>(sv, dpv, c2, l2, dl, lim, pk);
+        mbar_arrive(BAR_DSF);
       }
-      // the previous dQ product must have read the dS buffer
-      if (j > 0) {
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_DSE, (j - 1) & 1u, a.status, abort_flag)))) break;
+      t += static_cast<uint32_t>(n);
+      // ---- epilogue: dQ (times scale); a query tile that sees no key gets zeros
+      const bool have = ok && n > 0;
+      if (have) {
+        ok = __all_sync(0xffffffffu, mbar_wait(BAR_ACC, static_cast<uint32_t>(qi) & 1u, a.status, abort_flag));
         tc_fence_after();
       }
-      tmem_st32(tmem + L::kTmDS + lane_off + h * 32, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(BAR_DSF);
-    }
-    // ---- epilogue: dQ (times scale)
-    const bool have = ok && n > 0;
-    if (have) {
-      ok = __all_sync(0xffffffffu, mbar_wait(BAR_ACC, 0, a.status, abort_flag));
-      tc_fence_after();
-    }
-    // TMEM loads are warp-collective: every lane loads, only rows < Nq store
-    const bool store = qrow < a.Nq;
-    // this warpgroup's half of the row: columns [h D/2, (h+1) D/2)
-    __nv_bfloat16* dst_row = a.dq + (static_cast<size_t>(bh) * a.Nq + (store ? qrow : 0)) * D + h * (D / 2);
+      // TMEM loads are warp-collective: every lane loads, only rows < Nq store
+      const bool store = qrow < a.Nq;
+      // this warpgroup's half of the row: columns [h D/2, (h+1) D/2)
+      __nv_bfloat16* dst_row = a.dq + (static_cast<size_t>(it.bh) * a.Nq + (store ? qrow : 0)) * D + h * (D / 2);
 #pragma unroll 1
-    for (int c = 0; c < D / 64; ++c) {
-      uint32_t v[32];
-      if (have && ok) {
-        tmem_ld32(tmem + L::kTmDQ + lane_off + h * (D / 2) + c * 32, v);
-        tmem_wait_ld();
-      } else {
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t v[32];
+        if (have && ok) {
+          tmem_ld32(tmem + L::kTmDQ + lane_off + h * (D / 2) + c * 32, v);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0u;
-      }
-      if (store) {
-        uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * a.scale, __uint_as_float(v[8 * e + 1]) * a.scale);
-          w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * a.scale, __uint_as_float(v[8 * e + 3]) * a.scale);
-          w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * a.scale, __uint_as_float(v[8 * e + 5]) * a.scale);
-          w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * a.scale, __uint_as_float(v[8 * e + 7]) * a.scale);
-          dst[e] = w;
+          for (int e = 0; e < 4; ++e) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * a.scale, __uint_as_float(v[8 * e + 1]) * a.scale);
+            w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * a.scale, __uint_as_float(v[8 * e + 3]) * a.scale);
+            w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * a.scale, __uint_as_float(v[8 * e + 5]) * a.scale);
+            w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * a.scale, __uint_as_float(v[8 * e + 7]) * a.scale);
+            dst[e] = w;
+          }
         }
       }
+      if (n > 0) {
+        // the accumulator has been read: the next item's first dQ product may overwrite it
+        tc_fence_before();
+        mbar_arrive(BAR_DQE);
+        ++qi;
+      }
+      if (!ok) break;
+      // the next item (or none)
+      const int kn = k + 1, sl = kn & 1;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_ITF(sl), resp_parity(kn), a.status, abort_flag)))) break;
+      idx = clc_cancelled_ctaid_x(sResp + 16 * sl);
+      mbar_arrive(BAR_ITE(sl));
     }
   }
 
