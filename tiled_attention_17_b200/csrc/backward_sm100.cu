@@ -205,7 +205,14 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 }
 
 // ---------------------------------------------------------------------------
-// dK, dV: one CTA per (key tile, batch, KV head)
+// dK, dV: work items are (key tile, batch, KV head), key tiles that more
+// query tiles see first.  As in the dQ kernel, a CTA runs its own item and
+// then takes over the items of CTAs not yet launched (cluster launch
+// control).  The Q/dO ring and the S, P, dP and dS hand-offs run on across
+// items as one stream of (query head, query tile) pairs: the next key tile's
+// K and V load as soon as the current tile's last S^T and dP^T are issued,
+// and its first S^T and dP^T follow the current tile's last dV and dK while
+// the work warps write dK and dV out.
 // ---------------------------------------------------------------------------
 template <int D>
 struct DkdvLayout {
@@ -216,9 +223,11 @@ struct DkdvLayout {
   static constexpr int kDO = kQ + 2 * T::kTileBytes;         // 2 stages
   static constexpr int kVec = kDO + 2 * T::kTileBytes;       // 2 stages x {lse2, delta} x 128 floats
   static constexpr int kBar = kVec + 2 * 2 * kT * 4;
-  // kv_full, q_full[2], q_empty[2], s_full, p_full, dp_full, ds_full, acc_done
-  static constexpr int kNumBars = 10;
-  static constexpr int kMisc = kBar + kNumBars * 8;
+  // kv_full, kv_empty, q_full[2], q_empty[2], s_full, p_full, dp_full, ds_full, acc_done, acc_empty,
+  // item_full[2], item_empty[2], fin
+  static constexpr int kNumBars = 17;
+  static constexpr int kResp = (kBar + kNumBars * 8 + 15) & ~15;   // two 16-byte work-request answers
+  static constexpr int kMisc = kResp + 32;
   static constexpr int kAlloc = kMisc + 16 + 1024;
   static_assert(kAlloc <= 232448, "dynamic shared memory per block");
   // TMEM: S^T | dP^T | dV | dK
@@ -247,36 +256,58 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sK = sb + L::kK, sV = sb + L::kV, sQ = sb + L::kQ, sDO = sb + L::kDO;
   const float* vec = reinterpret_cast<const float*>(smem + L::kVec);
   const uint32_t bar0 = sb + L::kBar;
-  const uint32_t BAR_KV = bar0;
-  auto BAR_QF = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto BAR_QE = [&](int s) { return bar0 + 8u * (3 + s); };
-  const uint32_t BAR_SF = bar0 + 8u * 5, BAR_PF = bar0 + 8u * 6, BAR_DPF = bar0 + 8u * 7,
-                 BAR_DSF = bar0 + 8u * 8, BAR_ACC = bar0 + 8u * 9;
+  // kv_empty: the key tile's last S^T and dP^T have read K and V; acc_empty:
+  // the epilogue has read dV and dK; item_full / item_empty: a work request's
+  // answer has landed / has been read by every consumer
+  const uint32_t BAR_KV = bar0, BAR_KVE = bar0 + 8u;
+  auto BAR_QF = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto BAR_QE = [&](int s) { return bar0 + 8u * (4 + s); };
+  const uint32_t BAR_SF = bar0 + 8u * 6, BAR_PF = bar0 + 8u * 7, BAR_DPF = bar0 + 8u * 8,
+                 BAR_DSF = bar0 + 8u * 9, BAR_ACC = bar0 + 8u * 10, BAR_ACCE = bar0 + 8u * 11,
+                 BAR_FIN = bar0 + 8u * 16;
+  auto BAR_ITF = [&](int s) { return bar0 + 8u * (12 + s); };
+  auto BAR_ITE = [&](int s) { return bar0 + 8u * (14 + s); };
+  const uint32_t sResp = sb + L::kResp;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // key tiles that more query tiles see come first (causal: the early ones)
   const int bh_count = a.B * a.Hkv;
-  const int kt = static_cast<int>(blockIdx.x) / bh_count;
-  const int bhk = static_cast<int>(blockIdx.x) % bh_count;
-  const int b = bhk / a.Hkv, hkv = bhk % a.Hkv;
   const int G = a.Hq / a.Hkv;
-  const int i0 = first_query_tile(kt, a);
-  const int per_head = i0 < a.n_qt ? a.n_qt - i0 : 0;
-  const int n_items = G * per_head;   // (query head of the group, query tile) pairs
+  struct Item {
+    int kt, b, hkv, i0, per_head, n;   // n: (query head of the group, query tile) pairs
+  };
+  auto decode_item = [&](int idx) {
+    Item it;
+    it.kt = idx / bh_count;
+    const int bhk = idx % bh_count;
+    it.b = bhk / a.Hkv;
+    it.hkv = bhk % a.Hkv;
+    it.i0 = first_query_tile(it.kt, a);
+    it.per_head = it.i0 < a.n_qt ? a.n_qt - it.i0 : 0;
+    it.n = G * it.per_head;
+    return it;
+  };
+  // Work request k >= 1 (the item after the k-th) answers in slot k & 1; it is
+  // that slot's ((k - 1) >> 1)-th use.
+  auto resp_parity = [](int k) { return static_cast<uint32_t>((k - 1) >> 1) & 1u; };
 
   if (threadIdx.x == 0) {
     mbar_init(BAR_KV, 1);
+    mbar_init(BAR_KVE, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR_QF(s), 1);
       mbar_init(BAR_QE(s), 1);
+      mbar_init(BAR_ITF(s), 1);
+      mbar_init(BAR_ITE(s), 1 + 256);   // the MMA warp's leader and every work thread
     }
     mbar_init(BAR_SF, 1);
     mbar_init(BAR_PF, 256);
     mbar_init(BAR_DPF, 1);
     mbar_init(BAR_DSF, 256);
     mbar_init(BAR_ACC, 1);
+    mbar_init(BAR_ACCE, 256);
+    mbar_init(BAR_FIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -296,29 +327,64 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
   if (warp < kWorkWarp0) {
   setmaxnreg_dec<kBwdRegsControl>();
-  if (n_items > 0 && warp == 0 && lane == 0) {
+  if (warp == 0 && lane == 0) {
     // ======================= TMA producer =======================
-    const int zk = b * a.Hkv + hkv;
-    mbar_arrive_expect_tx(BAR_KV, 2 * T::kTileBytes);
-    for (int c = 0; c < T::kChunks; ++c) {
-      tma_load_3d(sK + c * T::kChunkBytes, &tmK, BAR_KV, c * 64, kt * kT, zk);
-      tma_load_3d(sV + c * T::kChunkBytes, &tmV, BAR_KV, c * 64, kt * kT, zk);
-    }
-    for (int it = 0; it < n_items; ++it) {
-      const int s = it & 1;
-      if (!mbar_wait(BAR_QE(s), ((it >> 1) & 1u) ^ 1u, a.status, abort_flag)) break;
-      const int hq = hkv * G + it / per_head, qt = i0 + it % per_head;
-      const int zq = b * a.Hq + hq;
-      mbar_arrive_expect_tx(BAR_QF(s), 2 * T::kTileBytes + 2 * kT * 4);
-      for (int c = 0; c < T::kChunks; ++c) {
-        tma_load_3d(sQ + s * T::kTileBytes + c * T::kChunkBytes, &tmQ, BAR_QF(s), c * 64, qt * kT, zq);
-        tma_load_3d(sDO + s * T::kTileBytes + c * T::kChunkBytes, &tmDO, BAR_QF(s), c * 64, qt * kT, zq);
+    bool ok = true;
+    uint32_t u = 0;   // (query head, query tile) pairs loaded so far: ring stage u & 1, use u >> 1
+    int qi = 0;       // key tiles whose K and V were loaded
+    int requested = 0, answered = 0;
+    int idx = static_cast<int>(blockIdx.x);
+    for (int k = 0; idx >= 0 && ok; ++k) {
+      // ask for the item after this one now, so the answer is back when it is needed
+      {
+        const int kn = k + 1, sl = kn & 1;
+        if (kn >= 3 && !(ok = mbar_wait(BAR_ITE(sl), resp_parity(kn - 2), a.status, abort_flag))) break;
+        fence_proxy_async_smem();   // the slot's previous answer was read through the generic proxy
+        mbar_arrive_expect_tx(BAR_ITF(sl), 16);
+        clc_try_cancel(sResp + 16 * sl, BAR_ITF(sl));
+        requested = kn;
       }
-      const size_t vrow = static_cast<size_t>(zq) * (a.n_qt * kT) + qt * kT;
-      bulk_load(sb + L::kVec + (s * 2 + 0) * kT * 4, a.lse2 + vrow, kT * 4, BAR_QF(s));
-      bulk_load(sb + L::kVec + (s * 2 + 1) * kT * 4, a.delta + vrow, kT * 4, BAR_QF(s));
+      const Item it = decode_item(idx);
+      if (it.n > 0) {
+        // K and V are free once the previous key tile's last S^T and dP^T completed
+        if (qi > 0 && !(ok = mbar_wait(BAR_KVE, static_cast<uint32_t>(qi - 1) & 1u, a.status, abort_flag))) break;
+        const int zk = it.b * a.Hkv + it.hkv;
+        mbar_arrive_expect_tx(BAR_KV, 2 * T::kTileBytes);
+        for (int c = 0; c < T::kChunks; ++c) {
+          tma_load_3d(sK + c * T::kChunkBytes, &tmK, BAR_KV, c * 64, it.kt * kT, zk);
+          tma_load_3d(sV + c * T::kChunkBytes, &tmV, BAR_KV, c * 64, it.kt * kT, zk);
+        }
+        ++qi;
+        for (int j = 0; j < it.n; ++j) {
+          const int s = static_cast<int>(u & 1u);
+          if (!(ok = mbar_wait(BAR_QE(s), ((u >> 1) & 1u) ^ 1u, a.status, abort_flag))) break;
+          const int hq = it.hkv * G + j / it.per_head, qt = it.i0 + j % it.per_head;
+          const int zq = it.b * a.Hq + hq;
+          mbar_arrive_expect_tx(BAR_QF(s), 2 * T::kTileBytes + 2 * kT * 4);
+          for (int c = 0; c < T::kChunks; ++c) {
+            tma_load_3d(sQ + s * T::kTileBytes + c * T::kChunkBytes, &tmQ, BAR_QF(s), c * 64, qt * kT, zq);
+            tma_load_3d(sDO + s * T::kTileBytes + c * T::kChunkBytes, &tmDO, BAR_QF(s), c * 64, qt * kT, zq);
+          }
+          const size_t vrow = static_cast<size_t>(zq) * (a.n_qt * kT) + qt * kT;
+          bulk_load(sb + L::kVec + (s * 2 + 0) * kT * 4, a.lse2 + vrow, kT * 4, BAR_QF(s));
+          bulk_load(sb + L::kVec + (s * 2 + 1) * kT * 4, a.delta + vrow, kT * 4, BAR_QF(s));
+          ++u;
+        }
+        if (!ok) break;
+      }
+      // the next item (or none)
+      const int kn = k + 1, sl = kn & 1;
+      if (!(ok = mbar_wait(BAR_ITF(sl), resp_parity(kn), a.status, abort_flag))) break;
+      answered = kn;
+      idx = clc_cancelled_ctaid_x(sResp + 16 * sl);
     }
-  } else if (n_items > 0 && warp == 1) {
+    // drain: no copy into this CTA's shared memory may still be in flight at exit
+    if (answered < requested)
+      mbar_wait(BAR_ITF(requested & 1), resp_parity(requested), nullptr, nullptr, kWaitLimitNs);
+    if (qi > 0) mbar_wait(BAR_KV, static_cast<uint32_t>(qi - 1) & 1u, nullptr, nullptr, kWaitLimitNs);
+    for (uint32_t g = (u > 2u ? u - 2u : 0u); g < u; ++g)
+      mbar_wait(BAR_QF(static_cast<int>(g & 1u)), (g >> 1) & 1u, nullptr, nullptr, kWaitLimitNs);
+  } else if (warp == 1) {
     // ======================= MMA issuer =======================
     // The whole warp runs the issue loop (warp-uniform descriptors and
     // waits); the elected lane issues the MMAs and their commits.
@@ -333,41 +399,69 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t dQk = smem_desc_sw128(sQ, 16, 1024), dDOk = smem_desc_sw128(sDO, 16, 1024);
     const uint64_t dQm = smem_desc_sw128(sQ, T::kChunkBytes, 1024), dDOm = smem_desc_sw128(sDO, T::kChunkBytes, 1024);
     constexpr uint64_t kStep = T::kTileBytes >> 4;
-    bool ok = mbar_wait_warp(BAR_KV, 0, a.status, abort_flag);
-    ok = ok && mbar_wait_warp(BAR_QF(0), 0, a.status, abort_flag);
-    if (ok) {
-      tc_fence_after();
-      // S^T = K Q^T and dP^T = V dO^T for the first item
-      mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dK, dQk, idesc_s);
-      commit(BAR_SF);
-      mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dV, dDOk, idesc_s);
-      commit(BAR_DPF);
-    }
-    for (int it = 0; it < n_items && ok; ++it) {
-      const int s = it & 1, s1 = s ^ 1;
-      const uint32_t ph = it & 1u;
-      // dV += P^T dO once P^T is in TMEM
-      if (!(ok = mbar_wait_warp(BAR_PF, ph, a.status, abort_flag))) break;
-      tc_fence_after();
-      mma_tmem_a(leader, tmem + L::kTmDV, tmem + L::kTmS, tmem + L::kTmS + 64, dDOm + s * kStep, idesc_acc, it > 0);
-      // next item's S^T: the S buffer is free once the dV product above has read P^T
-      if (it + 1 < n_items) {
-        if (!(ok = mbar_wait_warp(BAR_QF(s1), ((it + 1) >> 1) & 1u, a.status, abort_flag))) break;
+    bool ok = true;
+    uint32_t u = 0;   // (query head, query tile) pairs so far: ring stage and hand-off phases
+    int qi = 0;       // key tiles with work so far
+    int idx = static_cast<int>(blockIdx.x);
+    for (int k = 0; idx >= 0 && ok; ++k) {
+      const Item it = decode_item(idx);
+      if (it.n > 0) {
+        // the first pair's S^T = K Q^T and dP^T = V dO^T: this key tile's K and V
+        // and the pair's Q stage have landed; the previous tile's last dV and dK
+        // were issued before these, so they read P^T and dS^T first
+        if (!(ok = mbar_wait_warp(BAR_KV, static_cast<uint32_t>(qi) & 1u, a.status, abort_flag))) break;
+        if (!(ok = mbar_wait_warp(BAR_QF(static_cast<int>(u & 1u)), (u >> 1) & 1u, a.status, abort_flag))) break;
         tc_fence_after();
-        mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dK, dQk + s1 * kStep, idesc_s);
+        mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dK, dQk + (u & 1u) * kStep, idesc_s);
         commit(BAR_SF);
-      }
-      // dK += dS^T Q once dS^T is in TMEM
-      if (!(ok = mbar_wait_warp(BAR_DSF, ph, a.status, abort_flag))) break;
-      tc_fence_after();
-      mma_tmem_a(leader, tmem + L::kTmDK, tmem + L::kTmDP, tmem + L::kTmDP + 64, dQm + s * kStep, idesc_acc, it > 0);
-      commit(BAR_QE(s));   // this stage's Q, dO, lse and delta are read once these land
-      if (it + 1 < n_items) {
-        mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dV, dDOk + s1 * kStep, idesc_s);
+        mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dV, dDOk + (u & 1u) * kStep, idesc_s);
         commit(BAR_DPF);
+        if (it.n == 1) commit(BAR_KVE);
+        for (int j = 0; j < it.n; ++j) {
+          const uint32_t uj = u + static_cast<uint32_t>(j);
+          const int s = static_cast<int>(uj & 1u), s1 = s ^ 1;
+          const uint32_t ph = uj & 1u;
+          // dV += P^T dO once P^T is in TMEM; a key tile's first product
+          // overwrites the accumulators, which the previous epilogue must have read
+          if (!(ok = mbar_wait_warp(BAR_PF, ph, a.status, abort_flag))) break;
+          if (j == 0 && qi > 0 &&
+              !(ok = mbar_wait_warp(BAR_ACCE, static_cast<uint32_t>(qi - 1) & 1u, a.status, abort_flag)))
+            break;
+          tc_fence_after();
+          mma_tmem_a(leader, tmem + L::kTmDV, tmem + L::kTmS, tmem + L::kTmS + 64, dDOm + s * kStep, idesc_acc, j > 0);
+          // next pair's S^T: the S buffer is free once the dV product above has read P^T
+          if (j + 1 < it.n) {
+            if (!(ok = mbar_wait_warp(BAR_QF(s1), ((uj + 1) >> 1) & 1u, a.status, abort_flag))) break;
+            tc_fence_after();
+            mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmS, dK, dQk + s1 * kStep, idesc_s);
+            commit(BAR_SF);
+          }
+          // dK += dS^T Q once dS^T is in TMEM
+          if (!(ok = mbar_wait_warp(BAR_DSF, ph, a.status, abort_flag))) break;
+          tc_fence_after();
+          mma_tmem_a(leader, tmem + L::kTmDK, tmem + L::kTmDP, tmem + L::kTmDP + 64, dQm + s * kStep, idesc_acc, j > 0);
+          commit(BAR_QE(s));   // this stage's Q, dO, lse and delta are read once these land
+          if (j + 1 < it.n) {
+            mma_kmajor_tile<T::kChunks>(leader, tmem + L::kTmDP, dV, dDOk + s1 * kStep, idesc_s);
+            commit(BAR_DPF);
+            if (j + 2 == it.n) commit(BAR_KVE);   // the key tile's last S^T and dP^T: K and V are free
+          }
+        }
+        if (!ok) break;
+        commit(BAR_ACC);
+        u += static_cast<uint32_t>(it.n);
+        ++qi;
       }
+      // the next item (or none)
+      const int kn = k + 1, sl = kn & 1;
+      if (!(ok = mbar_wait_warp(BAR_ITF(sl), resp_parity(kn), a.status, abort_flag))) break;
+      idx = clc_cancelled_ctaid_x(sResp + 16 * sl);
+      __syncwarp();
+      if (leader) mbar_arrive(BAR_ITE(sl));
     }
-    if (ok) commit(BAR_ACC);
+    // no commit may still be pending when the CTA exits
+    commit(BAR_FIN);
+    mbar_wait_warp(BAR_FIN, 0, nullptr, nullptr);
   }
   } else {
     setmaxnreg_inc<kBwdRegsWork>();
@@ -375,107 +469,128 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int h = (warp - kWorkWarp0) / 4;         // query columns [64h, 64h + 64) of each tile
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;             // key row within the tile
-    const int key = kt * kT + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float c2 = a.scale_log2;
     const int off = a.Nkv - a.Nq;
     bool ok = true;
-    for (int it = 0; it < n_items; ++it) {
-      const int s = it & 1;
-      const uint32_t ph = it & 1u;
-      const int qt = i0 + it % per_head;
-      const int q0 = qt * kT;
-      // query columns c with key > q0 + c + off are masked: c < lim
-      const int lim = (a.causal ? key - off - q0 : 0) - h * 64;
-      const bool row_ok = key < a.Nkv;
-      const bool need_mask = !row_ok || lim > 0;
-      ok = mbar_wait(BAR_QF(s), (it >> 1) & 1u, a.status, abort_flag);
-      ok = ok && mbar_wait(BAR_SF, ph, a.status, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const float* l2v = vec + (s * 2 + 0) * kT + h * 64;
-      const float* dlv = vec + (s * 2 + 1) * kT + h * 64;
-      // P^T = exp2(S^T c2 - lse2[query]) over this half's 64 query columns,
-      // written as bf16 over the first 32 of the columns it was read from
-      uint32_t pk[32];
-      {
-        uint32_t sr[2][32];
-        tmem_ld32(tmem + L::kTmS + lane_off + h * 64, sr[0]);
-        tmem_ld32(tmem + L::kTmS + lane_off + h * 64 + 32, sr[1]);
-        tmem_wait_ld();
-        const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
-        // lanes that need no mask have lim <= 0 and keep every column
-        if (__any_sync(0xffffffffu, need_mask))
-          p_row_half<true>(sv, l2v, c2, row_ok ? lim : 64, pk);
-        else
-          p_row_half<false>(sv, l2v, c2, 0, pk);
-        tmem_st32(tmem + L::kTmS + lane_off + h * 64, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(BAR_PF);
-      // dS^T = P^T o (dP^T - delta[query]) over this half, written over dP^T
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_DPF, ph, a.status, abort_flag)))) break;
-      tc_fence_after();
-      {
-        uint32_t dr[2][32];
-        tmem_ld32(tmem + L::kTmDP + lane_off + h * 64, dr[0]);
-        tmem_ld32(tmem + L::kTmDP + lane_off + h * 64 + 32, dr[1]);
-        tmem_wait_ld();
-        const float* dpv = reinterpret_cast<const float*>(&dr[0][0]);
-        uint32_t dk[32];
-#pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          const float4 d4 = *reinterpret_cast<const float4*>(dlv + 4 * e2);
-          const uint32_t w0 = pk[2 * e2], w1 = pk[2 * e2 + 1];
-          dk[2 * e2] = pack_bf16x2(bf16lo(w0) * (dpv[4 * e2 + 0] - d4.x), bf16hi(w0) * (dpv[4 * e2 + 1] - d4.y));
-          dk[2 * e2 + 1] = pack_bf16x2(bf16lo(w1) * (dpv[4 * e2 + 2] - d4.z), bf16hi(w1) * (dpv[4 * e2 + 3] - d4.w));
-        }
-        tmem_st32(tmem + L::kTmDP + lane_off + h * 64, dk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(BAR_DSF);
-    }
-    // ---- epilogue: dK (times scale) and dV rows of this key tile
-    const bool have = ok && n_items > 0;
-    if (have) {
-      ok = __all_sync(0xffffffffu, mbar_wait(BAR_ACC, 0, a.status, abort_flag));
-      tc_fence_after();
-    }
-    // TMEM loads are warp-collective: every lane loads, only rows < Nkv store
-    const bool store = key < a.Nkv;
-    const size_t orow = (static_cast<size_t>(b) * a.Hkv + hkv) * a.Nkv + (store ? key : 0);
-#pragma unroll 1
-    for (int which = 0; which < 2; ++which) {
-      // this warpgroup's half of the row: columns [h D/2, (h+1) D/2)
-      __nv_bfloat16* dst_row = (which ? a.dv : a.dk) + orow * D + h * (D / 2);
-      const float mul = which ? 1.f : a.scale;
-      const uint32_t src = tmem + (which ? L::kTmDV : L::kTmDK) + lane_off + h * (D / 2);
-#pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t v[32];
-        if (have && ok) {
-          tmem_ld32(src + c * 32, v);
+    uint32_t u = 0;   // (query head, query tile) pairs so far
+    int qi = 0;       // key tiles with work so far
+    int idx = static_cast<int>(blockIdx.x);
+    for (int k = 0; idx >= 0; ++k) {
+      const Item it = decode_item(idx);
+      const int key = it.kt * kT + r;
+      for (int j = 0; j < it.n && ok; ++j) {
+        const uint32_t uj = u + static_cast<uint32_t>(j);
+        const int s = static_cast<int>(uj & 1u);
+        const uint32_t ph = uj & 1u;
+        const int qt = it.i0 + j % it.per_head;
+        const int q0 = qt * kT;
+        // query columns c with key > q0 + c + off are masked: c < lim
+        const int lim = (a.causal ? key - off - q0 : 0) - h * 64;
+        const bool row_ok = key < a.Nkv;
+        const bool need_mask = !row_ok || lim > 0;
+        ok = mbar_wait(BAR_QF(s), (uj >> 1) & 1u, a.status, abort_flag);
+        ok = ok && mbar_wait(BAR_SF, ph, a.status, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float* l2v = vec + (s * 2 + 0) * kT + h * 64;
+        const float* dlv = vec + (s * 2 + 1) * kT + h * 64;
+        // P^T = exp2(S^T c2 - lse2[query]) over this half's 64 query columns,
+        // written as bf16 over the first 32 of the columns it was read from
+        uint32_t pk[32];
+        {
+          uint32_t sr[2][32];
+          tmem_ld32(tmem + L::kTmS + lane_off + h * 64, sr[0]);
+          tmem_ld32(tmem + L::kTmS + lane_off + h * 64 + 32, sr[1]);
           tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0u;
+          const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+          // lanes that need no mask have lim <= 0 and keep every column
+          if (__any_sync(0xffffffffu, need_mask))
+            p_row_half<true>(sv, l2v, c2, row_ok ? lim : 64, pk);
+          else
+            p_row_half<false>(sv, l2v, c2, 0, pk);
+          tmem_st32(tmem + L::kTmS + lane_off + h * 64, pk);
         }
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR_PF);
+        // dS^T = P^T o (dP^T - delta[query]) over this half, written over dP^T
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_DPF, ph, a.status, abort_flag)))) break;
+        tc_fence_after();
+        {
+          uint32_t dr[2][32];
+          tmem_ld32(tmem + L::kTmDP + lane_off + h * 64, dr[0]);
+          tmem_ld32(tmem + L::kTmDP + lane_off + h * 64 + 32, dr[1]);
+          tmem_wait_ld();
+          const float* dpv = reinterpret_cast<const float*>(&dr[0][0]);
+          uint32_t dk[32];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * mul, __uint_as_float(v[8 * e + 1]) * mul);
-            w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * mul, __uint_as_float(v[8 * e + 3]) * mul);
-            w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * mul, __uint_as_float(v[8 * e + 5]) * mul);
-            w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * mul, __uint_as_float(v[8 * e + 7]) * mul);
-            dst[e] = w;
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const float4 d4 = *reinterpret_cast<const float4*>(dlv + 4 * e2);
+            const uint32_t w0 = pk[2 * e2], w1 = pk[2 * e2 + 1];
+            dk[2 * e2] = pack_bf16x2(bf16lo(w0) * (dpv[4 * e2 + 0] - d4.x), bf16hi(w0) * (dpv[4 * e2 + 1] - d4.y));
+            dk[2 * e2 + 1] = pack_bf16x2(bf16lo(w1) * (dpv[4 * e2 + 2] - d4.z), bf16hi(w1) * (dpv[4 * e2 + 3] - d4.w));
+          }
+          tmem_st32(tmem + L::kTmDP + lane_off + h * 64, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR_DSF);
+      }
+      u += static_cast<uint32_t>(it.n);
+      // ---- epilogue: dK (times scale) and dV rows of this key tile; a key
+      // tile that no query sees gets zeros
+      const bool have = ok && it.n > 0;
+      if (have) {
+        ok = __all_sync(0xffffffffu, mbar_wait(BAR_ACC, static_cast<uint32_t>(qi) & 1u, a.status, abort_flag));
+        tc_fence_after();
+      }
+      // TMEM loads are warp-collective: every lane loads, only rows < Nkv store
+      const bool store = key < a.Nkv;
+      const size_t orow = (static_cast<size_t>(it.b) * a.Hkv + it.hkv) * a.Nkv + (store ? key : 0);
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        // this warpgroup's half of the row: columns [h D/2, (h+1) D/2)
+        __nv_bfloat16* dst_row = (which ? a.dv : a.dk) + orow * D + h * (D / 2);
+        const float mul = which ? 1.f : a.scale;
+        const uint32_t src = tmem + (which ? L::kTmDV : L::kTmDK) + lane_off + h * (D / 2);
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t v[32];
+          if (have && ok) {
+            tmem_ld32(src + c * 32, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * mul, __uint_as_float(v[8 * e + 1]) * mul);
+              w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * mul, __uint_as_float(v[8 * e + 3]) * mul);
+              w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * mul, __uint_as_float(v[8 * e + 5]) * mul);
+              w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * mul, __uint_as_float(v[8 * e + 7]) * mul);
+              dst[e] = w;
+            }
           }
         }
       }
+      if (it.n > 0) {
+        // dV and dK have been read: the next key tile's first products may overwrite them
+        tc_fence_before();
+        mbar_arrive(BAR_ACCE);
+        ++qi;
+      }
+      if (!ok) break;
+      // the next item (or none)
+      const int kn = k + 1, sl = kn & 1;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_ITF(sl), resp_parity(kn), a.status, abort_flag)))) break;
+      idx = clc_cancelled_ctaid_x(sResp + 16 * sl);
+      mbar_arrive(BAR_ITE(sl));
     }
   }
 
