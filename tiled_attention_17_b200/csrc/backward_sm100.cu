@@ -117,15 +117,18 @@ __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w <
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // P^T over 64 query columns of one key row: p_c = exp2(s_c c2 - lse2_c) as
-// bf16 pairs.  kMask zeroes the columns c < lo (causally hidden, or every
+// bf16 pairs.  The caller loads the columns' lse2 into registers (lv) before
+// it waits for S^T, so those shared-memory loads, which queue behind the
+// tensor pipe's operand reads, overlap the wait instead of the
+// exponentials.  kMask zeroes the columns c < lo (causally hidden, or every
 // column of a key row past the keys).  The two forms are separate code
 // paths behind a warp-uniform branch: a compare-and-select per element on
 // every tile would cost more issue slots than the exponentials themselves.
 template <bool kMask>
-__device__ __forceinline__ void p_row_half(const float* sv, const float* l2v, float c2, int lo, uint32_t* pk) {
+__device__ __forceinline__ void p_row_half(const float* sv, const float4* lv, float c2, int lo, uint32_t* pk) {
 #pragma unroll
   for (int e4 = 0; e4 < 16; ++e4) {
-    const float4 l4 = *reinterpret_cast<const float4*>(l2v + 4 * e4);
+    const float4 l4 = lv[e4];
     const int c = 4 * e4;
     float p0 = ex2(fmaf(sv[c + 0], c2, -l4.x)), p1 = ex2(fmaf(sv[c + 1], c2, -l4.y));
     float p2 = ex2(fmaf(sv[c + 2], c2, -l4.z)), p3 = ex2(fmaf(sv[c + 3], c2, -l4.w));
@@ -490,12 +493,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool row_ok = key < a.Nkv;
         const bool need_mask = !row_ok || lim > 0;
         ok = mbar_wait(BAR_QF(s), (uj >> 1) & 1u, a.status, abort_flag);
+        const float* l2v = vec + (s * 2 + 0) * kT + h * 64;
+        const float* dlv = vec + (s * 2 + 1) * kT + h * 64;
+        // this half's 64 lse2 values into registers while S^T is computed
+        float4 lv[16];
+#pragma unroll
+        for (int e4 = 0; e4 < 16; ++e4) lv[e4] = reinterpret_cast<const float4*>(l2v)[e4];
         ok = ok && mbar_wait(BAR_SF, ph, a.status, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const float* l2v = vec + (s * 2 + 0) * kT + h * 64;
-        const float* dlv = vec + (s * 2 + 1) * kT + h * 64;
         // P^T = exp2(S^T c2 - lse2[query]) over this half's 64 query columns,
         // written as bf16 over the first 32 of the columns it was read from
         uint32_t pk[32];
@@ -507,15 +514,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
           // lanes that need no mask have lim <= 0 and keep every column
           if (__any_sync(0xffffffffu, need_mask))
-            p_row_half<true>(sv, l2v, c2, row_ok ? lim : 64, pk);
+            p_row_half<true>(sv, lv, c2, row_ok ? lim : 64, pk);
           else
-            p_row_half<false>(sv, l2v, c2, 0, pk);
+            p_row_half<false>(sv, lv, c2, 0, pk);
           tmem_st32(tmem + L::kTmS + lane_off + h * 64, pk);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(BAR_PF);
-        // dS^T = P^T o (dP^T - delta[query]) over this half, written over dP^T
+        // dS^T = P^T o (dP^T - delta[query]) over this half, written over dP^T; delta
+        // into registers while dP^T is computed
+        float4 dv4[16];
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) dv4[e2] = reinterpret_cast<const float4*>(dlv)[e2];
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(BAR_DPF, ph, a.status, abort_flag)))) break;
         tc_fence_after();
         {
@@ -527,7 +538,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t dk[32];
 #pragma unroll
           for (int e2 = 0; e2 < 16; ++e2) {
-            const float4 d4 = *reinterpret_cast<const float4*>(dlv + 4 * e2);
+            const float4 d4 = dv4[e2];
             const uint32_t w0 = pk[2 * e2], w1 = pk[2 * e2 + 1];
             dk[2 * e2] = pack_bf16x2(bf16lo(w0) * (dpv[4 * e2 + 0] - d4.x), bf16hi(w0) * (dpv[4 * e2 + 1] - d4.y));
             dk[2 * e2 + 1] = pack_bf16x2(bf16lo(w1) * (dpv[4 * e2 + 2] - d4.z), bf16hi(w1) * (dpv[4 * e2 + 3] - d4.w));
