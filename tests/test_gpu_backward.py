@@ -79,6 +79,10 @@ CASES = [
     (1, 1, 1, 1, 700, 128, False),        # one query row
     (1, 2, 1, 300, 100, 128, True),       # rows with no visible key
     (2, 40, 8, 512, 512, 128, True),      # more CTAs than SMs
+    # Persistent CTAs (more items than SMs): a CTA takes over further items.
+    (1, 32, 8, 1024, 256, 128, True),     # 256 dQ items, 6 of each head's 8 see no key
+    (2, 16, 8, 256, 2048, 128, True),     # 256 dK/dV key-tile items, Nq < Nkv
+    (1, 8, 8, 130, 2500, 64, False),      # 160 dK/dV items at d = 64, ragged last key tile
 ]
 
 
