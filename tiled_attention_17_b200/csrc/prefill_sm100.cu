@@ -64,11 +64,11 @@ constexpr float kRescaleLog2 = 8.0f;   // skip O rescale while max grew by <= 2^
 // Column pairs whose index i has bit (i % 8) set in the mask compute 2^x on
 // the FMA pipe (exp2_poly2) instead of the MUFU unit.  bf16: moving 1/8 to 4/8
 // of them there was measured, none was faster on B200, so all stay on MUFU.
-// fp8: the products take half the tensor cycles and MUFU limits more; 3/8
-// (pairs 0, 2, 5 of every 8) measured fastest, +6.5% and +6.7% on two boxes
-// (1/8: +4%, 2/8: +5%, 4/8: +2%).
+// fp8: the products take half the tensor cycles and MUFU limits more.  With
+// the current issue loop and persistent CTAs, 1/8 (pair 0 of every 8) is
+// fastest: +3% over none and over 3/8 (2/8: +1.5%, 4/8: -4%, 6/8: -13%).
 constexpr unsigned kPolyMask = 0x00u;
-constexpr unsigned kPolyMaskFp8 = 0x25u;
+constexpr unsigned kPolyMaskFp8 = 0x01u;
 
 template <int D, bool kFp8 = false>
 struct PrefillLayout {
