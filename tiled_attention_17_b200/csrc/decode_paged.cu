@@ -409,7 +409,7 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel_shared(uint32_t addr, uint3
 
 __global__ void __launch_bounds__(kG4Threads, 2) decode_split_g4_kernel(const DecodeArgs a) {
   using L = G4Layout;
-  constexpr int D = 128, LPR = 16;
+  constexpr int D = 128;
   extern __shared__ __align__(1024) uint8_t smem[];
 
   const int split = blockIdx.x, hkv = blockIdx.y, seq = blockIdx.z;
