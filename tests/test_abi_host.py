@@ -140,9 +140,9 @@ def test_decode_validation(lib):
 
 
 def test_workspace_plan(lib):
-    # 64 sequences x 8 KV heads x 2048 pages of 16: 1024-token splits -> 32 splits
+    # 64 sequences x 8 KV heads x 2048 pages of 16: 2048-token splits -> 16 splits
     ws = lib.attn_paged_decode_workspace_size(64, 32, 8, 128, 2048, 16)
-    rows = 64 * 32 * 32
+    rows = 64 * 32 * 16
     assert ws >= rows * 128 * 4 + rows * 4 + 256
     assert ws % 256 == 0
     assert lib.attn_paged_decode_workspace_size(64, 32, 8, 128, 2048, 12) == 0

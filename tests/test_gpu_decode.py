@@ -79,18 +79,19 @@ def test_decode_zero_length(torch_cuda):
 
 
 def test_decode_long_split_merge(torch_cuda):
-    # lengths spanning many splits, including split-boundary and chunk-boundary lengths
-    lens = [1024, 1025, 4095, 8193]
+    # lengths spanning many splits, including split-boundary (2048-token splits)
+    # and chunk-boundary lengths
+    lens = [1024, 2048, 2049, 4095, 8193]
     inp = small_paged(4, 8, 2, 128, 16, lens, seed=2)
     check_decode(torch_cuda, inp, "long split merge")
 
 
 GATHER_CASES = [
     # page_size, d, lens: partial last pages, lengths that span several splits
-    # (a split is 1024 tokens, 64 pages at page 8) and the split boundaries
-    (8, 128, [1, 37, 513, 1030]),
-    (16, 128, [1, 37, 1024, 1025, 3000]),
-    (32, 128, [31, 33, 2100]),
+    # (a split is 2048 tokens, 256 pages at page 8) and the split boundaries
+    (8, 128, [1, 37, 513, 2050]),
+    (16, 128, [1, 37, 2048, 2049, 5000]),
+    (32, 128, [31, 33, 4200]),
     (64, 128, [70, 1, 4097]),
     (8, 64, [5, 200, 600]),
     (64, 64, [130]),
