@@ -82,7 +82,7 @@ def test_decode_long_split_merge(torch_cuda):
     # lengths spanning many splits, including split-boundary (2048-token splits)
     # and chunk-boundary lengths
     lens = [1024, 2048, 2049, 4095, 8193]
-    inp = small_paged(4, 8, 2, 128, 16, lens, seed=2)
+    inp = small_paged(len(lens), 8, 2, 128, 16, lens, seed=2)
     check_decode(torch_cuda, inp, "long split merge")
 
 
