@@ -79,8 +79,9 @@ struct BwdArgs {
   // Items are launched in groups of heads (dK/dV: KV heads, dQ: query heads),
   // all of a group's tiles before the next group's, heaviest tile first
   // within the group.  The CTAs running at once then stream one or two
-  // groups' operands (sized on the host to ~24 MB, inside L2) instead of
-  // every head's, so each streamed tile is read from DRAM about once.
+  // groups' operands instead of every head's, so each streamed tile is read
+  // from DRAM about once.  The host sizes the groups (L2 and load-balance
+  // bounds, launch_bwd_d); one group is the tile-major order across all heads.
   int kv_group, q_group;
 };
 
