@@ -50,6 +50,7 @@ CASES = [
     ([64, 512], [64, 700], 2, 1, 64, 64),                              # d = 64, 64-token pages
     ([300], [200], 2, 2, 128, 16),                                     # more queries than keys: masked rows
     ([300, 5, 700], [300, 900, 1200], 6, 2, 128, 16),                  # GQA group 3: consecutive-tile pairs
+    ([150, 400], [500, 900], 4, 1, 128, 64),                           # d = 128, 64-token pages
 ]
 
 

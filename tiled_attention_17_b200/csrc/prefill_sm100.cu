@@ -293,16 +293,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       // K or V tile j into ring slot `dst`: one tile box (dense), or one box per
-      // page (paged, pages from lookup_pages)
-      auto load_kv = [&](const Item& it, const CUtensorMap* tm, uint32_t dst, uint32_t bar, int j) {
+      // page (paged, pages from lookup_pages).  Paged K keeps the dense layout
+      // (each 64-column chunk holds all 128 keys: the scores MMA needs a uniform
+      // key stride), one copy per page and chunk.  Paged V is stored page-major
+      // ([page][chunk][page rows][128 B]) and a page's chunks arrive in one
+      // copy: each 16-key step of P V addresses its own page block, and a
+      // copy's fixed cost, not its bytes, is what a small page pays for.
+      auto load_kv = [&](const Item& it, const CUtensorMap* tm, uint32_t dst, uint32_t bar, int j, bool is_v) {
         if constexpr (kPaged) {
           const int per_tile = kBN / a.page_size;
 #pragma unroll
           for (int p = 0; p < kMaxPagesPerTile; ++p) {
             if (p >= per_tile) break;
-            for (int c = 0; c < L::kChunks; ++c)
-              tma_load_4d(dst + c * L::kChunkBytes + p * a.page_size * 128, tm, bar, c * L::kChunkElems, 0, it.hkv,
-                          phys[p]);
+            if (L::kChunks == 2 && is_v) {
+              tma_load_5d(dst + p * a.page_size * 256, tm, bar, 0, 0, 0, it.hkv, phys[p]);
+            } else {
+              for (int c = 0; c < L::kChunks; ++c)
+                tma_load_4d(dst + c * L::kChunkBytes + p * a.page_size * 128, tm, bar, c * L::kChunkElems, 0,
+                            it.hkv, phys[p]);
+            }
           }
         } else {
           for (int c = 0; c < L::kChunks; ++c)
@@ -353,11 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             lookup_pages(it, j);   // before the wait, so the table reads overlap it
             if (!(ok = mbar_wait(BAR_KE(s), ph ^ 1u, a.status, abort_flag))) break;
             mbar_arrive_expect_tx(BAR_KF(s), L::kTileBytes);
-            load_kv(it, &tmK, sK + s * L::kTileBytes, BAR_KF(s), j);
+            load_kv(it, &tmK, sK + s * L::kTileBytes, BAR_KF(s), j, false);
             ++gk;
             if (!(ok = mbar_wait(BAR_VE(s), ph ^ 1u, a.status, abort_flag))) break;
             mbar_arrive_expect_tx(BAR_VF(s), L::kTileBytes);
-            load_kv(it, &tmV, sV + s * L::kTileBytes, BAR_VF(s), j);
+            load_kv(it, &tmV, sV + s * L::kTileBytes, BAR_VF(s), j, true);
             ++gv;
           }
           if (!ok) break;
@@ -407,8 +416,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // adds compile-time offsets instead of rebuilding descriptors.
       const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t dK = smem_desc_sw128(sK, 16, 1024);
-      const uint64_t dV = smem_desc_sw128(sV, L::kChunkBytes, 1024);
+      // Paged V with two chunks is page-major: the chunk stride is one page of
+      // 128-byte rows; 8-key groups are 1024 bytes apart inside a page, one
+      // page block (2 KB) apart when a page holds 8 keys.
+      constexpr bool kPagedV = kPaged && L::kChunks == 2;
+      const int ps = kPaged ? a.page_size : 128;
+      const uint64_t dV = kPagedV ? smem_desc_sw128(sV, static_cast<uint32_t>(ps) * 128u, ps >= 16 ? 1024u : 2048u)
+                                  : smem_desc_sw128(sV, L::kChunkBytes, 1024);
       constexpr uint64_t kTileStep = L::kTileBytes >> 4;
+      // 16-key step kk starts at byte 2048 (kk + (kk & vmask)): m = max(page / 16, 1) steps per
+      // page (a power of two), page blocks of m * 4096 bytes, 2048 bytes per step inside one
+      const int vmask = ~(max(ps / 16, 1) - 1);
 
       // S_t = Q_t K^T over d in 32-byte steps (K-major operands, 128B swizzle)
       auto issue_qk = [&](int t, int s) {
@@ -440,8 +458,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k4 = 0; k4 < kPerHalf; ++k4) {
             const int kk = half * kPerHalf + k4;
-            mma_t(d, a + kk * 8, b0 + static_cast<uint64_t>((kk * L::kKeysPerMma * 128) >> 4), idesc_pv,
-                  (acc || kk > 0) ? 1u : 0u);
+            uint32_t off = kk * L::kKeysPerMma * 128;   // dense: 16 keys of 128-byte rows per step
+            if constexpr (kPagedV) {
+              off = static_cast<uint32_t>((kk + (kk & vmask)) << 11);
+            }
+            mma_t(d, a + kk * 8, b0 + static_cast<uint64_t>(off >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
           }
         }
         __syncwarp();
@@ -813,7 +834,18 @@ static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, cons
                                  static_cast<uint64_t>(Hkv) * page_size * D * 2};
     const uint32_t box[4] = {64, static_cast<uint32_t>(page_size), 1, 1};
     if ((st = encode_bf16_tiled(&tk, k_cache, 4, dims, strides, box)) != TA_OK) return st;
-    if ((st = encode_bf16_tiled(&tv, v_cache, 4, dims, strides, box)) != TA_OK) return st;
+    if (L::kChunks == 1) {
+      if ((st = encode_bf16_tiled(&tv, v_cache, 4, dims, strides, box)) != TA_OK) return st;
+    } else {
+      // V: [P, Hkv, page, (2 chunks of 64)] seen as 5-D {64, page, chunk, Hkv, P}, so that one box
+      // {64, page, 2, 1, 1} lands a page as [chunk][page rows][128 B]
+      const uint64_t dv[5] = {64, static_cast<uint64_t>(page_size), 2, static_cast<uint64_t>(Hkv),
+                              static_cast<uint64_t>(num_pages_total)};
+      const uint64_t sv[4] = {static_cast<uint64_t>(D) * 2, 128, static_cast<uint64_t>(page_size) * D * 2,
+                              static_cast<uint64_t>(Hkv) * page_size * D * 2};
+      const uint32_t bv[5] = {64, static_cast<uint32_t>(page_size), 2, 1, 1};
+      if ((st = encode_bf16_tiled(&tv, v_cache, 5, dv, sv, bv)) != TA_OK) return st;
+    }
   }
   static int attr_done[64] = {0};
   cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, true, false>, L::kAlloc, attr_done);
