@@ -89,7 +89,8 @@ PFN_encodeTiled get_encode_tiled() {
 }
 
 static ta_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int rank,
-                              const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+                              const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   PFN_encodeTiled enc = get_encode_tiled();
   if (!enc) return fail(TA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t d[5], st[4];
@@ -101,7 +102,7 @@ static ta_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, const
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
   CUresult r = enc(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d,
-                   st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? TA_OK : fail_cu(TA_ERR_CUDA, "cuTensorMapEncodeTiled", static_cast<int>(r));
 }
@@ -109,6 +110,12 @@ static ta_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, const
 ta_status encode_bf16_tiled(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                             const uint64_t* strides_bytes, const uint32_t* box) {
   return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box);
+}
+
+ta_status encode_bf16_tiled_sw32(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                                 const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box,
+                      CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
 ta_status encode_u8_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {

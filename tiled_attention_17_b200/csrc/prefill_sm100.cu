@@ -293,12 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       // K or V tile j into ring slot `dst`: one tile box (dense), or one box per
-      // page (paged, pages from lookup_pages).  Paged K keeps the dense layout
-      // (each 64-column chunk holds all 128 keys: the scores MMA needs a uniform
-      // key stride), one copy per page and chunk.  Paged V is stored page-major
-      // ([page][chunk][page rows][128 B]) and a page's chunks arrive in one
-      // copy: each 16-key step of P V addresses its own page block, and a
-      // copy's fixed cost, not its bytes, is what a small page pays for.
+      // page (paged, pages from lookup_pages).  With two 64-column chunks a page
+      // arrives in one copy, not one per chunk: a copy's fixed cost, not its
+      // bytes, is what a small page pays for.  Paged V is page-major
+      // ([page][chunk][page rows][128 B]): each 16-key step of P V addresses its
+      // own page block.  Paged K uses the 32-byte swizzle as
+      // [8-row group][16-column K step][8 rows][32 B]: the scores MMA reads each
+      // K step of all 128 keys at one 8-row-group stride (2 KB), whichever page
+      // the group came from.
       auto load_kv = [&](const Item& it, const CUtensorMap* tm, uint32_t dst, uint32_t bar, int j, bool is_v) {
         if constexpr (kPaged) {
           const int per_tile = kBN / a.page_size;
@@ -307,6 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p >= per_tile) break;
             if (L::kChunks == 2 && is_v) {
               tma_load_5d(dst + p * a.page_size * 256, tm, bar, 0, 0, 0, it.hkv, phys[p]);
+            } else if (L::kChunks == 2) {
+              tma_load_5d(dst + p * a.page_size * 256, tm, bar, 0, 0, 0, 0, phys[p] * a.Hkv + it.hkv);
             } else {
               for (int c = 0; c < L::kChunks; ++c)
                 tma_load_4d(dst + c * L::kChunkBytes + p * a.page_size * 128, tm, bar, c * L::kChunkElems, 0,
@@ -415,7 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // only moves the start-address field (address >> 4), so the issue loop
       // adds compile-time offsets instead of rebuilding descriptors.
       const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
-      const uint64_t dK = smem_desc_sw128(sK, 16, 1024);
+      // paged K with two chunks: 32-byte swizzle, K step kk at byte 256 kk
+      constexpr bool kPagedK = kPaged && L::kChunks == 2;
+      const uint64_t dK = kPagedK ? smem_desc_sw32(sK, 2048) : smem_desc_sw128(sK, 16, 1024);
+      constexpr uint64_t kKStep = kPagedK ? 16 : 2;                              // one K step
+      constexpr uint64_t kKChunk = kPagedK ? 4 * kKStep : (L::kChunkBytes >> 4);   // four K steps
       // Paged V with two chunks is page-major: the chunk stride is one page of
       // 128-byte rows; 8-key groups are 1024 bytes apart inside a page, one
       // page block (2 KB) apart when a page holds 8 keys.
@@ -440,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < L::kChunks; ++c) {
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)
-              mma_s(d, a0 + 2 * k4, b0 + 2 * k4, idesc_qk, (c | k4) != 0 ? 1u : 0u);
+              mma_s(d, a0 + 2 * k4, b0 + kKStep * k4, idesc_qk, (c | k4) != 0 ? 1u : 0u);
             a0 += L::kChunkBytes >> 4;
-            b0 += L::kChunkBytes >> 4;
+            b0 += kKChunk;
           }
         }
         __syncwarp();
@@ -833,10 +841,18 @@ static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, cons
     const uint64_t strides[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(page_size) * D * 2,
                                  static_cast<uint64_t>(Hkv) * page_size * D * 2};
     const uint32_t box[4] = {64, static_cast<uint32_t>(page_size), 1, 1};
-    if ((st = encode_bf16_tiled(&tk, k_cache, 4, dims, strides, box)) != TA_OK) return st;
     if (L::kChunks == 1) {
+      if ((st = encode_bf16_tiled(&tk, k_cache, 4, dims, strides, box)) != TA_OK) return st;
       if ((st = encode_bf16_tiled(&tv, v_cache, 4, dims, strides, box)) != TA_OK) return st;
     } else {
+      // K: [P, Hkv, page, 128] seen as 5-D {16 columns, 8 rows, 8 column groups, page / 8 row
+      // groups, P * Hkv (page, head) blocks}, box {16, 8, 8, page / 8, 1}, 32-byte swizzle: one
+      // copy lands a page as [row group][column group][8 rows][32 B]
+      const uint64_t dk[5] = {16, 8, 8, static_cast<uint64_t>(page_size / 8),
+                              static_cast<uint64_t>(num_pages_total) * Hkv};
+      const uint64_t sk[4] = {static_cast<uint64_t>(D) * 2, 32, 8ull * D * 2, static_cast<uint64_t>(page_size) * D * 2};
+      const uint32_t bk[5] = {16, 8, 8, static_cast<uint32_t>(page_size / 8), 1};
+      if ((st = encode_bf16_tiled_sw32(&tk, k_cache, 5, dk, sk, bk)) != TA_OK) return st;
       // V: [P, Hkv, page, (2 chunks of 64)] seen as 5-D {64, page, chunk, Hkv, P}, so that one box
       // {64, page, 2, 1, 1} lands a page as [chunk][page rows][128 B]
       const uint64_t dv[5] = {64, static_cast<uint64_t>(page_size), 2, static_cast<uint64_t>(Hkv),

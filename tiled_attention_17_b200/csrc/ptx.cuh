@@ -307,6 +307,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 //   bits 49-51 base offset (0: tiles are 1024-byte aligned)
 //   bits 61-63 layout: 2 = 128-byte swizzle
 // ----------------------------------------------------------------------------
+// K-major operand in the 32-byte swizzle: one 16-element K step per 32-byte
+// row (the leading offset is unused), 8-row groups `sbo_bytes` apart.
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t addr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(6) << 61;
+  return d;
+}
+
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);

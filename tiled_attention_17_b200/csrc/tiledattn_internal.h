@@ -29,6 +29,9 @@ ta_status encode_u8_rows_3d(CUtensorMap* map, const void* base, int d, int rows,
 // bounds); strides_bytes has rank - 1 entries.
 ta_status encode_bf16_tiled(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                             const uint64_t* strides_bytes, const uint32_t* box);
+// The same with the 32-byte swizzle (box rows of 32 bytes).
+ta_status encode_bf16_tiled_sw32(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                                 const uint64_t* strides_bytes, const uint32_t* box);
 
 // Records a description of the last host-side failure of this thread
 // (returned by ta_last_error) and returns `code`.
