@@ -118,18 +118,27 @@ ta_status encode_bf16_tiled_sw32(CUtensorMap* map, const void* base, int rank, c
                       CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
-ta_status encode_u8_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
-  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows), static_cast<uint64_t>(slices)};
-  const uint64_t strides[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows) * d};
-  const uint32_t box[3] = {128, 128, 1};
-  return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 3, dims, strides, box);
+// Tiles of 128 rows of a [slices, rows, d] tensor, each in ONE copy: the map
+// is 4-D {one 128-byte chunk of columns, rows, d / chunk, slices} with the
+// chunk stride of 128 bytes, so a box {chunk, 128, d / chunk, 1} lands a tile
+// as [chunk][128 rows][128 B], the 128-byte-swizzle layout of every chunk.
+// (A copy has a fixed cost in the SM's copy engine.  For these 16 KB chunks it
+// is small beside the bytes: one copy per tile times the same as one per
+// chunk.  For page-sized copies it is not; see the paged prefill.)
+ta_status encode_u8_rows_chunked(CUtensorMap* map, const void* base, int d, int rows, int slices) {
+  const uint64_t dims[4] = {128, static_cast<uint64_t>(rows), static_cast<uint64_t>(d / 128),
+                            static_cast<uint64_t>(slices)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(d), 128, static_cast<uint64_t>(rows) * d};
+  const uint32_t box[4] = {128, 128, static_cast<uint32_t>(d / 128), 1};
+  return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 4, dims, strides, box);
 }
 
-ta_status encode_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices) {
-  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(rows), static_cast<uint64_t>(slices)};
-  const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(rows) * d * 2};
-  const uint32_t box[3] = {64, 128, 1};
-  return encode_bf16_tiled(map, base, 3, dims, strides, box);
+ta_status encode_rows_chunked(CUtensorMap* map, const void* base, int d, int rows, int slices) {
+  const uint64_t dims[4] = {64, static_cast<uint64_t>(rows), static_cast<uint64_t>(d / 64),
+                            static_cast<uint64_t>(slices)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(d) * 2, 128, static_cast<uint64_t>(rows) * d * 2};
+  const uint32_t box[4] = {64, 128, static_cast<uint32_t>(d / 64), 1};
+  return encode_bf16_tiled(map, base, 4, dims, strides, box);
 }
 
 static thread_local char g_last_error[256] = "";

@@ -366,10 +366,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (qi > 0 && !(ok = mbar_wait(BAR_KVE, static_cast<uint32_t>(qi - 1) & 1u, a.status, abort_flag))) break;
         const int zk = it.b * a.Hkv + it.hkv;
         mbar_arrive_expect_tx(BAR_KV, 2 * T::kTileBytes);
-        for (int c = 0; c < T::kChunks; ++c) {
-          tma_load_3d(sK + c * T::kChunkBytes, &tmK, BAR_KV, c * 64, it.kt * kT, zk);
-          tma_load_3d(sV + c * T::kChunkBytes, &tmV, BAR_KV, c * 64, it.kt * kT, zk);
-        }
+        tma_load_4d(sK, &tmK, BAR_KV, 0, it.kt * kT, 0, zk);
+        tma_load_4d(sV, &tmV, BAR_KV, 0, it.kt * kT, 0, zk);
         ++qi;
         for (int j = 0; j < it.n; ++j) {
           const int s = static_cast<int>(u & 1u);
@@ -377,10 +375,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int hq = it.hkv * G + j / it.per_head, qt = it.i0 + j % it.per_head;
           const int zq = it.b * a.Hq + hq;
           mbar_arrive_expect_tx(BAR_QF(s), 2 * T::kTileBytes + 2 * kT * 4);
-          for (int c = 0; c < T::kChunks; ++c) {
-            tma_load_3d(sQ + s * T::kTileBytes + c * T::kChunkBytes, &tmQ, BAR_QF(s), c * 64, qt * kT, zq);
-            tma_load_3d(sDO + s * T::kTileBytes + c * T::kChunkBytes, &tmDO, BAR_QF(s), c * 64, qt * kT, zq);
-          }
+          tma_load_4d(sQ + s * T::kTileBytes, &tmQ, BAR_QF(s), 0, qt * kT, 0, zq);
+          tma_load_4d(sDO + s * T::kTileBytes, &tmDO, BAR_QF(s), 0, qt * kT, 0, zq);
           const size_t vrow = static_cast<size_t>(zq) * (a.n_qt * kT) + qt * kT;
           bulk_load(sb + L::kVec + (s * 2 + 0) * kT * 4, a.lse2 + vrow, kT * 4, BAR_QF(s));
           bulk_load(sb + L::kVec + (s * 2 + 1) * kT * 4, a.delta + vrow, kT * 4, BAR_QF(s));
@@ -786,22 +782,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (qi > 0 && !(ok = mbar_wait(BAR_QE, static_cast<uint32_t>(qi - 1) & 1u, a.status, abort_flag))) break;
         const int zq = it.b * a.Hq + it.hq, zk = it.b * a.Hkv + it.hkv;
         mbar_arrive_expect_tx(BAR_Q, 2 * T::kTileBytes);
-        for (int c = 0; c < T::kChunks; ++c) {
-          tma_load_3d(sQ + c * T::kChunkBytes, &tmQ, BAR_Q, c * 64, it.q0, zq);
-          tma_load_3d(sDO + c * T::kChunkBytes, &tmDO, BAR_Q, c * 64, it.q0, zq);
-        }
+        tma_load_4d(sQ, &tmQ, BAR_Q, 0, it.q0, 0, zq);
+        tma_load_4d(sDO, &tmDO, BAR_Q, 0, it.q0, 0, zq);
         ++qi;
         for (int j = 0; j < it.n; ++j) {
           const int sk = static_cast<int>(gk % kSK), sv = static_cast<int>(gv % kSV);
           if (!(ok = mbar_wait(BAR_KE(sk), ((gk / kSK) & 1u) ^ 1u, a.status, abort_flag))) break;
           mbar_arrive_expect_tx(BAR_KF(sk), T::kTileBytes);
-          for (int c = 0; c < T::kChunks; ++c)
-            tma_load_3d(sK + sk * T::kTileBytes + c * T::kChunkBytes, &tmK, BAR_KF(sk), c * 64, j * kT, zk);
+          tma_load_4d(sK + sk * T::kTileBytes, &tmK, BAR_KF(sk), 0, j * kT, 0, zk);
           ++gk;
           if (!(ok = mbar_wait(BAR_VE(sv), ((gv / kSV) & 1u) ^ 1u, a.status, abort_flag))) break;
           mbar_arrive_expect_tx(BAR_VF(sv), T::kTileBytes);
-          for (int c = 0; c < T::kChunks; ++c)
-            tma_load_3d(sV + sv * T::kTileBytes + c * T::kChunkBytes, &tmV, BAR_VF(sv), c * 64, j * kT, zk);
+          tma_load_4d(sV + sv * T::kTileBytes, &tmV, BAR_VF(sv), 0, j * kT, 0, zk);
           ++gv;
         }
         if (!ok) break;
@@ -1094,10 +1086,10 @@ ta_status launch_bwd_d(const void* q, const void* k, const void* v, const void* 
   }
   CUtensorMap tq, tk, tv, tdo;
   ta_status st;
-  if ((st = encode_rows_3d(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
-  if ((st = encode_rows_3d(&tdo, dout, D, Nq, B * Hq)) != TA_OK) return st;
-  if ((st = encode_rows_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
-  if ((st = encode_rows_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_rows_chunked(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
+  if ((st = encode_rows_chunked(&tdo, dout, D, Nq, B * Hq)) != TA_OK) return st;
+  if ((st = encode_rows_chunked(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_rows_chunked(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
   static int done_kv[64] = {0}, done_q[64] = {0};
   cudaError_t e = ensure_smem_limit(bwd_dkdv_kernel<D>, DkdvLayout<D>::kAlloc, done_kv);
   if (e != cudaSuccess) return fail(TA_ERR_CUDA, "attn_bwd: shared-memory limit (dK/dV)", e);

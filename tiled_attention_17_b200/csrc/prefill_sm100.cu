@@ -318,8 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_load_3d(dst + c * L::kChunkBytes, tm, bar, c * L::kChunkElems, j * kBN, it.b * a.Hkv + it.hkv);
+          tma_load_4d(dst, tm, bar, 0, j * kBN, 0, it.b * a.Hkv + it.hkv);
         }
       };
       bool ok = true;
@@ -350,14 +349,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int q0 = t ? it.q0_1 : it.q0_0;
             const int hq = t ? it.hq_1 : it.hq_0;
             if (q0 >= it.Nq) continue;
-            for (int c = 0; c < L::kChunks; ++c) {
-              if constexpr (kPaged)   // packed [total_q, Hq, d]: box of 128 rows of one head
-                tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, hq,
-                            it.q_base + q0);
-              else
-                tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tmQ, BAR_Q(), c * L::kChunkElems, q0,
-                            it.b * a.Hq + hq);
-            }
+            if constexpr (kPaged)   // packed [total_q, Hq, d]: box of 128 rows of one head
+              tma_load_4d(sQ + t * L::kTileBytes, &tmQ, BAR_Q(), 0, hq, it.q_base + q0, 0);
+            else
+              tma_load_4d(sQ + t * L::kTileBytes, &tmQ, BAR_Q(), 0, q0, 0, it.b * a.Hq + hq);
           }
           ++qi;
           for (int j = 0; j < it.n_max && ok; ++j, ++g) {
@@ -793,9 +788,9 @@ static ta_status launch_prefill_d(const void* q, const void* k, const void* v, v
   using L = PrefillLayout<D>;
   CUtensorMap tq, tk, tv;
   ta_status st;
-  if ((st = encode_rows_3d(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
-  if ((st = encode_rows_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
-  if ((st = encode_rows_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_rows_chunked(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
+  if ((st = encode_rows_chunked(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_rows_chunked(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
   static int attr_done[64] = {0};
   cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, false, false>, L::kAlloc, attr_done);
   if (e != cudaSuccess) return fail(TA_ERR_CUDA, "prefill: shared-memory limit", e);
@@ -829,11 +824,12 @@ static ta_status launch_paged_prefill_d(const void* q, const void* k_cache, cons
   using L = PrefillLayout<D>;
   CUtensorMap tq, tk, tv;
   ta_status st;
-  {  // packed queries [total_q, Hq, d]: boxes of 128 rows of one head
-    const uint64_t dims[3] = {D, static_cast<uint64_t>(Hq), static_cast<uint64_t>(total_q)};
-    const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(Hq) * D * 2};
-    const uint32_t box[3] = {64, 1, 128};
-    if ((st = encode_bf16_tiled(&tq, q, 3, dims, strides, box)) != TA_OK) return st;
+  {  // packed queries [total_q, Hq, d] as {64, Hq, total_q, d / 64}: one box of 128 rows of one head
+     // lands as [chunk][128 rows][128 B]
+    const uint64_t dims[4] = {64, static_cast<uint64_t>(Hq), static_cast<uint64_t>(total_q), D / 64};
+    const uint64_t strides[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(Hq) * D * 2, 128};
+    const uint32_t box[4] = {64, 1, 128, D / 64};
+    if ((st = encode_bf16_tiled(&tq, q, 4, dims, strides, box)) != TA_OK) return st;
   }
   {  // pool [P, Hkv, page, d]: boxes of one page of one KV head
     const uint64_t dims[4] = {D, static_cast<uint64_t>(page_size), static_cast<uint64_t>(Hkv),
@@ -912,9 +908,9 @@ ta_status launch_prefill_fp8(const void* q, const void* k, const void* v, float 
   }
   CUtensorMap tq, tk, tv;
   ta_status st;
-  if ((st = encode_u8_rows_3d(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
-  if ((st = encode_u8_rows_3d(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
-  if ((st = encode_u8_rows_3d(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_u8_rows_chunked(&tq, q, D, Nq, B * Hq)) != TA_OK) return st;
+  if ((st = encode_u8_rows_chunked(&tk, k, D, Nkv, B * Hkv)) != TA_OK) return st;
+  if ((st = encode_u8_rows_chunked(&tv, v, D, Nkv, B * Hkv)) != TA_OK) return st;
   static int attr_done[64] = {0};
   cudaError_t e = ensure_smem_limit(prefill_fwd_kernel<D, false, true>, L::kAlloc, attr_done);
   if (e != cudaSuccess) return fail(TA_ERR_CUDA, "fp8 prefill: shared-memory limit", e);

@@ -16,14 +16,15 @@ using PFN_encodeTiled = PFN_cuTensorMapEncodeTiled_v12000;
 // cuTensorMapEncodeTiled fetched through the runtime (no libcuda link).
 PFN_encodeTiled get_encode_tiled();
 
-// Tensor map over a bf16 array [slices, rows, d] (d contiguous) that loads
-// 128-row x 64-column boxes with the 128-byte swizzle; rows past `rows` read
-// as zero.
-ta_status encode_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices);
+// Tensor map over a bf16 array [slices, rows, d] (d contiguous, d = 64 or
+// 128) whose box is a whole tile of 128 rows: 4-D {64, rows, d / 64, slices},
+// coordinates (0, row, 0, slice), landing [64-column chunk][128 rows][128 B]
+// with the 128-byte swizzle; rows past `rows` read as zero.
+ta_status encode_rows_chunked(CUtensorMap* map, const void* base, int d, int rows, int slices);
 
 // The same for a one-byte-per-element array (FP8 codes) [slices, rows, d],
-// d = 128: 128-row x 128-column boxes (one 128-byte swizzle row per row).
-ta_status encode_u8_rows_3d(CUtensorMap* map, const void* base, int d, int rows, int slices);
+// d = 128: {128, rows, 1, slices}, one 128-byte swizzle row per row.
+ta_status encode_u8_rows_chunked(CUtensorMap* map, const void* base, int d, int rows, int slices);
 
 // General bf16 tensor map (rank 2-5, 128-byte swizzle, zero fill out of
 // bounds); strides_bytes has rank - 1 entries.
