@@ -61,12 +61,14 @@ def test_paged_prefill_parity(torch_cuda, q_lens, kv_lens, Hq, Hkv, d, ps, causa
     check(torch_cuda, inp, causal, f"{q_lens} {kv_lens} {Hq}/{Hkv} d{d} p{ps} c={causal}")
 
 
-def test_paged_prefill_equals_dense_bitwise(torch_cuda):
+@pytest.mark.parametrize("ps", [8, 16, 32, 64])
+def test_paged_prefill_equals_dense_bitwise(torch_cuda, ps):
     # one sequence whose pages are in order is the dense prefill of its rows:
-    # the same arithmetic on the same values, so the same bits
+    # the same arithmetic on the same values, so the same bits (at every page
+    # size: each lands its K and V pages in its own shared-memory layout)
     torch = torch_cuda
     from tiled_attention_17_b200 import binding
-    Hq, Hkv, d, ps, n = 4, 2, 128, 16, 700
+    Hq, Hkv, d, n = 4, 2, 128, 700
     inp = paged_prefill_inputs([n], [n], Hq, Hkv, d, ps, seed=5, extra_pages=0)
     npages = (n + ps - 1) // ps
     inp.block_table[0, :npages] = np.arange(npages, dtype=np.int32)   # pages in order
