@@ -325,6 +325,20 @@ ta_status ta_device_status(unsigned *flags, int reset);
  */
 ta_status ta_selftest_bounded_wait(unsigned limit_us, ta_stream_t stream);
 
+/*
+ * Test/diagnostic export: y[i] = 2^x[i] for i < n as computed by the FMA-pipe
+ * exponential that the FP8 prefill uses for part of its softmax weights
+ * (exp((s - m) * scale) with the max subtracted, FlashAttention optimisation
+ * article, online softmax section), in place of the MUFU unit.  x and y are
+ * device fp32 arrays of n elements (4-byte aligned; they may be the same
+ * array); n >= 0, odd n allowed.  Within x >= -125 the maximum relative error is 7.5e-5;
+ * below -125, and for NaN inputs, the result is 2^-125.  Returns
+ * TA_ERR_INVALID_ARG for n < 0 or a null or misaligned pointer with n > 0,
+ * TA_ERR_CUDA if the launch fails.  Asynchronous on `stream`; allocates
+ * nothing.
+ */
+ta_status ta_exp2_poly_debug(const float *x, float *y, int64_t n, ta_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -165,6 +165,14 @@ def test_selftest_validation(lib):
     assert code(lib, lib.ta_selftest_bounded_wait(2_000_000, stream=0)) == "TA_ERR_INVALID_ARG"
 
 
+def test_exp2_poly_debug_validation(lib):
+    # argument checks only: nothing is launched
+    assert code(lib, lib.ta_exp2_poly_debug(256, 256, -1, stream=0, check=False)) == "TA_ERR_INVALID_ARG"
+    assert code(lib, lib.ta_exp2_poly_debug(None, 256, 8, stream=0, check=False)) == "TA_ERR_INVALID_ARG"
+    assert code(lib, lib.ta_exp2_poly_debug(258, 256, 8, stream=0, check=False)) == "TA_ERR_INVALID_ARG"
+    assert code(lib, lib.ta_exp2_poly_debug(None, None, 0, stream=0, check=False)) == "TA_OK"
+
+
 def test_bwd_validation(lib):
     a = 256
     ws = lib.attn_bwd_workspace_size(4, 16, 4096)

@@ -177,3 +177,30 @@ def test_fp8_rising_scores_exact(torch_cuda):
         o, lse = run_fp8(torch_cuda, q8, k8, v8, desc, causal, math.log(2.0))
         o_ref, lse_ref = oracle.attn_fp8(q8, k8, v8, desc, causal, scale=math.log(2.0))
         parity(o, o_ref, lse, lse_ref, f"fp8 rising scores causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_huge_score_gaps(torch_cuda, causal):
+    """Scores far apart: queries hold 448 in one dimension; keys 16t+2 hold 2
+    there, keys 16t and 16t+1 hold -16, the rest 0.  The opposed keys sit about
+    1,000 exp2 units below the row max on the columns whose weights the
+    FMA-pipe exponential computes (below its range of exact results); they must
+    weigh 0, not NaN.  Every weight is 0 or 1 within E4M3 rounding, so the bf16
+    bar applies; |lse| stays below 700, where fp32 holds it to 1e-4."""
+    B, Hq, Hkv, N = 1, 2, 1, 300
+    big, up, down = inputs.f32_to_e4m3_bits(np.array([448.0, 2.0, -16.0], dtype=np.float32))
+    q8 = np.zeros((B, Hq, N, 128), dtype=np.uint8)
+    q8[..., 0] = big
+    k8 = np.zeros((B, Hkv, N, 128), dtype=np.uint8)
+    pos = np.arange(N) % 16
+    k8[0, 0, pos == 2, 0] = up
+    k8[0, 0, (pos == 0) | (pos == 1), 0] = down
+    rng = np.random.Generator(np.random.PCG64(79))
+    v8, dv = inputs.quantize_e4m3(rng.standard_normal(N * 128).astype(np.float32))
+    v8 = v8.reshape(B, Hkv, N, 128)
+    desc = (1.0, 1.0, dv)
+    o, lse = run_fp8(torch_cuda, q8, k8, v8, desc, causal)
+    o_ref, lse_ref = oracle.attn_fp8(q8, k8, v8, desc, causal)
+    assert np.all(np.isfinite(o)), "non-finite output"
+    parity(o, o_ref, lse, lse_ref, f"fp8 huge score gaps causal={causal}")
+

@@ -29,7 +29,7 @@ EXPORTS = ["ta_status_string", "ta_version", "ta_last_error", "attn_fwd", "attn_
            "attn_paged_prefill", "attn_lse_merge", "attn_lse_merge_finish",
            "attn_paged_decode_workspace_size",
            "attn_paged_decode", "attn_paged_decode_noalloc", "attn_paged_decode_check", "attn_paged_gather_debug",
-           "ta_device_status", "ta_selftest_bounded_wait"]
+           "ta_device_status", "ta_selftest_bounded_wait", "ta_exp2_poly_debug"]
 
 
 class TiledAttnError(RuntimeError):
@@ -86,6 +86,8 @@ def load(path: str | None = None):
     L.ta_device_status.restype = i32
     L.ta_selftest_bounded_wait.argtypes = [u32, vp]
     L.ta_selftest_bounded_wait.restype = i32
+    L.ta_exp2_poly_debug.argtypes = [vp, vp, i64, vp]
+    L.ta_exp2_poly_debug.restype = i32
     if path is None:
         _lib = L
     return L
@@ -239,6 +241,13 @@ def ta_device_status(reset: bool = True):
 
 def ta_selftest_bounded_wait(limit_us: int, stream=None) -> int:
     return load().ta_selftest_bounded_wait(int(limit_us), _stream(stream))
+
+
+def ta_exp2_poly_debug(x, y, n: int, stream=None, check: bool = True) -> int:
+    code = load().ta_exp2_poly_debug(_ptr(x), _ptr(y), int(n), _stream(stream))
+    if check:
+        _check("ta_exp2_poly_debug", code)
+    return code
 
 
 # ---------------------------------------------------------------------------

@@ -162,6 +162,18 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 using namespace ta;
 
+// The FMA-pipe exponential of the FP8 softmax, evaluated on its own (the
+// ta_exp2_poly_debug test export): pairs, as the softmax evaluates them.
+__global__ void __launch_bounds__(256) exp2_poly_debug_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                                              long long n) {
+  const long long i = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 2;
+  if (i >= n) return;
+  const bool two = i + 1 < n;
+  const float2 r = exp2_poly2(make_float2(x[i], two ? x[i + 1] : 0.f));
+  y[i] = r.x;
+  if (two) y[i + 1] = r.y;
+}
+
 extern "C" {
 
 const char* ta_status_string(ta_status s) {
@@ -397,6 +409,17 @@ ta_status ta_device_status(unsigned* flags, int reset) {
 ta_status ta_selftest_bounded_wait(unsigned limit_us, ta_stream_t stream) {
   if (limit_us == 0 || limit_us > 1000000u) return TA_ERR_INVALID_ARG;
   return launch_selftest_wait(limit_us, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ta_status ta_exp2_poly_debug(const float* x, float* y, int64_t n, ta_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y)) || (reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u))
+    return TA_ERR_INVALID_ARG;
+  if (n == 0) return TA_OK;
+  const long long pairs = (n + 1) / 2;
+  exp2_poly_debug_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      x, y, static_cast<long long>(n));
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? TA_OK : fail(TA_ERR_CUDA, "ta_exp2_poly_debug: launch", e);
 }
 
 }  // extern "C"

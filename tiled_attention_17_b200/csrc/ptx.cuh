@@ -407,14 +407,16 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // [-0.5, 0.5], and 2^n applied by adding n to the exponent field.  The
 // coefficients were fitted here (iteratively reweighted least squares towards
 // minimax relative error; max relative error 7.5e-5 in fp32, below the bf16
-// rounding that P receives).  Inputs below -127 are clamped (the result is then
-// a denormal near 0, as 2^x is).
+// rounding that P receives).  Inputs are clamped at -125 (NaN reads as -125):
+// below that the result is 2^-125 (2.4e-38), where 2^x would be smaller still.
+// The clamp keeps the exponent field normal.  At -127 (the clamp this had
+// before) n = -127 and p < 1 borrowed into the sign bit and returned NaN.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f, c2 = 0.2426111400127411f,
                   c3 = 0.0551716685295105f;
-  x.x = fmaxf(x.x, -127.f);
-  x.y = fmaxf(x.y, -127.f);
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
   const float2 t = fadd2(x, make_float2(kMagic, kMagic));
   const float2 n = fadd2(t, make_float2(-kMagic, -kMagic));
   const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
