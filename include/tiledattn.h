@@ -136,7 +136,9 @@ ta_status attn_fwd_fp8(const void *q, const void *k, const void *v, float q_desc
  * = 1 it sees keys j <= that position (the bottom-right alignment of
  * attn_fwd), with causal = 0 all keys.  A row with no visible key gets O = 0,
  * lse = -inf.  Supported: d in {64, 128}, page_size in {8, 16, 32, 64},
- * Hq % Hkv == 0.  Out-of-range lengths, offsets and table entries are clamped
+ * Hq % Hkv == 0, num_pages_total * Hkv < 2^31 (else TA_ERR_UNSUPPORTED: the
+ * copies address a (page, KV head) block by one 32-bit coordinate).
+ * Out-of-range lengths, offsets and table entries are clamped
  * on the device (never dereferenced) and flagged in the library status word
  * (ta_device_status).  Allocates nothing.
  */

@@ -218,6 +218,7 @@ def test_paged_prefill_validation(lib):
     assert call(cu=None) == "TA_ERR_INVALID_ARG"
     assert call(lse=a + 2) == "TA_ERR_INVALID_ARG"
     assert call(P=0) == "TA_ERR_INVALID_ARG"
+    assert call(P=2 ** 30, Hkv=2, Hq=4) == "TA_ERR_UNSUPPORTED"   # (page, head) blocks past a 32-bit coordinate
     assert call(S=0) == "TA_OK"
     assert call(T=0) == "TA_OK"
 

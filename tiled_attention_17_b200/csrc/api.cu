@@ -247,6 +247,8 @@ ta_status attn_paged_prefill(const void* q, const void* k_cache, const void* v_c
   if (d != 64 && d != 128) return TA_ERR_UNSUPPORTED;
   if (page_size != 8 && page_size != 16 && page_size != 32 && page_size != 64) return TA_ERR_UNSUPPORTED;
   if (static_cast<long long>(max_pages) * page_size > (1 << 30) || Hq > 65535) return TA_ERR_UNSUPPORTED;
+  // the K copies address a (page, KV head) block by one 32-bit coordinate
+  if (static_cast<long long>(num_pages_total) * Hkv > INT32_MAX) return TA_ERR_UNSUPPORTED;
   if (num_seqs == 0 || total_q == 0 || max_q_len == 0) return TA_OK;
   const long long pairs = (static_cast<long long>(max_q_len) + 255) / 256;
   if (pairs * num_seqs * Hq > INT32_MAX) return TA_ERR_UNSUPPORTED;
