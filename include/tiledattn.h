@@ -137,7 +137,12 @@ ta_status attn_fwd_fp8(const void *q, const void *k, const void *v, float q_desc
  * attn_fwd), with causal = 0 all keys.  A row with no visible key gets O = 0,
  * lse = -inf.  Supported: d in {64, 128}, page_size in {8, 16, 32, 64},
  * Hq % Hkv == 0, num_pages_total * Hkv < 2^31 (else TA_ERR_UNSUPPORTED: the
- * copies address a (page, KV head) block by one 32-bit coordinate).
+ * copies address a (page, KV head) block by one 32-bit coordinate).  Keys
+ * are read a page at a time: the rows of a sequence's last page past its
+ * length, and physical page 0 (read in place of pages past the sequence),
+ * are loaded and given zero weight.  They may hold any finite values, but
+ * not NaN or infinity (0 * inf is NaN): zero a pool allocated uninitialised
+ * once.
  * Out-of-range lengths, offsets and table entries are clamped
  * on the device (never dereferenced) and flagged in the library status word
  * (ta_device_status).  Allocates nothing.

@@ -104,3 +104,25 @@ def test_paged_prefill_serving_mix_sampled(torch_cuda):
     kv_lens = q_lens + rng.integers(0, 8192, size=32, endpoint=True)
     inp = paged_prefill_inputs(q_lens, kv_lens, 32, 8, 128, 16, seed=77)
     check(torch_cuda, inp, True, "serving mix", seqs=[0, int(np.argmax(q_lens)), 31])
+
+
+def test_paged_prefill_page_tails_hold_huge_finite_values(torch_cuda):
+    # Keys are read a page at a time: the rows of a sequence's last page past
+    # its length are loaded and given exactly zero weight (their scores are
+    # masked to -inf before the row max).  Any finite values there, even the
+    # largest bf16 ones, leave the result unchanged.
+    import dataclasses
+    ps = 16
+    inp = paged_prefill_inputs([50, 77, 3], [300, 77, 40], 4, 2, 128, ps, seed=8)
+    k, v = inp.k_cache.copy(), inp.v_cache.copy()
+    big = np.array([0x7F7F, 0xFF7F], dtype=np.uint16)   # +-3.39e38, the largest finite bf16
+    for sq, n in enumerate(inp.seq_lens):
+        if n % ps:
+            page = inp.block_table[sq, n // ps]
+            tail = np.resize(big, k[page, :, n % ps:, :].shape)
+            k[page, :, n % ps:, :] = tail
+            v[page, :, n % ps:, :] = tail[..., ::-1]
+    huge = dataclasses.replace(inp, k_cache=k, v_cache=v)
+    for causal in (True, False):
+        check(torch_cuda, huge, causal, f"huge finite page tails causal={causal}")
+
